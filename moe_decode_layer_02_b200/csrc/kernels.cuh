@@ -1,0 +1,70 @@
+// Kernel arguments and host launchers of the MoE decode layer (internal).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+enum Counter { kCntOproj = 0, kCntRouter = 1, kCntGateUp = 2, kNumCounters = 4 };
+
+// Library-owned device workspace (one per handle).
+struct Workspace {
+  float* h;          // [maxB][d]   residual + o_proj, fp32
+  float* x;          // [maxB][d]   RMSNorm output, fp32
+  float* rstd;       // [maxB]
+  float* ss_part;    // [G][maxB]   per-CTA sums of h^2
+  float* logits;     // [maxB][E]   fp32
+  int* topk_idx;     // [maxB][k]
+  float* topk_gate;  // [maxB][k]
+  int* n_union;      // [1]         number of distinct selected experts U
+  int* union_e;      // [E]         selected experts, ascending
+  int* union_off;    // [E+1]       CSR offsets of each union expert's token entries
+  int* entry_tok;    // [maxB*k]    token of each entry (ascending within an expert)
+  int* entry_slot;   // [maxB*k]    slot j of that token's top-k list
+  float* a;          // [maxB*k][I] SwiGLU activations per entry
+  float* gu_part;    // split-K partials [maxB*k][n_split][2I]
+  unsigned* gu_tick; // [E]         split-K per-union-expert tickets
+  unsigned* counters;  // [kNumCounters]
+  unsigned* err;       // error word (kErrTimeout | kErrBounds)
+};
+
+struct KTune {
+  int stages = 0;          // ring stages
+  int rows_per_stage = 0;  // weight rows (or row pairs) per stage
+  int rows_max = 0;        // max rows owned by one CTA
+  int n_split = 0;         // split-K factor (gate/up large-batch variant)
+  size_t smem = 0;         // dynamic shared memory bytes
+};
+
+struct LayerArgs {
+  int B, maxB, d, d_o, E, k, I;
+  float eps;
+  const uint16_t *w_o, *gamma, *w_r, *w_gu, *w_down;  // this layer's weights
+  const uint16_t* attn;   // [B][d_o]
+  const uint16_t* resid;  // [B][d]
+  uint16_t* out;          // [B][d]
+  int* user_idx;          // [B][k] or null
+  float* user_gate;       // [B][k] or null
+  Workspace ws;
+  KTune k1, k2, k3, k4;
+};
+
+struct PrefetchArgs {
+  const void* ptr[4];
+  unsigned long long bytes[4];
+  int n;
+};
+
+// Host-side planning (sets the KTune fields, returns false if unsupported).
+bool plan_layer(LayerArgs& a, int num_sms, size_t smem_optin);
+
+// Launchers (pdl: launch with programmatic stream serialisation).
+cudaError_t launch_oproj(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_router(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_gateup_small(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_gateup_splitk(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_down(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_prefetch(const PrefetchArgs& p, int grid, cudaStream_t s);
+cudaError_t set_kernel_attributes(size_t smem_optin);
+
+}  // namespace moe

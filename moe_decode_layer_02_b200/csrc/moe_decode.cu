@@ -1,0 +1,559 @@
+// C ABI of the MoE decode-layer library: handle life cycle, workspace, CUDA-graph
+// capture of the per-layer kernel chain, and the host-buffer variant of the step.
+//
+// A step of n_layers layers is captured once per (batch, buffer addresses) into one
+// CUDA graph: per layer K1 o_proj+residual+RMS stats -> K2 router+top-k+routing ->
+// K3 expert gate/up (small-M or split-K by batch) -> K4 down+combine, chained with
+// programmatic dependent launch so each kernel's CTAs start (and fetch their static
+// weights) while the previous kernel drains.  With prefetch on, a forked side stream
+// prefetches layer l+1's router, RMSNorm scale and the head of its W_o into L2 once
+// layer l's router is done; it joins the main stream at the end of the graph.
+//
+// Sources: "vLLM speeds up Kimi K3 up to 1.9x on NVIDIA GB300 with agent-assisted
+// kernels", section "How the specialised decode path works" (kernel choice by batch
+// size; next-layer weight prefetch on a side kernel); "vLLM and NVIDIA use coding agents
+// to nearly double Kimi K3 decode speed, then rethink how to review it" (fewer kernels
+// per layer); "vLLM tests a fast-track review model with Kimi K3's specialized decode
+// path", section "Why the review model matters" (reject unsupported configurations at
+// startup).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <unordered_set>
+#include <vector>
+
+#include "../../include/moe_decode.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+struct GraphEntry {
+  int batch;
+  const void *attn, *resid, *out, *idx, *gate;
+  cudaGraphExec_t exec;
+  int kernels;
+};
+
+constexpr size_t kPrefetchWoHead = 24ull << 20;  // bytes of the next W_o prefetched into L2
+constexpr int kGraphCacheMax = 16;
+
+}  // namespace
+
+struct moe_decode_handle {
+  moe_decode_config cfg;
+  std::vector<moe_decode_layer_weights> w;
+  int device = 0, num_sms = 0;
+  size_t smem_optin = 0;
+  int n_split = 0;  // split-K factor, 0 if the shape has none
+  Workspace ws{};
+  void* ws_base = nullptr;
+  uint16_t* resid_pp[2] = {nullptr, nullptr};
+  // staging for moe_decode_step_host
+  void *h_attn = nullptr, *h_resid = nullptr, *h_out = nullptr, *h_idx = nullptr, *h_gate = nullptr;
+  LayerArgs plan_small{}, plan_splitk{};
+  bool has_splitk = false;
+  cudaStream_t cap = nullptr, side = nullptr;
+  std::vector<cudaEvent_t> events;
+  std::vector<GraphEntry> graphs;
+  int last_batch = 0;
+  bool poisoned = false;
+};
+
+namespace {
+
+// Live handles: destroy and step reject pointers that are not (or no longer) handles.
+std::mutex g_live_mu;
+std::unordered_set<const moe_decode_handle*> g_live;
+
+bool is_live(const moe_decode_handle* h) {
+  std::lock_guard<std::mutex> lk(g_live_mu);
+  return g_live.count(h) != 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const moe_decode_config* c) {
+  if (c->d < 64 || c->d > 8192 || c->d % 64) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->d_o < 64 || c->d_o > 8192 || c->d_o % 64) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->top_k < 1 || c->top_k > 32) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->n_experts < c->top_k || c->n_experts > 1024) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->inter < 32 || c->inter > 512 || c->inter % 32) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->max_batch < 1 || c->max_batch > 64) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->n_layers < 1 || c->n_layers > 64) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (!(c->rms_eps > 0.f)) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->force_variant < 0 || c->force_variant > 2) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int pick_split(int d) {
+  for (int ns = 1; ns <= d / 256; ++ns)
+    if (d % ns == 0 && (d / ns) % 256 == 0 && d / ns <= 1024) return ns;
+  return 0;
+}
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+void release(moe_decode_handle* h) {
+  for (auto& g : h->graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  h->graphs.clear();
+  for (auto e : h->events) cudaEventDestroy(e);
+  h->events.clear();
+  if (h->cap) cudaStreamDestroy(h->cap);
+  if (h->side) cudaStreamDestroy(h->side);
+  if (h->ws_base) cudaFree(h->ws_base);
+  h->cap = h->side = nullptr;
+  h->ws_base = nullptr;
+}
+
+bool use_splitk(const moe_decode_handle* h, int B) {
+  if (!h->has_splitk) return false;
+  if (h->cfg.force_variant == 1) return false;
+  if (h->cfg.force_variant == 2) return true;
+  return B >= 3;  // small-matrix kernels at batch one or two, split-K above
+}
+
+LayerArgs layer_args(const moe_decode_handle* h, int l, int B, const void* attn, const void* resid,
+                     void* out, int32_t* idx, float* gate) {
+  const moe_decode_config& c = h->cfg;
+  LayerArgs a = use_splitk(h, B) ? h->plan_splitk : h->plan_small;
+  a.B = B;
+  a.w_o = static_cast<const uint16_t*>(h->w[l].w_o);
+  a.gamma = static_cast<const uint16_t*>(h->w[l].gamma);
+  a.w_r = static_cast<const uint16_t*>(h->w[l].w_router);
+  a.w_gu = static_cast<const uint16_t*>(h->w[l].w_gate_up);
+  a.w_down = static_cast<const uint16_t*>(h->w[l].w_down);
+  a.attn = static_cast<const uint16_t*>(attn) + (size_t)l * B * c.d_o;
+  a.resid = (l == 0) ? static_cast<const uint16_t*>(resid) : h->resid_pp[(l - 1) & 1];
+  a.out = (l == c.n_layers - 1) ? static_cast<uint16_t*>(out) : h->resid_pp[l & 1];
+  a.user_idx = idx ? idx + (size_t)l * B * c.top_k : nullptr;
+  a.user_gate = gate ? gate + (size_t)l * B * c.top_k : nullptr;
+  return a;
+}
+
+// Records the whole step on h->cap (which is in capture mode).  Returns kernels launched.
+int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid, void* out,
+                int32_t* idx, float* gate, cudaError_t* err) {
+  const moe_decode_config& c = h->cfg;
+  const int G = h->num_sms;
+  const bool prefetch = c.enable_prefetch && c.n_layers > 1;
+  int kernels = 0, ev = 0;
+  cudaError_t e = cudaSuccess;
+  bool forked = false;
+  for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
+    LayerArgs a = layer_args(h, l, B, attn, resid, out, idx, gate);
+    e = launch_oproj(a, G, h->cap, l > 0);
+    if (e == cudaSuccess) e = launch_router(a, G, h->cap, true);
+    kernels += 2;
+    if (e == cudaSuccess && prefetch && l + 1 < c.n_layers) {
+      // Fork: once this layer's router is done, warm L2 with the next layer's
+      // router slice, RMSNorm scale and the head of its W_o.
+      e = cudaEventRecord(h->events[ev], h->cap);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->events[ev++], 0);
+      PrefetchArgs p{};
+      const moe_decode_layer_weights& nw = h->w[l + 1];
+      p.ptr[0] = nw.w_router;
+      p.bytes[0] = (unsigned long long)c.n_experts * c.d * 2;
+      p.ptr[1] = nw.gamma;
+      p.bytes[1] = (unsigned long long)c.d * 2;
+      p.ptr[2] = nw.w_o;
+      p.bytes[2] = std::min<unsigned long long>(kPrefetchWoHead, (unsigned long long)c.d * c.d_o * 2);
+      p.n = 3;
+      if (e == cudaSuccess) e = launch_prefetch(p, G, h->side);
+      ++kernels;
+      forked = true;
+    }
+    if (e == cudaSuccess)
+      e = use_splitk(h, B) ? launch_gateup_splitk(a, G, h->cap, true) : launch_gateup_small(a, G, h->cap, true);
+    if (e == cudaSuccess) e = launch_down(a, G, h->cap, true);
+    kernels += 2;
+  }
+  if (e == cudaSuccess && forked) {
+    e = cudaEventRecord(h->events[ev], h->side);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->cap, h->events[ev++], 0);
+  }
+  *err = e;
+  return kernels;
+}
+
+int get_graph(moe_decode_handle* h, int B, const void* attn, const void* resid, void* out,
+              int32_t* idx, float* gate, GraphEntry** ge) {
+  for (auto& g : h->graphs)
+    if (g.batch == B && g.attn == attn && g.resid == resid && g.out == out && g.idx == idx && g.gate == gate) {
+      *ge = &g;
+      return MOE_OK;
+    }
+  if ((int)h->graphs.size() >= kGraphCacheMax) {
+    cudaGraphExecDestroy(h->graphs.front().exec);
+    h->graphs.erase(h->graphs.begin());
+  }
+  cudaGraph_t graph = nullptr;
+  if (cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t rec = cudaSuccess;
+  const int kernels = record_step(h, B, attn, resid, out, idx, gate, &rec);
+  const cudaError_t end = cudaStreamEndCapture(h->cap, &graph);
+  if (rec != cudaSuccess || end != cudaSuccess || !graph) {
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t inst = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (inst != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  h->graphs.push_back(GraphEntry{B, attn, resid, out, idx, gate, exec, kernels});
+  *ge = &h->graphs.back();
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weights* weights, void* stream,
+                      moe_decode_handle** out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg || !weights) return MOE_ERR_INVALID_ARG;
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const moe_decode_layer_weights& w = weights[l];
+    if (!w.w_o || !w.gamma || !w.w_router || !w.w_gate_up || !w.w_down) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w.w_o) || !aligned16(w.gamma) || !aligned16(w.w_router) || !aligned16(w.w_gate_up) ||
+        !aligned16(w.w_down))
+      return MOE_ERR_ALIGNMENT;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (prop.major != 10 || prop.minor != 0) return MOE_ERR_UNSUPPORTED_CONFIG;  // sm_100 only
+
+  moe_decode_handle* h = new (std::nothrow) moe_decode_handle();
+  if (!h) return MOE_ERR_OOM;
+  h->cfg = *cfg;
+  h->w.assign(weights, weights + cfg->n_layers);
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  h->smem_optin = prop.sharedMemPerBlockOptin;
+  const int G = h->num_sms, maxB = cfg->max_batch, d = cfg->d, E = cfg->n_experts, K = cfg->top_k,
+            I = cfg->inter;
+  if ((long long)G * kConsumerThreads < d) {
+    delete h;
+    return MOE_ERR_UNSUPPORTED_CONFIG;
+  }
+  h->n_split = pick_split(d);
+
+  // ---- plans ---------------------------------------------------------------------------
+  LayerArgs base{};
+  base.maxB = maxB;
+  base.d = d;
+  base.d_o = cfg->d_o;
+  base.E = E;
+  base.k = K;
+  base.I = I;
+  base.eps = cfg->rms_eps;
+  h->plan_small = base;
+  h->plan_small.k3.n_split = 0;
+  if (!plan_layer(h->plan_small, G, h->smem_optin)) {
+    delete h;
+    return MOE_ERR_UNSUPPORTED_CONFIG;
+  }
+  if (h->n_split > 0) {
+    h->plan_splitk = base;
+    h->plan_splitk.k3.n_split = h->n_split;
+    h->has_splitk = plan_layer(h->plan_splitk, G, h->smem_optin);
+  }
+  if (cfg->force_variant == 2 && !h->has_splitk) {
+    delete h;
+    return MOE_ERR_UNSUPPORTED_CONFIG;
+  }
+
+  // ---- workspace -----------------------------------------------------------------------
+  const int NS = std::max(h->n_split, 1);
+  const size_t entries = (size_t)maxB * K;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += up256(bytes);
+    return o;
+  };
+  const size_t o_h = take(sizeof(float) * maxB * d), o_x = take(sizeof(float) * maxB * d),
+               o_rstd = take(sizeof(float) * maxB), o_ss = take(sizeof(float) * G * maxB),
+               o_lg = take(sizeof(float) * maxB * E), o_ti = take(sizeof(int) * entries),
+               o_tg = take(sizeof(float) * entries), o_nu = take(sizeof(int)), o_ue = take(sizeof(int) * E),
+               o_uo = take(sizeof(int) * (E + 1)), o_et = take(sizeof(int) * entries),
+               o_es = take(sizeof(int) * entries), o_a = take(sizeof(float) * entries * I),
+               o_gp = take(h->has_splitk ? sizeof(float) * entries * NS * 2 * I : 16),
+               o_gt = take(sizeof(unsigned) * E), o_cnt = take(sizeof(unsigned) * kNumCounters),
+               o_err = take(sizeof(unsigned)), o_r0 = take(2ull * maxB * d), o_r1 = take(2ull * maxB * d);
+  if (cudaMalloc(&h->ws_base, off) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return MOE_ERR_OOM;
+  }
+  char* b = static_cast<char*>(h->ws_base);
+  Workspace& ws = h->ws;
+  ws.h = (float*)(b + o_h);
+  ws.x = (float*)(b + o_x);
+  ws.rstd = (float*)(b + o_rstd);
+  ws.ss_part = (float*)(b + o_ss);
+  ws.logits = (float*)(b + o_lg);
+  ws.topk_idx = (int*)(b + o_ti);
+  ws.topk_gate = (float*)(b + o_tg);
+  ws.n_union = (int*)(b + o_nu);
+  ws.union_e = (int*)(b + o_ue);
+  ws.union_off = (int*)(b + o_uo);
+  ws.entry_tok = (int*)(b + o_et);
+  ws.entry_slot = (int*)(b + o_es);
+  ws.a = (float*)(b + o_a);
+  ws.gu_part = (float*)(b + o_gp);
+  ws.gu_tick = (unsigned*)(b + o_gt);
+  ws.counters = (unsigned*)(b + o_cnt);
+  ws.err = (unsigned*)(b + o_err);
+  h->resid_pp[0] = (uint16_t*)(b + o_r0);
+  h->resid_pp[1] = (uint16_t*)(b + o_r1);
+  h->plan_small.ws = ws;
+  h->plan_splitk.ws = ws;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(h->ws_base, 0, off, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = set_kernel_attributes(h->smem_optin);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
+  for (int i = 0; i < 2 * cfg->n_layers + 2 && e == cudaSuccess; ++i) {
+    cudaEvent_t ev;
+    e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (e == cudaSuccess) h->events.push_back(ev);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    release(h);
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    g_live.insert(h);
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+int moe_decode_step(moe_decode_handle* h, int batch, const void* attn_out, const void* residual_in, void* out,
+                    int32_t* topk_idx, float* topk_gate, void* stream) {
+  if (!h || !is_live(h) || h->poisoned) return MOE_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MOE_ERR_INVALID_ARG;
+  if (!attn_out || !residual_in || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(attn_out) || !aligned16(residual_in) || !aligned16(out) || (topk_idx && !aligned16(topk_idx)) ||
+      (topk_gate && !aligned16(topk_gate)))
+    return MOE_ERR_ALIGNMENT;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MOE_ERR_INVALID_ARG;
+  GraphEntry* ge = nullptr;
+  int rc = get_graph(h, batch, attn_out, residual_in, out, topk_idx, topk_gate, &ge);
+  if (rc) return rc;
+  if (cudaGraphLaunch(ge->exec, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  h->last_batch = batch;
+  return MOE_OK;
+}
+
+int moe_decode_step_host(moe_decode_handle* h, int batch, const void* attn_out_host, const void* residual_in_host,
+                         void* out_host, int32_t* topk_idx_host, float* topk_gate_host, void* stream) {
+  if (!h || !is_live(h) || h->poisoned) return MOE_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch) return MOE_ERR_INVALID_ARG;
+  if (!attn_out_host || !residual_in_host || !out_host) return MOE_ERR_INVALID_ARG;
+  const moe_decode_config& c = h->cfg;
+  const size_t maxB = c.max_batch;
+  if (!h->h_attn) {
+    size_t sz = up256(2ull * c.n_layers * maxB * c.d_o) + 2 * up256(2ull * maxB * c.d) +
+                2 * up256(4ull * c.n_layers * maxB * c.top_k);
+    void* p = nullptr;
+    if (cudaMalloc(&p, sz) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_OOM;
+    }
+    char* b = static_cast<char*>(p);
+    h->h_attn = b;
+    b += up256(2ull * c.n_layers * maxB * c.d_o);
+    h->h_resid = b;
+    b += up256(2ull * maxB * c.d);
+    h->h_out = b;
+    b += up256(2ull * maxB * c.d);
+    h->h_idx = b;
+    b += up256(4ull * c.n_layers * maxB * c.top_k);
+    h->h_gate = b;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t n_attn = 2ull * c.n_layers * batch * c.d_o, n_res = 2ull * batch * c.d,
+               n_tk = 4ull * c.n_layers * batch * c.top_k;
+  cudaError_t e = cudaMemcpyAsync(h->h_attn, attn_out_host, n_attn, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h->h_resid, residual_in_host, n_res, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  int rc = moe_decode_step(h, batch, h->h_attn, h->h_resid, h->h_out, topk_idx_host ? (int32_t*)h->h_idx : nullptr,
+                           topk_gate_host ? (float*)h->h_gate : nullptr, stream);
+  if (rc) return rc;
+  e = cudaMemcpyAsync(out_host, h->h_out, n_res, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && topk_idx_host) e = cudaMemcpyAsync(topk_idx_host, h->h_idx, n_tk, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && topk_gate_host)
+    e = cudaMemcpyAsync(topk_gate_host, h->h_gate, n_tk, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+int moe_decode_sync_status(moe_decode_handle* h, void* stream) {
+  if (!h || !is_live(h)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  unsigned word = 0;
+  if (cudaMemcpy(&word, h->ws.err, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  if (word) {
+    cudaMemset(h->ws.err, 0, sizeof word);
+    cudaDeviceSynchronize();
+    return (word & kErrTimeout) ? MOE_ERR_DEVICE_TIMEOUT : MOE_ERR_DEVICE_BOUNDS;
+  }
+  return MOE_OK;
+}
+
+int moe_decode_get_intermediate(moe_decode_handle* h, int which, void* dst, size_t bytes, void* stream) {
+  if (!h || !is_live(h) || !dst || h->last_batch < 1) return MOE_ERR_INVALID_ARG;
+  const int B = h->last_batch;
+  const void* src = nullptr;
+  size_t size = 0;
+  switch (which) {
+    case 0: src = h->ws.h; size = 4ull * B * h->cfg.d; break;
+    case 1: src = h->ws.rstd; size = 4ull * B; break;
+    case 2: src = h->ws.x; size = 4ull * B * h->cfg.d; break;
+    case 3: src = h->ws.logits; size = 4ull * B * h->cfg.n_experts; break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  if (cudaMemcpyAsync(dst, src, std::min(bytes, size), cudaMemcpyDeviceToDevice,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+int moe_decode_kernels_per_step(moe_decode_handle* h, int batch) {
+  if (!h || !is_live(h) || batch < 1 || batch > h->cfg.max_batch) return MOE_ERR_INVALID_ARG;
+  const int L = h->cfg.n_layers;
+  return 4 * L + ((h->cfg.enable_prefetch && L > 1) ? L - 1 : 0);
+}
+
+int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_out, const void* residual_in,
+                            void* out, int32_t* topk_idx, float* topk_gate, void* stream, float* kernel_ms,
+                            int* kernel_id, int max_kernels) {
+  if (!h || !is_live(h) || h->poisoned || !kernel_ms || max_kernels < 1) return MOE_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch || !attn_out || !residual_in || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(attn_out) || !aligned16(residual_in) || !aligned16(out) || (topk_idx && !aligned16(topk_idx)) ||
+      (topk_gate && !aligned16(topk_gate)))
+    return MOE_ERR_ALIGNMENT;
+  const moe_decode_config& c = h->cfg;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int G = h->num_sms;
+  const int n = std::min(max_kernels, moe_decode_kernels_per_step(h, batch));
+  std::vector<cudaEvent_t> ev(2 * n, nullptr);
+  cudaError_t e = cudaSuccess;
+  for (auto& x : ev)
+    if (e == cudaSuccess) e = cudaEventCreate(&x);
+  int k = 0;
+  auto timed = [&](int id, cudaStream_t st, auto&& fn) {
+    if (e != cudaSuccess || k >= n) return;
+    e = cudaEventRecord(ev[2 * k], st);
+    if (e == cudaSuccess) e = fn(st);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[2 * k + 1], st);
+    if (kernel_id) kernel_id[k] = id;
+    ++k;
+  };
+  for (int l = 0; l < c.n_layers; ++l) {
+    LayerArgs a = layer_args(h, l, batch, attn_out, residual_in, out, topk_idx, topk_gate);
+    timed(1, s, [&](cudaStream_t st) { return launch_oproj(a, G, st, false); });
+    timed(2, s, [&](cudaStream_t st) { return launch_router(a, G, st, false); });
+    if (c.enable_prefetch && c.n_layers > 1 && l + 1 < c.n_layers) {
+      PrefetchArgs p{};
+      const moe_decode_layer_weights& nw = h->w[l + 1];
+      p.ptr[0] = nw.w_router;
+      p.bytes[0] = (unsigned long long)c.n_experts * c.d * 2;
+      p.ptr[1] = nw.gamma;
+      p.bytes[1] = (unsigned long long)c.d * 2;
+      p.ptr[2] = nw.w_o;
+      p.bytes[2] = std::min<unsigned long long>(kPrefetchWoHead, (unsigned long long)c.d * c.d_o * 2);
+      p.n = 3;
+      timed(6, s, [&](cudaStream_t st) { return launch_prefetch(p, G, st); });
+    }
+    const bool sk = use_splitk(h, batch);
+    timed(sk ? 4 : 3, s, [&](cudaStream_t st) {
+      return sk ? launch_gateup_splitk(a, G, st, false) : launch_gateup_small(a, G, st, false);
+    });
+    timed(5, s, [&](cudaStream_t st) { return launch_down(a, G, st, false); });
+  }
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  for (int i = 0; i < k && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&kernel_ms[i], ev[2 * i], ev[2 * i + 1]);
+  for (auto& x : ev)
+    if (x) cudaEventDestroy(x);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  h->last_batch = batch;
+  return k;
+}
+
+int moe_decode_destroy(moe_decode_handle* h) {
+  if (!h) return MOE_OK;
+  {
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    if (!g_live.erase(h)) return MOE_ERR_INVALID_ARG;  // not a live handle (e.g. destroyed twice)
+  }
+  cudaDeviceSynchronize();
+  release(h);
+  if (h->h_attn) cudaFree(h->h_attn);
+  h->poisoned = true;
+  delete h;
+  return MOE_OK;
+}
+
+const char* moe_decode_strerror(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_CONFIG: return "unsupported configuration";
+    case MOE_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case MOE_ERR_OOM: return "out of device memory";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_BOUNDS: return "device index out of range";
+    default: return "unknown error";
+  }
+}
+
+}  // extern "C"

@@ -63,21 +63,31 @@ def token_resid(seed, dims, b, attempt):
 
 
 def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=None,
-               min_gap: float = 1e-3, max_attempts: int = 200, resid0=None, refs=None) -> dict:
+               min_gap: float = 1e-3, max_attempts: int = 200, resid0=None, attn0=None,
+               refs=None, moe_tokens=None) -> dict:
     """Seeded inputs for a B-token, n_layers-deep step and the oracle's answers.
 
     ``checked`` lists the tokens the oracle follows through every layer (all
     of them by default); those tokens satisfy the gap rule at every layer.
     Unchecked tokens keep attempt 0.  ``resid0`` ([B][d] bf16 bits) replaces
-    the drawn layer-0 residual (used by constructed batch-2 cases).
+    the drawn layer-0 residual and ``attn0`` ([B][d_o]) the drawn layer-0 attention
+    output (used by constructed batch-2 cases); fixed inputs are never redrawn.
+    ``moe_tokens`` (one-layer cases only) limits the expert half of the oracle to a
+    subset of the checked tokens; the others get indices and gates only.
 
     Returns attn [L][B][d_o] and resid [B][d] (bf16 bits), the attempts used,
     and per layer the oracle's front results and outputs for checked tokens.
     """
     checked = list(range(B)) if checked is None else list(checked)
+    if moe_tokens is not None and n_layers != 1:
+        raise ValueError("moe_tokens needs a one-layer case")
+    moe_set = set(checked if moe_tokens is None else moe_tokens)
     refs = refs or [LayerRef(seed, dims, l) for l in range(n_layers)]
     attn = np.stack([np.stack([token_attn(seed, dims, l, b, 0) for b in range(B)])
                      for l in range(n_layers)])
+    fixed0 = resid0 is not None or attn0 is not None
+    if attn0 is not None:
+        attn[0] = np.array(attn0, np.uint16).reshape(B, dims.d_o)
     if resid0 is None:
         resid = np.stack([token_resid(seed, dims, b, 0) for b in range(B)])
     else:
@@ -93,22 +103,23 @@ def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=N
             for att in range(max_attempts):
                 if att:
                     attn[l, b] = token_attn(seed, dims, l, b, att)
-                    if l == 0 and resid0 is None:
+                    if l == 0:
                         cur[b] = token_resid(seed, dims, b, att)
                         resid[b] = cur[b]
                 f = ref.front(attn[l, b][None], cur[b][None])
                 if top_gap(f["logits64"][0], dims.k) >= min_gap:
                     break
-                if resid0 is not None and l == 0:
-                    raise RuntimeError("constructed residual violates the gap rule")
+                if fixed0 and l == 0:
+                    raise RuntimeError("fixed layer-0 inputs violate the gap rule")
             else:
                 raise RuntimeError(f"no gapped draw for token {b} layer {l}")
             attempts[l, b] = att
-            out_ref, out_bf16, a = ref.moe(f, 0)
             for key in ("idx", "gate", "h", "x", "logits32", "logits64", "rstd"):
                 per[key][b] = f[key][0]
-            per["out_ref"][b], per["out_bf16"][b], per["a"][b] = out_ref, out_bf16, a
-            cur[b] = out_bf16
+            if b in moe_set:
+                out_ref, out_bf16, a = ref.moe(f, 0)
+                per["out_ref"][b], per["out_bf16"][b], per["a"][b] = out_ref, out_bf16, a
+                cur[b] = out_bf16
         layers.append(per)
     return {"attn": attn, "resid": resid, "attempts": attempts, "layers": layers,
             "checked": checked, "refs": refs}

@@ -1,0 +1,144 @@
+"""Shared helpers of the parity tests: seeded device weights, oracle cases, tolerances.
+
+Tolerances (floating point), from the layer's stated acceptance bar:
+  * selected expert indices and their order: exact;
+  * bf16 output, per element: |gpu - ref| <= 2e-2 + ulp_bf16(ref) / 2, where ref is
+    the oracle's fp64 value before rounding (a perfectly rounded bf16 output can be
+    half an ulp away, and half an ulp exceeds 2e-2 once |ref| >= 8);
+  * bf16 output, relative L2: ||gpu - ref|| / ||ref|| <= 5e-3;
+  * in a stack, each earlier layer boundary adds one bf16 ulp of that layer's output
+    per element (the two chains round independently; a different rounding is
+    carried unchanged by the residual path), and gates of layers after the first
+    are compared within GATE_ATOL_STACKED.
+Intermediates are checked more tightly than the output (fp32 vs fp64 arithmetic).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+from oracle.layer import LayerRef, build_case, token_attn, top_gap
+
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+GATE_ATOL = 2e-6
+# Later layers of a stack see inputs that carry the two chains' independent bf16
+# roundings (a few elements one ulp apart); that moves their logits by ~1e-4 at most
+# and the gates (d gate / d logit <= 1/4) by less than 1e-4.
+GATE_ATOL_STACKED = 1e-4
+
+
+def ulp_bf16(v: np.ndarray) -> np.ndarray:
+    a = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.ldexp(1.0, (e - 7).astype(np.int64))
+
+
+def check_out(gpu_bits: np.ndarray, ref: np.ndarray, extra_tol: np.ndarray | float = 0.0) -> dict:
+    g = synth.bf16_bits_to_f32(gpu_bits).astype(np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(g - ref)
+    tol = MAX_ABS + 0.5 * ulp_bf16(ref) + extra_tol
+    rel = float(np.linalg.norm(g - ref) / np.linalg.norm(ref))
+    res = {"max_abs": float(err.max()), "worst_excess": float((err - tol).max()), "rel_l2": rel,
+           "n_bad": int((err > tol).sum())}
+    assert res["n_bad"] == 0, res
+    assert rel <= REL_L2, res
+    return res
+
+
+# --- device side -------------------------------------------------------------------------
+def device_weights(seed: int, dims: synth.Dims, n_layers: int, device="cuda"):
+    import torch
+    sz = dims.sizes()
+    layers = []
+    for l in range(n_layers):
+        t = {}
+        for kind in (synth.W_O, synth.GAMMA, synth.W_R, synth.W_GU, synth.W_DOWN):
+            x = torch.empty(sz[kind], dtype=torch.bfloat16, device=device)
+            synth.device_fill(x, seed, kind, layer=l)
+            t[kind] = x
+        layers.append((t[synth.W_O], t[synth.GAMMA], t[synth.W_R], t[synth.W_GU], t[synth.W_DOWN]))
+    torch.cuda.synchronize()
+    return layers
+
+
+class GpuStack:
+    """A handle over seeded device weights, plus a step with numpy in/out."""
+
+    def __init__(self, seed, dims, n_layers=1, max_batch=1, prefetch=0, force_variant=0, weights=None):
+        import torch
+        import moe_decode_layer_02_b200 as md
+        self.md, self.torch = md, torch
+        self.dims, self.L, self.maxB = dims, n_layers, max_batch
+        self.weights = weights or device_weights(seed, dims, n_layers)
+        cfg = md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, max_batch, n_layers,
+                        enable_prefetch=prefetch, force_variant=force_variant)
+        self.h = md.moe_decode_create(cfg, self.weights, torch.cuda.current_stream())
+
+    def step(self, attn_bits: np.ndarray, resid_bits: np.ndarray, reps: int = 1):
+        torch, md, D = self.torch, self.md, self.dims
+        L, B = attn_bits.shape[0], attn_bits.shape[1]
+        dev = "cuda"
+        attn = torch.from_numpy(attn_bits.view(np.int16).copy()).to(dev).view(torch.bfloat16)
+        resid = torch.from_numpy(resid_bits.view(np.int16).copy()).to(dev).view(torch.bfloat16)
+        out = torch.empty((B, D.d), dtype=torch.bfloat16, device=dev)
+        idx = torch.full((L, B, D.k), -1, dtype=torch.int32, device=dev)
+        gate = torch.full((L, B, D.k), -1.0, dtype=torch.float32, device=dev)
+        s = torch.cuda.current_stream()
+        for _ in range(reps):
+            md.moe_decode_step(self.h, B, attn, resid, out, idx, gate, s)
+        rc = md.moe_decode_sync_status(self.h, s)
+        assert rc == 0, md.strerror(rc)
+        return (out.view(torch.int16).cpu().numpy().view(np.uint16), idx.cpu().numpy(), gate.cpu().numpy())
+
+    def intermediate(self, which: int, B: int):
+        torch, D = self.torch, self.dims
+        n = {0: B * D.d, 1: B, 2: B * D.d, 3: B * D.E}[which]
+        buf = torch.empty(n, dtype=torch.float32, device="cuda")
+        self.md.moe_decode_get_intermediate(self.h, which, buf, n * 4, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        return buf.cpu().numpy()
+
+    def close(self):
+        if self.h:
+            self.md.moe_decode_destroy(self.h)
+            self.h = 0
+
+
+# --- constructed batch-2 overlaps ---------------------------------------------------------------
+def constructed_b2(seed: int, dims: synth.Dims, overlap: int, lift: float = 15.0, ref: LayerRef | None = None):
+    """Batch-2 inputs whose two top-k sets share exactly `overlap` experts.
+
+    Token b's normalised activation is steered towards a chosen set S_b:
+    x* = z + lift * sum_{e in S_b} W_r[e] / |W_r[e]|^2 with z ~ N(0, 1) from the seeded
+    generator, h* = x* / gamma, and residual_in = bf16(h* - W_o . attn_out).  The oracle
+    then confirms top-k(x) = S_b and the gap rule; otherwise z is redrawn.
+    """
+    from oracle import get as get_oracle
+    o = get_oracle()
+    ref = ref or LayerRef(seed, dims, 0)
+    E, k, d = dims.E, dims.k, dims.d
+    rng = np.random.default_rng(seed * 1000 + overlap)
+    S0 = rng.choice(E, k, replace=False)
+    rest = np.setdiff1d(np.arange(E), S0)
+    S1 = np.concatenate([S0[:overlap], rng.choice(rest, k - overlap, replace=False)])
+    Wr = synth.bf16_bits_to_f32(ref.W_r).astype(np.float64).reshape(E, d)
+    gam = synth.bf16_bits_to_f32(ref.gamma).astype(np.float64)
+    attn0, resid0 = [], []
+    for b, S in enumerate((S0, S1)):
+        for att in range(50):
+            attn = token_attn(seed, dims, 0, b, att)
+            z = synth.bf16_bits_to_f32(synth.host_token(seed, synth.LIFT_Z, d, token=b, attempt=att)).astype(np.float64)
+            xs = z + lift * (Wr[S] / (Wr[S] ** 2).sum(1, keepdims=True)).sum(0)
+            hs = xs / gam
+            wo_attn = o.oproj_residual(ref.W_o, attn, np.zeros(d, np.uint16), 1, d, dims.d_o)[0]
+            resid = synth.f64_to_bf16_bits(hs - wo_attn)
+            f = ref.front(attn[None], resid[None])
+            if set(f["idx"][0].tolist()) == set(S.tolist()) and top_gap(f["logits64"][0], k) >= 1e-3:
+                break
+        else:
+            raise RuntimeError("construction failed")
+        attn0.append(attn)
+        resid0.append(resid)
+    return np.stack(attn0), np.stack(resid0), (S0, S1)

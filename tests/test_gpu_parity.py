@@ -1,0 +1,200 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Every case uses seeded synthetic inputs; indices and their order must match
+exactly, gates and intermediates within fp32-vs-fp64 tolerances, the bf16
+output within the layer's bar (tests/harness.py).
+"""
+import gc
+
+import numpy as np
+import pytest
+
+import synth
+from oracle.layer import LayerRef, build_case
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import moe_decode_layer_02_b200 as md
+    md.load()
+    synth.build_device_fill()
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def check_case(stack: H.GpuStack, case: dict, sampled=None, check_intermediates=True):
+    """Runs the step and compares every checked token (outputs for `sampled`)."""
+    out, idx, gate = stack.step(case["attn"], case["resid"])
+    L = len(case["layers"])
+    B = case["attn"].shape[1]
+    for l, per in enumerate(case["layers"]):
+        for b in per["idx"]:
+            assert np.array_equal(idx[l, b], per["idx"][b]), (l, b, idx[l, b], per["idx"][b])
+            tol = H.GATE_ATOL if l == 0 else H.GATE_ATOL_STACKED
+            assert np.allclose(gate[l, b], per["gate"][b], atol=tol, rtol=0), (l, b)
+    last = case["layers"][-1]
+    toks = sorted(last["out_ref"]) if sampled is None else sampled
+    res = []
+    for b in toks:
+        extra = sum(H.ulp_bf16(case["layers"][l]["out_ref"][b]) for l in range(L - 1)) if L > 1 else 0.0
+        res.append(H.check_out(out[b], last["out_ref"][b], extra))
+    if check_intermediates and L == 1:
+        D = stack.dims
+        hg = stack.intermediate(0, B).reshape(B, D.d)
+        rs = stack.intermediate(1, B)
+        xg = stack.intermediate(2, B).reshape(B, D.d)
+        lg = stack.intermediate(3, B).reshape(B, D.E)
+        for b in last["h"]:
+            assert np.allclose(hg[b], last["h"][b], atol=1e-4, rtol=1e-5)
+            assert abs(rs[b] - last["rstd"][b]) <= 1e-5 * last["rstd"][b]
+            assert np.allclose(xg[b], last["x"][b], atol=1e-5, rtol=1e-5)
+            assert np.allclose(lg[b], last["logits64"][b], atol=1e-4, rtol=0)
+    return out, idx, gate, res
+
+
+# --- tiny layer (d=256, d_o=256, E=16, k=2, I=128), batch 1 -----------------------------
+def test_tiny_b1():
+    seed = synth.config_seed(0)
+    st = H.GpuStack(seed, synth.TINY, max_batch=1)
+    try:
+        case = build_case(seed, synth.TINY, 1)
+        check_case(st, case)
+    finally:
+        st.close()
+
+
+@pytest.mark.parametrize("B", [2, 3, 5, 16, 64])
+@pytest.mark.parametrize("variant", [0, 1, 2])
+def test_tiny_batches_and_variants(B, variant):
+    seed = synth.config_seed(0) + 100 * B
+    st = H.GpuStack(seed, synth.TINY, max_batch=64, force_variant=variant)
+    try:
+        case = build_case(seed, synth.TINY, B)
+        check_case(st, case)
+    finally:
+        st.close()
+
+
+def test_synth_device_matches_host():
+    import torch
+    seed = 12345
+    for kind, n, start in [(synth.W_O, 1000, 0), (synth.W_GU, 777, 13), (synth.ATTN, 64, 5)]:
+        x = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        synth.device_fill(x, seed, kind, layer=3, start=start)
+        got = x.view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, synth.gen_bf16(seed, kind, n, layer=3, start=start))
+
+
+# --- ragged shapes: d not a multiple of 256 (no split-K), odd d_o/E/k/I ----------------------
+@pytest.mark.parametrize("B", [1, 2, 3, 7])
+def test_ragged_shapes(B):
+    dims = synth.Dims(320, 192, 40, 5, 96)
+    seed = synth.config_seed(9) + B
+    st = H.GpuStack(seed, dims, max_batch=8)
+    try:
+        check_case(st, build_case(seed, dims, B))
+    finally:
+        st.close()
+
+
+def test_degenerate_k_equals_e_and_k1():
+    for dims in (synth.Dims(128, 64, 4, 4, 32), synth.Dims(128, 128, 8, 1, 64)):
+        seed = synth.config_seed(11) + dims.k
+        st = H.GpuStack(seed, dims, max_batch=4)
+        try:
+            check_case(st, build_case(seed, dims, 3))
+        finally:
+            st.close()
+
+
+def test_determinism_replay():
+    seed = synth.config_seed(0) + 7
+    st = H.GpuStack(seed, synth.TINY, max_batch=16)
+    try:
+        case = build_case(seed, synth.TINY, 16)
+        o1, i1, g1 = st.step(case["attn"], case["resid"])
+        o2, i2, g2 = st.step(case["attn"], case["resid"], reps=3)
+        assert np.array_equal(o1, o2) and np.array_equal(i1, i2) and np.array_equal(g1, g2)
+    finally:
+        st.close()
+
+
+# --- full-size layer (one GPU's 1/16 tensor-parallel shard), batch 1 --------------------------
+@pytest.fixture(scope="module")
+def tp16():
+    seed = synth.config_seed(1)
+    st = H.GpuStack(seed, synth.TP16, max_batch=64)
+    ref = LayerRef(seed, synth.TP16, 0)
+    yield seed, st, ref
+    st.close()
+
+
+@pytest.mark.slow
+def test_tp16_b1(tp16):
+    seed, st, ref = tp16
+    check_case(st, build_case(seed, synth.TP16, 1, refs=[ref]))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("overlap", [16, 8, 0])
+def test_tp16_b2_overlap(tp16, overlap):
+    seed, st, ref = tp16
+    attn0, resid0, (S0, S1) = H.constructed_b2(seed, synth.TP16, overlap, ref=ref)
+    case = build_case(seed, synth.TP16, 2, attn0=attn0, resid0=resid0, refs=[ref])
+    out, idx, gate, _ = check_case(st, case)
+    assert len(set(idx[0, 0]) & set(idx[0, 1])) == overlap
+
+
+# --- full-size layer (1/8 shard, I=256), batch 16 and 64 -------------------------------------
+@pytest.fixture(scope="module")
+def tp8():
+    seed = synth.config_seed(3)
+    st = H.GpuStack(seed, synth.TP8, max_batch=64)
+    ref = LayerRef(seed, synth.TP8, 0)
+    yield seed, st, ref
+    st.close()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("B", [16, 64])
+def test_tp8_batches(tp8, B):
+    seed, st, ref = tp8
+    sampled = [0, B // 2, B - 1]
+    case = build_case(seed, synth.TP8, B, refs=[ref], moe_tokens=sampled)
+    out, idx, gate, _ = check_case(st, case, sampled=sampled)
+    # every token: valid, distinct, and gates a descending distribution
+    assert np.all((idx >= 0) & (idx < synth.TP8.E))
+    for b in range(B):
+        assert len(set(idx[0, b])) == synth.TP8.k
+        assert abs(gate[0, b].sum() - 1) < 1e-5 and np.all(np.diff(gate[0, b]) <= 0)
+
+
+# --- stack of 8 full-size layers, batch 1 and 64, prefetch on and off -----------------------------
+@pytest.fixture(scope="module")
+def stack8():
+    seed = synth.config_seed(4)
+    w = H.device_weights(seed, synth.TP16, 8)
+    refs = [LayerRef(seed, synth.TP16, l) for l in range(8)]
+    yield seed, w, refs
+    del w
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("prefetch", [0, 1])
+@pytest.mark.parametrize("B", [1, 64])
+def test_stack8(stack8, B, prefetch):
+    seed, w, refs = stack8
+    st = H.GpuStack(seed, synth.TP16, n_layers=8, max_batch=64, prefetch=prefetch, weights=w)
+    try:
+        sampled = [0] if B == 1 else [0, 37]
+        case = build_case(seed, synth.TP16, B, n_layers=8, checked=sampled, refs=refs)
+        check_case(st, case, sampled=sampled)
+    finally:
+        st.close()
