@@ -45,6 +45,10 @@ WORKLOADS = {
     "tp8_b64": ("TP8", 64, 1, "indep"),
     "stack8_b1": ("TP16", 1, 8, "indep"),
     "stack8_b64": ("TP16", 64, 8, "indep"),
+    # profiling case: tp16 o_proj/router/expert shapes with 64 experts (~0.6 GB on the device)
+    "tp16e64_b1": ("TP16E64", 1, 1, "indep"),
+    "tp16e64_b2": ("TP16E64", 2, 1, "indep"),
+    "tp8e64_b64": ("TP8E64", 64, 1, "indep"),
 }
 
 KERNEL_FILE = os.path.join(ROOT, "moe_decode_layer_02_b200", "csrc", "kernels.cu")
@@ -60,7 +64,13 @@ def peaks():
 
 def dims_of(name):
     import synth
-    return getattr(synth, name)
+    small = {"TP16E64": synth.Dims(7168, 8192, 64, 16, 128), "TP8E64": synth.Dims(7168, 8192, 64, 16, 256)}
+    return small[name] if name in small else getattr(synth, name)
+
+
+def seed_of(dname, L):
+    import synth
+    return synth.config_seed({"TP16": 1, "TP8": 3, "TP16E64": 21, "TP8E64": 23}[dname] + (10 if L > 1 else 0))
 
 
 def token_inputs(seed, dims, B, L, mode):
@@ -174,7 +184,7 @@ def run_ours(args, rank, world):
     md.load()
     dname, B, L, mode = WORKLOADS[args.workload]
     dims = dims_of(dname)
-    seed = synth.config_seed({"TP16": 1, "TP8": 3}[dname] + (10 if L > 1 else 0))
+    seed = seed_of(dname, L)
     sz = dims.sizes()
     weights = []
     for l in range(L):
@@ -201,6 +211,15 @@ def run_ours(args, rank, world):
 
     for _ in range(max(args.warmup, 3)):
         step()
+    if args.profile_run:
+        # Profiling mode (for ncu): a few plain graph replays, no timing.
+        for _ in range(args.profile_run):
+            step()
+        rc = md.moe_decode_sync_status(h, s)
+        md.moe_decode_destroy(h)
+        if rc:
+            raise RuntimeError(md.strerror(rc))
+        return None
     rc = md.moe_decode_sync_status(h, s)
     if rc:
         raise RuntimeError(md.strerror(rc))
@@ -285,7 +304,7 @@ def cpu_baseline(args, budget_s=12.0):
     o = oracle.get()
     dname, B, L, mode = WORKLOADS[args.workload]
     dims = dims_of(dname)
-    seed = synth.config_seed({"TP16": 1, "TP8": 3}[dname] + (10 if L > 1 else 0))
+    seed = seed_of(dname, L)
     ref = LayerRef(seed, dims, 0, oracle=o)
     attn_np, resid_np = token_inputs(seed, dims, B, 1, mode)
     # Warm the expert cache (host generation of weights is setup, not oracle work).
@@ -319,6 +338,8 @@ def main():
     ap.add_argument("--workload", default="tp16_b1", choices=sorted(WORKLOADS))
     ap.add_argument("--prefetch", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-run", type=int, default=0,
+                    help="profiling mode: warm up, replay the step N times, print nothing")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -352,7 +373,7 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
-    if rank != 0:
+    if rank != 0 or r is None:
         return
     hbm, bf16, src = peaks()
     dims = r["dims"]

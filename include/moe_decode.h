@@ -75,8 +75,8 @@ enum {
  *   rms_eps    RMSNorm epsilon (> 0; the layer uses 1e-6)
  *   enable_prefetch  1: a side stream prefetches layer l+1's router, RMSNorm scale and
  *                    the head of its W_o into L2 while layer l runs its experts
- *   force_variant    0: expert kernel by batch size (small-M at B <= 2, split-K above);
- *                    1: always small-M; 2: always split-K (testing)                       */
+ *   force_variant    0 or 1: expert gate/up kernel by batch size (small-M at B <= 2,
+ *                    split-K above); 2: split-K at every batch size (testing)              */
 typedef struct {
   int d, d_o, n_experts, top_k, inter, max_batch, n_layers;
   float rms_eps;

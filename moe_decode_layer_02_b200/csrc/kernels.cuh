@@ -30,9 +30,13 @@ struct Workspace {
 
 struct KTune {
   int stages = 0;          // ring stages
-  int rows_per_stage = 0;  // weight rows (or row pairs) per stage
+  int rows_per_stage = 0;  // weight rows (or row pairs) per stage (CUDA-core kernels)
   int rows_max = 0;        // max rows owned by one CTA
   int n_split = 0;         // split-K factor (gate/up large-batch variant)
+  int kc = 0;              // K chunk of one MMA stage (multiple of 64)
+  int nch = 0;             // K chunks per row (K = kc * nch)
+  int tok_group = 0;       // tokens per pass over the weights
+  int a_in_smem = 0;       // down kernel: all SwiGLU activations staged in shared memory
   size_t smem = 0;         // dynamic shared memory bytes
 };
 
@@ -55,7 +59,7 @@ struct PrefetchArgs {
   int n;
 };
 
-// Host-side planning (sets the KTune fields, returns false if unsupported).
+// Host-side planning for a.B tokens (sets the KTune fields, returns false if unsupported).
 bool plan_layer(LayerArgs& a, int num_sms, size_t smem_optin);
 
 // Launchers (pdl: launch with programmatic stream serialisation).

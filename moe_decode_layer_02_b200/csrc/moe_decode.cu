@@ -93,8 +93,8 @@ int check_cfg(const moe_decode_config* c) {
 }
 
 int pick_split(int d) {
-  for (int ns = 1; ns <= d / 256; ++ns)
-    if (d % ns == 0 && (d / ns) % 256 == 0 && d / ns <= 1024) return ns;
+  for (int ns = 1; ns <= d / 64; ++ns)
+    if (d % ns == 0 && (d / ns) % 64 == 0 && d / ns <= 1024) return ns;
   return 0;
 }
 
@@ -114,10 +114,8 @@ void release(moe_decode_handle* h) {
 }
 
 bool use_splitk(const moe_decode_handle* h, int B) {
-  if (!h->has_splitk) return false;
-  if (h->cfg.force_variant == 1) return false;
-  if (h->cfg.force_variant == 2) return true;
-  return B >= 3;  // small-matrix kernels at batch one or two, split-K above
+  if (B >= 3) return true;                        // split-K above batch two
+  return h->cfg.force_variant == 2;               // small-matrix kernels at batch one or two
 }
 
 LayerArgs layer_args(const moe_decode_handle* h, int l, int B, const void* attn, const void* resid,
@@ -125,6 +123,7 @@ LayerArgs layer_args(const moe_decode_handle* h, int l, int B, const void* attn,
   const moe_decode_config& c = h->cfg;
   LayerArgs a = use_splitk(h, B) ? h->plan_splitk : h->plan_small;
   a.B = B;
+  plan_layer(a, h->num_sms, h->smem_optin);  // validated for every batch size at create
   a.w_o = static_cast<const uint16_t*>(h->w[l].w_o);
   a.gamma = static_cast<const uint16_t*>(h->w[l].gamma);
   a.w_r = static_cast<const uint16_t*>(h->w[l].w_router);
@@ -255,7 +254,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   }
   h->n_split = pick_split(d);
 
-  // ---- plans ---------------------------------------------------------------------------
+  // ---- plans: every batch size 1..max_batch must fit ------------------------------------
   LayerArgs base{};
   base.maxB = maxB;
   base.d = d;
@@ -266,16 +265,21 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   base.eps = cfg->rms_eps;
   h->plan_small = base;
   h->plan_small.k3.n_split = 0;
-  if (!plan_layer(h->plan_small, G, h->smem_optin)) {
-    delete h;
-    return MOE_ERR_UNSUPPORTED_CONFIG;
+  h->plan_splitk = base;
+  h->plan_splitk.k3.n_split = h->n_split;
+  h->has_splitk = h->n_split > 0;
+  bool ok = h->has_splitk;
+  for (int B = 1; B <= maxB && ok; ++B) {
+    LayerArgs t = (B <= 2) ? h->plan_small : h->plan_splitk;
+    t.B = B;
+    ok = plan_layer(t, G, h->smem_optin);
+    if (ok && B <= 2) {
+      LayerArgs u = h->plan_splitk;
+      u.B = B;
+      ok = plan_layer(u, G, h->smem_optin);
+    }
   }
-  if (h->n_split > 0) {
-    h->plan_splitk = base;
-    h->plan_splitk.k3.n_split = h->n_split;
-    h->has_splitk = plan_layer(h->plan_splitk, G, h->smem_optin);
-  }
-  if (cfg->force_variant == 2 && !h->has_splitk) {
+  if (!ok) {
     delete h;
     return MOE_ERR_UNSUPPORTED_CONFIG;
   }
