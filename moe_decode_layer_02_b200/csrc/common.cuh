@@ -92,6 +92,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Waits for a phase while ignoring the abort flag (used to drain copies in flight).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      atomicOr(err, kErrTimeout);
+      return;
+    }
+  }
+}
+
+// ---- shared-memory ring of S stages (full: TMA completion, empty: consumer warps) ----
+__device__ __forceinline__ void init_ring(uint64_t* full, uint64_t* empty, int S, int consumers = kConsumerWarps) {
+  for (int s = 0; s < S; ++s) {
+    mbar_init(&full[s], 1);
+    if (empty) mbar_init(&empty[s], consumers);
+  }
+}
+
+// Producer: waits until the slot of fill number `it` is free (bounded).
+__device__ __forceinline__ bool ring_acquire(uint64_t* empty, int it, int S, volatile int* abort_flag, uint32_t* err) {
+  if (it < S) return !*abort_flag;
+  return mbar_wait(&empty[it % S], ((it / S) - 1) & 1, abort_flag, err);
+}
+
+// Producer epilogue: waits (bounded, ignoring abort) for the last min(S, issued) fills, so
+// that no copy is still writing into shared memory when the CTA exits.
+__device__ __forceinline__ void ring_drain(uint64_t* full, int issued, int S, uint32_t* err) {
+  for (int i = issued - S < 0 ? 0 : issued - S; i < issued; ++i) mbar_drain(&full[i % S], (i / S) & 1, err);
+}
+
 // ---- TMA bulk copies (1-D, global -> shared) ---------------------------------------
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;

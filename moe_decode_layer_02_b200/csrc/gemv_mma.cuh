@@ -91,3 +91,84 @@ __device__ __forceinline__ void warp_steps(int S, int w, int& s0, int& s1) {
 }
 
 }  // namespace moe
+
+namespace moe {
+
+// ---------------------------------------------------------------------------------------
+// Register-streamed variant: weights go from global memory straight into the B fragments.
+//
+// One warp covers 8 weight rows x one 64-element k-block per step.  Lane (g, q) loads
+// two 16-byte vectors of row g: elements [8q, 8q+8) and [32+8q, 32+8q+8) of the block, so
+// each load instruction reads 64 contiguous bytes of every row (no shared memory, no
+// unpacking).  The MMA's logical k order is a permutation of the block's 64 elements;
+// the same permutation is applied to the activations, so the products and the sum over
+// the block are unchanged:
+//   step 0: lane q's words 0,1 of the first vector (elements 8q + 0..3)
+//   step 1: words 2,3 of the first vector (8q + 4..7)
+//   step 2: words 0,1 of the second vector (32 + 8q + 0..3)
+//   step 3: words 2,3 of the second vector (32 + 8q + 4..7)
+// with a0/b0 the first word of a step and a2/b1 the second.
+// ---------------------------------------------------------------------------------------
+struct Frag {
+  uint4 lo, hi;  // elements [8q, 8q+8) and [32+8q, 32+8q+8) of a 64-element block
+};
+
+// 128-bit weight load with an L2 256-byte fetch hint (static weights only).
+__device__ __forceinline__ uint4 ld_w128(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Weight fragment of k-block starting at `row_kb` (row base + 64*kb elements); zeros if !ok.
+__device__ __forceinline__ void load_wfrag(Frag& f, const uint16_t* row_kb, int q, bool ok) {
+  if (ok) {
+    f.lo = ld_w128(row_kb + 8 * q);
+    f.hi = ld_w128(row_kb + 32 + 8 * q);
+  } else {
+    f.lo = make_uint4(0, 0, 0, 0);
+    f.hi = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Activation fragment (bf16 row in shared memory, `row_kb` = row + 64*kb elements).
+__device__ __forceinline__ void load_afrag(Frag& f, const uint16_t* row_kb, int q, bool ok) {
+  if (ok) {
+    f.lo = *reinterpret_cast<const uint4*>(row_kb + 8 * q);
+    f.hi = *reinterpret_cast<const uint4*>(row_kb + 32 + 8 * q);
+  } else {
+    f.lo = make_uint4(0, 0, 0, 0);
+    f.hi = make_uint4(0, 0, 0, 0);
+  }
+}
+
+__device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 64-element k-block: activation rows g (ag) and g + 8 (ag8) against weight rows.
+__device__ __forceinline__ void mma_kblock(float* d, const Frag& ag, const Frag& ag8, const Frag& w) {
+  mma16816(d, ag.lo.x, ag8.lo.x, ag.lo.y, ag8.lo.y, w.lo.x, w.lo.y);
+  mma16816(d, ag.lo.z, ag8.lo.z, ag.lo.w, ag8.lo.w, w.lo.z, w.lo.w);
+  mma16816(d, ag.hi.x, ag8.hi.x, ag.hi.y, ag8.hi.y, w.hi.x, w.hi.y);
+  mma16816(d, ag.hi.z, ag8.hi.z, ag.hi.w, ag8.hi.w, w.hi.z, w.hi.w);
+}
+
+// D fragment ownership: lane (g, q): d0 = D[g][2q], d1 = D[g][2q+1], d2 = D[g+8][2q], d3 = D[g+8][2q+1]
+// (rows = activation rows, columns = weight rows).  Writes all of it to red[16][8].
+__device__ __forceinline__ void store_d(float* red, const float* d, int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  red[g * 8 + 2 * q] = d[0];
+  red[g * 8 + 2 * q + 1] = d[1];
+  red[(g + 8) * 8 + 2 * q] = d[2];
+  red[(g + 8) * 8 + 2 * q + 1] = d[3];
+}
+
+}  // namespace moe

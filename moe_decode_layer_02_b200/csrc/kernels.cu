@@ -1,18 +1,12 @@
 // sm_100a kernels of one MoE decode-layer step.
 //
+// Large-batch kernels (the small-batch path and the router are in kernels_small.cu):
 //   K1 k_oproj           h = residual + W_o . attn_out on the tensor cores (weights as the
-//                        MMA's N operand) and per-CTA sums of h^2 (no grid-wide step: every
-//                        router CTA reduces the partial sums itself, in one fixed order).
-//   K2 k_router_topk     rstd from the o_proj partial sums; x = h * rstd * gamma (fp32, split
-//                        into bf16 hi + lo for the MMA);
-//                        logits = W_r . x; the last CTA selects the top-k per token with
-//                        warp shuffles, computes the softmax gates and builds the routing
-//                        tables (union of selected experts, per-expert token entries, CSR).
-//   K3 k_gateup_small    small-M expert gate/up (batch <= 2): every (union expert, row pair)
-//                        streamed once and multiplied with all tokens; a = silu(g) * u.
-//      k_gateup_splitk   split-K expert gate/up for larger batches: (expert, K chunk) units
+//                        MMA's N operand, staged through a shared-memory ring by TMA bulk
+//                        copies), tokens in groups of up to 8, per-CTA sums of h^2.
+//   K3 k_gateup_splitk   split-K expert gate/up for batches above two: (expert, K chunk) units
 //                        whose partial sums are reduced in chunk order by the last unit of
-//                        each expert.
+//                        each expert (atomic ticket per expert, no spinning).
 //   K4 k_down_combine    out = bf16(h + sum_j gate_j * W_down[e_j] . a_j): rows of d split over
 //                        CTAs, experts streamed in ascending order, fixed reduction order.
 //   k_prefetch_l2        side-stream L2 prefetch of the next layer's weights.
@@ -42,54 +36,11 @@ __device__ __forceinline__ float ld_act_bf16(const uint16_t* p) {
   return bf16f(__ldcg(reinterpret_cast<const unsigned short*>(p)));
 }
 
-__device__ __forceinline__ void unpack8(uint4 w, float* f) {
-  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
-}
 
-// Waits for a phase while ignoring the abort flag (used to drain copies in flight).
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint32_t* err) {
-  const unsigned long long t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      atomicOr(err, kErrTimeout);
-      return;
-    }
-  }
-}
 
-// Producer side of the ring: waits until stage `it % S` is free.
-__device__ __forceinline__ bool ring_acquire(uint64_t* empty, int it, int S, volatile int* abort_flag,
-                                             uint32_t* err) {
-  if (it < S) return !*abort_flag;
-  return mbar_wait(&empty[it % S], ((it / S) - 1) & 1, abort_flag, err);
-}
 
-// Producer epilogue: wait (bounded, ignoring abort) for the last min(S, issued) copies.
-__device__ __forceinline__ void ring_drain(uint64_t* full, int issued, int S, uint32_t* err) {
-  for (int i = issued - S < 0 ? 0 : issued - S; i < issued; ++i) mbar_drain(&full[i % S], (i / S) & 1, err);
-}
 
-// Last-CTA ticket: returns true in the CTA that arrives last.  All threads call it.
-__device__ __forceinline__ bool last_cta(unsigned* counter, int* s_flag) {
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned prev = atomicAdd(counter, 1u);
-    *s_flag = (prev == gridDim.x - 1);
-  }
-  __syncthreads();
-  const bool last = *s_flag != 0;
-  if (last) __threadfence();
-  return last;
-}
 
-__device__ __forceinline__ void init_ring(uint64_t* full, uint64_t* empty, int S) {
-  for (int s = 0; s < S; ++s) {
-    mbar_init(&full[s], 1);
-    if (empty) mbar_init(&empty[s], kConsumerWarps);
-  }
-}
 
 __device__ __forceinline__ size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
 
@@ -199,446 +150,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_oproj(const LayerArgs a) {
 
 }
 
-// =============================================================================
-// K2: RMSNorm apply + router GEMV + top-k + gates + routing tables
-// =============================================================================
-namespace {
-
-constexpr int kCandMax = 128;           // candidates kept per token by the threshold pass
-constexpr int kTopkScratch = 48 * 1024;  // shared memory used by the last CTA
-
-__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
-}
-
-// Exact top-K of one token's E logits by one warp: (value desc, index asc).
-// Threshold pass: the K-th largest of the 32 lane maxima is a lower bound T of the
-// K-th largest logit, so every selected expert has a logit >= T.  Those candidates are
-// compacted and ranked exactly; the fallback (more than kCandMax candidates, e.g. mass
-// ties) repeats a warp arg-max K times.  Lane j < K returns the j-th selection.
-__device__ void warp_topk(const float* logits, int E, int K, float* cand_v, int* cand_i, int lane,
-                          float& my_v, int& my_i) {
-  float v[32];
-  float lm = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = lane + 32 * i;
-    float x = -INFINITY;
-    if (e < E) {
-      x = ld_act(logits + e);
-      if (x != x) x = -INFINITY;  // NaN never outranks a number
-    }
-    v[i] = x;
-    if (e < E) lm = fmaxf(lm, x);
-  }
-  // Rank of this lane's maximum among the 32 (ties by lane id); T = the (K-1)-ranked one.
-  int rank = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float o = __shfl_sync(0xffffffffu, lm, j);
-    rank += (o > lm) || (o == lm && j < lane);
-  }
-  const unsigned who = __ballot_sync(0xffffffffu, rank == K - 1);
-  const float T = __shfl_sync(0xffffffffu, lm, __ffs(who) - 1);
-  int cnt = 0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) cnt += (lane + 32 * i < E && v[i] >= T);
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int C = __shfl_sync(0xffffffffu, incl, 31);
-  if (C <= kCandMax) {
-    int w = incl - cnt;
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (lane + 32 * i < E && v[i] >= T) {
-        cand_v[w] = v[i];
-        cand_i[w] = lane + 32 * i;
-        ++w;
-      }
-    __syncwarp();
-    // Exact rank of each candidate among the candidates = its rank among all experts.
-    for (int cidx = lane; cidx < C; cidx += 32) {
-      const float cv = cand_v[cidx];
-      const int ci = cand_i[cidx];
-      int r = 0;
-      for (int o = 0; o < C; ++o) r += better(cand_v[o], cand_i[o], cv, ci);
-      cand_v[kCandMax + cidx] = __int_as_float(r);
-    }
-    __syncwarp();
-    for (int cidx = lane; cidx < C; cidx += 32) {
-      const int r = __float_as_int(cand_v[kCandMax + cidx]);
-      if (r < K) {  // slots [2*kCandMax, 2*kCandMax + 32): selections in rank order
-        cand_v[2 * kCandMax + r] = cand_v[cidx];
-        cand_i[2 * kCandMax + r] = cand_i[cidx];
-      }
-    }
-    __syncwarp();
-    if (lane < K) {
-      my_v = cand_v[2 * kCandMax + lane];
-      my_i = cand_i[2 * kCandMax + lane];
-    }
-    __syncwarp();
-    return;
-  }
-  // Fallback: K rounds of warp arg-max over the remaining elements.
-  uint32_t taken = 0;
-#pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if (lane + 32 * i >= E) taken |= 1u << i;
-  float lbv = -INFINITY;
-  int lbi = 0x7fffffff;
-#pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if (!((taken >> i) & 1u) && better(v[i], lane + 32 * i, lbv, lbi)) { lbv = v[i]; lbi = lane + 32 * i; }
-  for (int j = 0; j < K; ++j) {
-    float bv = lbv;
-    int bi = lbi;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-    }
-    if (lane == j) { my_v = bv; my_i = bi; }
-    if ((bi & 31) == lane) {
-      taken |= 1u << (bi >> 5);
-      lbv = -INFINITY;
-      lbi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (!((taken >> i) & 1u) && better(v[i], lane + 32 * i, lbv, lbi)) { lbv = v[i]; lbi = lane + 32 * i; }
-    }
-  }
-}
-
-// Executed by every thread of the last router CTA.
-__device__ void topk_route(const LayerArgs& a, unsigned char* scratch) {
-  const int B = a.B, E = a.E, K = a.k;
-  unsigned long long* mask = reinterpret_cast<unsigned long long*>(scratch);  // [1024]
-  int* off_e = reinterpret_cast<int*>(mask + 1024);                         // [1024]
-  int* sidx = off_e + 1024;                                                 // [64*32]
-  float* cand = reinterpret_cast<float*>(sidx + 64 * 32);                   // [nwarps][2*kCandMax+32] x2
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  const int cstride = 2 * kCandMax + 32;
-  float* cv = cand + warp * 2 * cstride;
-  int* ci = reinterpret_cast<int*>(cv + cstride);
-
-  for (int e = threadIdx.x; e < E; e += blockDim.x) mask[e] = 0ull;
-
-  for (int t = warp; t < B; t += nwarps) {
-    float my_v = 0.f;
-    int my_i = 0;
-    warp_topk(a.ws.logits + (size_t)t * E, E, K, cv, ci, lane, my_v, my_i);
-    const float v0 = __shfl_sync(0xffffffffu, my_v, 0);
-    const float w = (lane < K) ? expf(my_v - v0) : 0.f;
-    const float sum = warp_sum(w);
-    if (lane < K) {
-      const float gte = w / sum;
-      const int e = (my_i >= 0 && my_i < E) ? my_i : 0;
-      if (e != my_i) atomicOr(a.ws.err, kErrBounds);
-      a.ws.topk_idx[t * K + lane] = e;
-      a.ws.topk_gate[t * K + lane] = gte;
-      if (a.user_idx) a.user_idx[t * K + lane] = e;
-      if (a.user_gate) a.user_gate[t * K + lane] = gte;
-      sidx[t * K + lane] = e;
-    }
-  }
-  __syncthreads();
-  for (int p = threadIdx.x; p < B * K; p += blockDim.x) atomicOr(&mask[sidx[p]], 1ull << (p / K));
-  __syncthreads();
-
-  // Union of experts and CSR offsets: warp 0 scans E <= 1024 in 32-expert strips.
-  if (warp == 0) {
-    int cnt = 0, nu = 0;
-    const int e0 = lane * 32;
-    for (int e = e0; e < e0 + 32 && e < E; ++e) {
-      const int c = __popcll(mask[e]);
-      cnt += c;
-      nu += (c > 0);
-    }
-    int icnt = cnt, inu = nu;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, icnt, o);
-      const int z = __shfl_up_sync(0xffffffffu, inu, o);
-      if (lane >= o) { icnt += y; inu += z; }
-    }
-    int off = icnt - cnt, u = inu - nu;
-    for (int e = e0; e < e0 + 32 && e < E; ++e) {
-      const int c = __popcll(mask[e]);
-      off_e[e] = off;
-      if (c > 0) {
-        a.ws.union_e[u] = e;
-        a.ws.union_off[u] = off;
-        ++u;
-      }
-      off += c;
-    }
-    if (lane == 31) {
-      *a.ws.n_union = inu;
-      a.ws.union_off[inu] = icnt;
-    }
-  }
-  __syncthreads();
-  for (int p = threadIdx.x; p < B * K; p += blockDim.x) {
-    const int t = p / K, j = p % K, e = sidx[p];
-    const unsigned long long below = (t == 0) ? 0ull : (mask[e] & ((~0ull) >> (64 - t)));
-    const int pos = off_e[e] + __popcll(below);
-    a.ws.entry_tok[pos] = t;
-    a.ws.entry_slot[pos] = j;
-  }
-}
-
-}  // namespace
-
-//   CTA c owns rows [e0, e0 + nrows) of W_r (at most 8): all K chunks stay resident;
-//   tokens in groups of 2 (4 MMA rows: hi and lo of each token's x).
-__global__ void __launch_bounds__(kThreads, 1) k_router_topk(const LayerArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int G = gridDim.x, c = blockIdx.x;
-  const int d = a.d, E = a.E, B = a.B;
-  const int kc = a.k2.kc, nch = a.k2.nch;
-  const int wp = pitch_bytes(kc), ap = pitch_bytes(d);
-  const size_t SB = align128((size_t)kGroupRows * wp);
-  long long lo, hi;
-  split_range(E, G, c, lo, hi);
-  const int e0 = (int)lo, nrows = (int)(hi - lo);
-
-  unsigned char* wst = smem;                                          // [nch][8][wp]
-  unsigned char* act = wst + (size_t)nch * SB;                        // [4][ap]
-  unsigned char* scratch = act + align128((size_t)4 * ap);            // last CTA
-  uint64_t* full = reinterpret_cast<uint64_t*>(scratch + kTopkScratch);
-  float* red = reinterpret_cast<float*>(full + nch);
-  float* rstd_s = red + kConsumerWarps * 64;  // [B]
-  int* s_misc = reinterpret_cast<int*>(rstd_s + 64);
-  volatile int* abort_flag = s_misc;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  if (tid == 0) {
-    init_ring(full, nullptr, nch);
-    s_misc[0] = 0;
-    s_misc[1] = 0;
-    fence_barrier_init();
-  }
-  __syncthreads();
-  pdl_trigger();
-
-  const uint32_t seg = (uint32_t)kc * 2u;
-  if (warp == kConsumerWarps) {
-    // The router slice is static: fetch all of it before the dependency resolves.
-    if (lane == 0 && nrows > 0) {
-      const uint64_t pol = policy_evict_first();
-      for (int ch = 0; ch < nch; ++ch) {
-        mbar_arrive_expect_tx(&full[ch], nrows * seg);
-        for (int j = 0; j < nrows; ++j)
-          bulk_g2s(wst + ch * SB + j * wp, a.w_r + (size_t)(e0 + j) * d + (size_t)ch * kc, seg, &full[ch], pol);
-      }
-      for (int ch = 0; ch < nch; ++ch) mbar_drain(&full[ch], 0, a.ws.err);
-    }
-  } else {
-    pdl_wait();  // h and the sums of h^2 come from the o_proj kernel
-    // rstd[t] = 1/sqrt(sum_c ss_part[c][t] / d + eps): warp t%8 sums the G partials in a
-    // fixed order (lane strides, then a butterfly), so every CTA gets the same bits.
-    for (int t = warp; t < B; t += kConsumerWarps) {
-      float ss = 0.f;
-      for (int cc = lane; cc < G; cc += 32) ss += ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]);
-      ss = warp_sum(ss);
-      if (lane == 0) {
-        const float r = 1.0f / sqrtf(ss / (float)d + a.eps);
-        rstd_s[t] = r;
-        if (c == 0) a.ws.rstd[t] = r;
-      }
-    }
-    consumer_sync();
-    const int S_k = kc / 16;
-    int s0, s1;
-    warp_steps(S_k, warp, s0, s1);
-    const int cpr = d / 8;
-    bool have_w = false;
-    for (int t0 = 0; t0 < B; t0 += 2) {
-      const int nt = min(2, B - t0);
-      for (int t = 0; t < nt; ++t) {
-        const float r = rstd_s[t0 + t];
-        for (int q = tid; q < cpr; q += kConsumerThreads) {
-          const float* hp = a.ws.h + (size_t)(t0 + t) * d + (size_t)q * 8;
-          const float4 h0 = ld_act4(hp), h1 = ld_act4(hp + 4);
-          float gm[8];
-          unpack8(ld_weight_u4(a.gamma + (size_t)q * 8), gm);
-          const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-          float xv[8];
-          uint16_t xh[8], xl[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            xv[e] = hv[e] * r * gm[e];
-            split_bf16(xv[e], xh[e], xl[e]);
-          }
-          uint4 ph, pl;
-          ph.x = xh[0] | ((uint32_t)xh[1] << 16); ph.y = xh[2] | ((uint32_t)xh[3] << 16);
-          ph.z = xh[4] | ((uint32_t)xh[5] << 16); ph.w = xh[6] | ((uint32_t)xh[7] << 16);
-          pl.x = xl[0] | ((uint32_t)xl[1] << 16); pl.y = xl[2] | ((uint32_t)xl[3] << 16);
-          pl.z = xl[4] | ((uint32_t)xl[5] << 16); pl.w = xl[6] | ((uint32_t)xl[7] << 16);
-          *reinterpret_cast<uint4*>(act + (size_t)(2 * t) * ap + (size_t)q * 16) = ph;
-          *reinterpret_cast<uint4*>(act + (size_t)(2 * t + 1) * ap + (size_t)q * 16) = pl;
-          if (q % G == c) {  // each chunk of x is written by exactly one CTA
-            float* xp = a.ws.x + (size_t)(t0 + t) * d + (size_t)q * 8;
-            *reinterpret_cast<float4*>(xp) = make_float4(xv[0], xv[1], xv[2], xv[3]);
-            *reinterpret_cast<float4*>(xp + 4) = make_float4(xv[4], xv[5], xv[6], xv[7]);
-          }
-        }
-      }
-      consumer_sync();
-      float dacc[4] = {0.f, 0.f, 0.f, 0.f};
-      if (nrows > 0) {
-        for (int ch = 0; ch < nch; ++ch) {
-          if (!have_w) mbar_wait(&full[ch], 0, abort_flag, a.ws.err);
-          mma_stage(dacc, wst + ch * SB, wp, act, ap, 2 * nt, ch * kc, s0, s1, lane);
-        }
-        have_w = true;
-      }
-      mma_store_partial(red, dacc, 2 * nt, warp, lane);
-      consumer_sync();
-      for (int z = tid; z < nrows * nt; z += kConsumerThreads) {
-        const int n = z / nt, t = z % nt;
-        const float v = mma_reduce(red, 2 * t, n) + mma_reduce(red, 2 * t + 1, n);
-        a.ws.logits[(size_t)(t0 + t) * E + e0 + n] = v;
-      }
-      consumer_sync();
-    }
-  }
-
-  if (last_cta(&a.ws.counters[kCntRouter], &s_misc[1])) {
-    topk_route(a, scratch);
-    if (tid == 0) a.ws.counters[kCntRouter] = 0;
-  }
-}
-
-// =============================================================================
-// K3 (small-M, batch <= 2): expert gate/up + SiLU*mul on the tensor cores.
-//   Units are (union expert u, row pair p) in flattened order; a CTA takes a contiguous
-//   range, 4 pairs per MMA group (rows 0..3 gate p.., rows 4..7 up p..), K in chunks.
-//   Every token's x is an MMA row pair (hi, lo); a is written only for tokens routed to u.
-// =============================================================================
-__global__ void __launch_bounds__(kThreads, 1) k_gateup_small(const LayerArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int G = gridDim.x, c = blockIdx.x;
-  const int d = a.d, I = a.I, E = a.E, B = a.B, K = a.k;
-  const int S = a.k3.stages, kc = a.k3.kc, nch = a.k3.nch;
-  const int wp = pitch_bytes(kc), ap = pitch_bytes(d);
-  const size_t SB = align128((size_t)kGroupRows * wp);
-  const int umax = min(E, B * K);
-
-  unsigned char* ring = smem;
-  unsigned char* act = ring + (size_t)S * SB;                          // [2B][ap]
-  int* un_e = reinterpret_cast<int*>(act + align128((size_t)4 * ap));  // [umax]
-  int* un_off = un_e + umax;                                           // [umax+1]
-  int* ent_tok = un_off + umax + 1;                                    // [B*K]
-  uint64_t* full = reinterpret_cast<uint64_t*>(align128(reinterpret_cast<size_t>(ent_tok + B * K) -
-                                                        reinterpret_cast<size_t>(smem)) + smem);
-  uint64_t* empty = full + S;
-  float* red = reinterpret_cast<float*>(empty + S);
-  int* s_misc = reinterpret_cast<int*>(red + kConsumerWarps * 64);
-  volatile int* abort_flag = s_misc;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  if (tid == 0) {
-    init_ring(full, empty, S);
-    s_misc[0] = 0;
-    fence_barrier_init();
-  }
-  pdl_wait();  // routing tables and x come from the router kernel
-  pdl_trigger();
-  int U = ld_act_i(a.ws.n_union);
-  if (U < 0 || U > umax) {
-    if (tid == 0) atomicOr(a.ws.err, kErrBounds);
-    U = 0;
-  }
-  for (int i = tid; i < U; i += blockDim.x) {
-    int e = ld_act_i(&a.ws.union_e[i]);
-    if (e < 0 || e >= E) { atomicOr(a.ws.err, kErrBounds); e = 0; }
-    un_e[i] = e;
-  }
-  for (int i = tid; i <= U; i += blockDim.x) un_off[i] = ld_act_i(&a.ws.union_off[i]);
-  for (int i = tid; i < B * K; i += blockDim.x) ent_tok[i] = ld_act_i(&a.ws.entry_tok[i]);
-  __syncthreads();
-
-  const long long total = (long long)U * I;
-  long long q0, q1;
-  split_range(total, G, c, q0, q1);
-  const uint32_t seg = (uint32_t)kc * 2u;
-
-  if (warp == kConsumerWarps) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int it = 0;
-      bool ok = true;
-      for (long long q = q0; q < q1 && ok; q += 4) {
-        const int np = (int)min(4LL, q1 - q);
-        for (int ch = 0; ch < nch; ++ch, ++it) {
-          if (!ring_acquire(empty, it, S, abort_flag, a.ws.err)) { ok = false; break; }
-          const int s = it % S;
-          mbar_arrive_expect_tx(&full[s], 2 * np * seg);
-          for (int i = 0; i < np; ++i) {
-            const int u = (int)((q + i) / I), p = (int)((q + i) % I);
-            const uint16_t* base = a.w_gu + ((size_t)un_e[u] * 2 * I + p) * d + (size_t)ch * kc;
-            bulk_g2s(ring + s * SB + i * wp, base, seg, &full[s], pol);
-            bulk_g2s(ring + s * SB + (4 + i) * wp, base + (size_t)I * d, seg, &full[s], pol);
-          }
-        }
-      }
-      ring_drain(full, it, S, a.ws.err);
-    }
-  } else {
-    // x of every token as (hi, lo) bf16 rows.
-    const int cpr = d / 8;
-    for (int z = tid; z < B * cpr; z += kConsumerThreads) {
-      const int t = z / cpr, qq = z % cpr;
-      const float* xp = a.ws.x + (size_t)t * d + (size_t)qq * 8;
-      const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
-      const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      uint16_t xh[8], xl[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) split_bf16(xv[e], xh[e], xl[e]);
-      uint4 ph, pl;
-      ph.x = xh[0] | ((uint32_t)xh[1] << 16); ph.y = xh[2] | ((uint32_t)xh[3] << 16);
-      ph.z = xh[4] | ((uint32_t)xh[5] << 16); ph.w = xh[6] | ((uint32_t)xh[7] << 16);
-      pl.x = xl[0] | ((uint32_t)xl[1] << 16); pl.y = xl[2] | ((uint32_t)xl[3] << 16);
-      pl.z = xl[4] | ((uint32_t)xl[5] << 16); pl.w = xl[6] | ((uint32_t)xl[7] << 16);
-      *reinterpret_cast<uint4*>(act + (size_t)(2 * t) * ap + (size_t)qq * 16) = ph;
-      *reinterpret_cast<uint4*>(act + (size_t)(2 * t + 1) * ap + (size_t)qq * 16) = pl;
-    }
-    consumer_sync();
-    const int S_k = kc / 16;
-    int s0, s1;
-    warp_steps(S_k, warp, s0, s1);
-    int it = 0;
-    for (long long q = q0; q < q1; q += 4) {
-      const int np = (int)min(4LL, q1 - q);
-      float dacc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int ch = 0; ch < nch; ++ch, ++it) {
-        const int s = it % S;
-        mbar_wait(&full[s], (it / S) & 1, abort_flag, a.ws.err);
-        mma_stage(dacc, ring + s * SB, wp, act, ap, 2 * B, ch * kc, s0, s1, lane);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-      }
-      mma_store_partial(red, dacc, 2 * B, warp, lane);
-      consumer_sync();
-      for (int z = tid; z < np * B; z += kConsumerThreads) {
-        const int i = z / B, t = z % B;
-        const int u = (int)((q + i) / I), p = (int)((q + i) % I);
-        const float gs = mma_reduce(red, 2 * t, i) + mma_reduce(red, 2 * t + 1, i);
-        const float us = mma_reduce(red, 2 * t, 4 + i) + mma_reduce(red, 2 * t + 1, 4 + i);
-        for (int en = un_off[u]; en < un_off[u + 1]; ++en)
-          if (ent_tok[en] == t) a.ws.a[(size_t)en * I + p] = gs / (1.0f + expf(-gs)) * us;
-      }
-      consumer_sync();
-    }
-  }
-}
 // =============================================================================
 // K3 (split-K): expert gate/up for larger batches
 //   unit (u, c): rows 0..2I-1 of expert union_e[u] over K chunk c; tokens in groups of NT.
@@ -1058,18 +569,8 @@ bool plan_layer(LayerArgs& a, int G, size_t optin) {
     if (t.stages < 2) return false;
     t.smem = (size_t)t.stages * SB + act + extra;
   }
-  // K2: the router slice (<= 8 rows) resident in all its K chunks.
-  {
-    KTune& t = a.k2;
-    t.rows_max = (a.E + G - 1) / G;
-    if (t.rows_max > kGroupRows) return false;
-    t.kc = pick_kc(a.d, 34 * 1024);
-    t.nch = a.d / t.kc;
-    const size_t SB = a128((size_t)kGroupRows * (t.kc * 2 + 16));
-    t.smem = (size_t)t.nch * SB + a128((size_t)4 * (a.d * 2 + 16)) + 48 * 1024 + (size_t)t.nch * 8 +
-             kConsumerWarps * 64 * 4 + 64 * 4 + 64;
-    if (t.smem > budget) return false;
-  }
+  // K2 (router, kernels_small.cu): rows of W_r per CTA.
+  a.k2.rows_max = (a.E + G - 1) / G;
   // K3: small-M (tensor cores, batch <= 2) or split-K (row segments of one K chunk).
   {
     KTune& t = a.k3;
@@ -1081,16 +582,6 @@ bool plan_layer(LayerArgs& a, int G, size_t optin) {
       const size_t stage = (size_t)t.rows_per_stage * seg;
       t.stages = (int)std::min<size_t>(kMaxStages, (std::min<size_t>(budget, 200 * 1024) - 64) / stage);
       t.smem = (size_t)t.stages * stage + 2 * t.stages * 8 + 16;
-    } else {
-      t.kc = pick_kc(a.d, 34 * 1024);
-      t.nch = a.d / t.kc;
-      const int umax = std::min(a.E, maxB * Kk);
-      const size_t SB = a128((size_t)kGroupRows * (t.kc * 2 + 16));
-      const size_t act = a128((size_t)4 * (a.d * 2 + 16));
-      const size_t extra = a128((size_t)(2 * umax + 1 + maxB * Kk) * 4) + 2 * kMaxStages * 8 +
-                           kConsumerWarps * 64 * 4 + 64 + 128;
-      t.stages = (int)std::min<size_t>(kMaxStages, (budget - act - extra) / SB);
-      t.smem = (size_t)t.stages * SB + act + extra;
     }
     if (t.stages < 2) return false;
   }
@@ -1111,7 +602,7 @@ bool plan_layer(LayerArgs& a, int G, size_t optin) {
     if (t.stages < 2) return false;
     t.smem = (size_t)t.stages * SB + fixed + (t.a_in_smem ? a_bytes : 0);
   }
-  return a.k1.smem <= budget && a.k2.smem <= budget && a.k3.smem <= budget && a.k4.smem <= budget;
+  return a.k1.smem <= budget && a.k3.smem <= budget && a.k4.smem <= budget;
 }
 
 cudaError_t set_kernel_attributes(size_t optin) {
@@ -1121,12 +612,8 @@ cudaError_t set_kernel_attributes(size_t optin) {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, v); \
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100)
   SET(k_oproj);
-  SET(k_router_topk);
-  SET(k_gateup_small);
   SET(k_gateup_splitk<2>);
   SET(k_down_combine<0>);
-  SET(k_down_combine<1>);
-  SET(k_down_combine<2>);
 #undef SET
   return e;
 }
@@ -1135,22 +622,11 @@ cudaError_t launch_oproj(const LayerArgs& a, int grid, cudaStream_t s, bool pdl)
   return launch_k(k_oproj, grid, a.k1.smem, s, pdl, a);
 }
 
-cudaError_t launch_router(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
-  return launch_k(k_router_topk, grid, a.k2.smem, s, pdl, a);
-}
-
-cudaError_t launch_gateup_small(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
-  if (a.B > 2) return cudaErrorInvalidValue;  // small-M covers batch 1 and 2
-  return launch_k(k_gateup_small, grid, a.k3.smem, s, pdl, a);
-}
-
 cudaError_t launch_gateup_splitk(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
   return launch_k(k_gateup_splitk<2>, grid, a.k3.smem, s, pdl, a);
 }
 
 cudaError_t launch_down(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
-  if (a.B == 1) return launch_k(k_down_combine<1>, grid, a.k4.smem, s, pdl, a);
-  if (a.B == 2) return launch_k(k_down_combine<2>, grid, a.k4.smem, s, pdl, a);
   return launch_k(k_down_combine<0>, grid, a.k4.smem, s, pdl, a);
 }
 

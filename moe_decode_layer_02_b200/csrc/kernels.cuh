@@ -49,6 +49,7 @@ struct LayerArgs {
   uint16_t* out;          // [B][d]
   int* user_idx;          // [B][k] or null
   float* user_gate;       // [B][k] or null
+  int route_tables;       // the router's last CTA builds the global routing tables
   Workspace ws;
   KTune k1, k2, k3, k4;
 };
@@ -64,11 +65,20 @@ bool plan_layer(LayerArgs& a, int num_sms, size_t smem_optin);
 
 // Launchers (pdl: launch with programmatic stream serialisation).
 cudaError_t launch_oproj(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
-cudaError_t launch_router(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
-cudaError_t launch_gateup_small(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_gateup_splitk(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_down(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_prefetch(const PrefetchArgs& p, int grid, cudaStream_t s);
+
+// Small-batch kernels and the router (kernels_small.cu): whole rows streamed by TMA.
+bool plan_small(LayerArgs& a, int grid, size_t smem_optin);
+bool small_path_ok(const LayerArgs& a, size_t smem_optin);   // o_proj, gate/up, down at batch <= 2
+bool oproj_small_ok(const LayerArgs& a, size_t smem_optin);
+bool router_ok(const LayerArgs& a, size_t smem_optin);       // router at this batch
+cudaError_t set_small_attributes(size_t smem_optin);
+cudaError_t launch_oproj_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
+cudaError_t launch_router_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
+cudaError_t launch_gateup_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
+cudaError_t launch_down_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t set_kernel_attributes(size_t smem_optin);
 
 }  // namespace moe

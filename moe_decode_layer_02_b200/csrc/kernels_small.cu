@@ -1,0 +1,708 @@
+// Small-batch kernels: whole weight rows streamed by TMA, fp32 dot products.
+//
+// A decode step at batch 1-2 reads 218-306 MB of weights and does about one flop per
+// byte, so every kernel here is a weight stream.  What limits it is keeping enough bytes
+// in flight with few expensive operations:
+//   * the producer warp moves weights with one 1-D bulk copy per stage of whole,
+//     contiguous rows (12-56 KB per copy; each bulk copy has a fixed issue cost of the
+//     order of a hundred nanoseconds, so many small copies cannot feed an SM);
+//   * a ring of up to 8 stages keeps ~100-200 KB in flight per SM;
+//   * the 8 consumer warps split K: each holds its slice of the activations in registers
+//     as fp32 (exact; x is not rounded for the router), reads 16-byte weight chunks from
+//     shared memory (lanes contiguous, conflict-free) and accumulates in fp32;
+//   * row partials go to shared memory and are reduced once, in a fixed order, at the end.
+// No grid-wide synchronisation: RMSNorm statistics are per-CTA partial sums that the router
+// reduces itself, and the top-k selection and routing are recomputed in every expert CTA.
+//
+//   k_oproj_f    h = residual + W_o . attn_out, per-CTA sums of h^2            (batch <= 2)
+//   k_router_f   rstd, x = h * rstd * gamma, logits = W_r . x   (any batch; at batch >= 3
+//                the last CTA also builds the global routing tables)
+//   k_gateup_f   routing per CTA, then a = silu(W_g x) * (W_u x) for each (selected expert,
+//                row pair), each pair streamed once                            (batch <= 2)
+//   k_down_f     routing per CTA, then out = bf16(h + sum_j gate_j * W_down[e_j] . a_j);
+//                every lane accumulates its share of a row over all experts in registers
+//                and reduces once                                              (batch <= 2)
+//
+// Weights are static, so producers issue their first copies before the programmatic-
+// launch dependency wait; activations are read only after it, with L2 loads.
+//
+// Sources: "vLLM speeds up Kimi K3 up to 1.9x on NVIDIA GB300 with agent-assisted
+// kernels", section "How the specialised decode path works" (small-matrix kernels at
+// batch one or two; o_proj fused with the residual step; 16 of 896 experts per token).
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "topk.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kCPLf = 4;  // 8-element chunks per lane: K <= 8 warps * 32 lanes * 4 * 8 = 8192
+
+__device__ __forceinline__ size_t al128(size_t x) { return (x + 127) & ~size_t(127); }
+
+__device__ __forceinline__ void unpack8f(uint4 w, float* f) {
+  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
+  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
+}
+
+// Chunk of lane `lane` in warp w's K slice: q = w * qpw + j * 32 + lane, valid if j*32+lane < qpw.
+__device__ __forceinline__ bool cvalid(int qpw, int j, int lane) { return j * 32 + lane < qpw; }
+
+// Dot of one bf16 row (shared memory) with NT register slices; two accumulators per token.
+template <int NT>
+__device__ __forceinline__ void row_dot(const uint16_t* row, const float (&x)[NT][kCPLf][8], int qbase, int qpw,
+                                        int lane, float (&out)[NT]) {
+  float acc0[NT], acc1[NT];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) acc0[t] = acc1[t] = 0.f;
+#pragma unroll
+  for (int j = 0; j < kCPLf; ++j) {
+    if (!cvalid(qpw, j, lane)) continue;
+    const uint4 w = *reinterpret_cast<const uint4*>(row + (size_t)(qbase + j * 32 + lane) * 8);
+    float wf[8];
+    unpack8f(w, wf);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float& acc = (j & 1) ? acc1[t] : acc0[t];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc = fmaf(wf[e], x[t][j][e], acc);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t) out[t] = acc0[t] + acc1[t];
+}
+
+}  // namespace
+
+// =============================================================================
+// K1: o_proj + residual + per-CTA sums of h^2 (batch <= 2)
+//   CTA c owns rows [r0, r1) of W_o (contiguous); a stage is RS whole rows (one copy).
+// =============================================================================
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1) k_oproj_f(const LayerArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int G = gridDim.x, c = blockIdx.x;
+  const int d = a.d, d_o = a.d_o, B = a.B;
+  const int S = a.k1.stages, RS = a.k1.rows_per_stage, RM = a.k1.rows_max;
+  const uint32_t row_bytes = (uint32_t)d_o * 2u;
+  const size_t SB = al128((size_t)RS * row_bytes);
+  long long lo, hi;
+  split_range(d, G, c, lo, hi);
+  const int r0 = (int)lo, r1 = (int)hi, rows = r1 - r0;
+
+  unsigned char* ring = smem;
+  float* part = reinterpret_cast<float*>(ring + (size_t)S * SB);  // [RM][8][NT]
+  float* sq = part + RM * kConsumerWarps * NT;                     // [NT][RM]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + al128((size_t)S * SB + ((size_t)RM * kConsumerWarps * NT +
+                                                                              (size_t)NT * RM) * 4));
+  uint64_t* empty = full + S;
+  int* s_misc = reinterpret_cast<int*>(empty + S);
+  volatile int* abort_flag = s_misc;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  if (tid == 0) {
+    init_ring(full, empty, S);
+    s_misc[0] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_trigger();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {  // W_o is static: stream it before the dependency resolves
+      const uint64_t pol = policy_evict_first();
+      int it = 0;
+      for (int r = r0; r < r1; r += RS, ++it) {
+        const int n = min(RS, r1 - r);
+        if (!ring_acquire(empty, it, S, abort_flag, a.ws.err)) break;
+        const int s = it % S;
+        mbar_arrive_expect_tx(&full[s], n * row_bytes);
+        bulk_g2s(ring + s * SB, a.w_o + (size_t)r * d_o, n * row_bytes, &full[s], pol);
+      }
+      ring_drain(full, it, S, a.ws.err);
+    }
+    return;
+  }
+
+  pdl_wait();  // attn_out and residual may come from the previous kernel
+  const int qpw = d_o / 64, qbase = warp * qpw;
+  float xa[NT][kCPLf][8];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int j = 0; j < kCPLf; ++j) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (t < B && cvalid(qpw, j, lane)) u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)(qbase + j * 32 + lane) * 8);
+      unpack8f(u, xa[t][j]);
+    }
+  int it = 0;
+  for (int r = r0; r < r1; r += RS, ++it) {
+    const int n = min(RS, r1 - r), s = it % S;
+    mbar_wait(&full[s], (it / S) & 1, abort_flag, a.ws.err);
+    const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB);
+    for (int j = 0; j < n; ++j) {
+      float v[NT];
+      row_dot<NT>(st + (size_t)j * d_o, xa, qbase, qpw, lane, v);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const float w = warp_sum(v[t]);
+        if (lane == 0) part[((r - r0 + j) * kConsumerWarps + warp) * NT + t] = w;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+  consumer_sync();
+  for (int z = tid; z < rows * B; z += kConsumerThreads) {
+    const int rr = z / B, t = z % B;
+    float sacc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) sacc += part[(rr * kConsumerWarps + w) * NT + t];
+    const size_t o = (size_t)t * d + r0 + rr;
+    const float hv = bf16f(__ldcg(reinterpret_cast<const unsigned short*>(a.resid + o))) + sacc;
+    a.ws.h[o] = hv;
+    sq[t * RM + rr] = hv * hv;
+  }
+  consumer_sync();
+  if (warp < B) {  // per-CTA sum of h^2, fixed order
+    float ss = 0.f;
+    for (int rr = lane; rr < rows; rr += 32) ss += sq[warp * RM + rr];
+    ss = warp_sum(ss);
+    if (lane == 0) a.ws.ss_part[(size_t)c * a.maxB + warp] = ss;
+  }
+}
+
+// =============================================================================
+// K2: RMSNorm apply + router GEMV (any batch, tokens in groups of NT)
+//   CTA c owns rows [e0, e0 + nrows) of W_r: the whole slice is one bulk copy, issued before
+//   the dependency wait.  x is exact fp32 in registers.
+// =============================================================================
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int G = gridDim.x, c = blockIdx.x;
+  const int d = a.d, E = a.E, B = a.B;
+  const int RM = a.k2.rows_max;
+  long long lo, hi;
+  split_range(E, G, c, lo, hi);
+  const int e0 = (int)lo, nrows = (int)(hi - lo);
+  const uint32_t row_bytes = (uint32_t)d * 2u;
+
+  uint16_t* wsl = reinterpret_cast<uint16_t*>(smem);                                 // [RM][d]
+  float* part = reinterpret_cast<float*>(smem + al128((size_t)RM * row_bytes));    // [RM][8][NT]
+  float* rstd_s = part + RM * kConsumerWarps * NT;                                  // [64]
+  uint64_t* full = reinterpret_cast<uint64_t*>(
+      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(rstd_s + 64) - smem)));
+  int* s_misc = reinterpret_cast<int*>(full + 1);
+  unsigned char* scratch = reinterpret_cast<unsigned char*>(s_misc + 32);          // routing tables
+  volatile int* abort_flag = s_misc;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  if (tid == 0) {
+    init_ring(full, nullptr, 1);
+    s_misc[0] = 0;
+    s_misc[1] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_trigger();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0 && nrows > 0) {
+      mbar_arrive_expect_tx(&full[0], nrows * row_bytes);
+      bulk_g2s(wsl, a.w_r + (size_t)e0 * d, nrows * row_bytes, &full[0], policy_evict_first());
+      mbar_drain(&full[0], 0, a.ws.err);
+    }
+  } else {
+    const int qpw = d / 64, qbase = warp * qpw;
+    float gam[kCPLf][8];
+#pragma unroll
+    for (int j = 0; j < kCPLf; ++j) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (cvalid(qpw, j, lane)) u = ld_weight_u4(a.gamma + (size_t)(qbase + j * 32 + lane) * 8);
+      unpack8f(u, gam[j]);
+    }
+    pdl_wait();  // h and the sums of h^2 come from the o_proj kernel
+    for (int t = warp; t < B; t += kConsumerWarps) {  // fixed order: same bits in every CTA
+      float ss = 0.f;
+      for (int cc = lane; cc < G; cc += 32) ss += ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]);
+      ss = warp_sum(ss);
+      if (lane == 0) {
+        const float r = 1.0f / sqrtf(ss / (float)d + a.eps);
+        rstd_s[t] = r;
+        if (c == 0) a.ws.rstd[t] = r;
+      }
+    }
+    consumer_sync();
+    bool have_w = false;
+    for (int t0 = 0; t0 < B; t0 += NT) {
+      const int nt = min(NT, B - t0);
+      float xr[NT][kCPLf][8];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const float r = (t < nt) ? rstd_s[t0 + t] : 0.f;
+#pragma unroll
+        for (int j = 0; j < kCPLf; ++j) {
+          const int q = qbase + j * 32 + lane;
+          if (t < nt && cvalid(qpw, j, lane)) {
+            const float* hp = a.ws.h + (size_t)(t0 + t) * d + (size_t)q * 8;
+            const float4 h0 = ld_act4(hp), h1 = ld_act4(hp + 4);
+            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[t][j][e] = hv[e] * r * gam[j][e];
+            if (q % G == c) {  // each chunk of x is written to global memory by exactly one CTA
+              float* xp = a.ws.x + (size_t)(t0 + t) * d + (size_t)q * 8;
+              *reinterpret_cast<float4*>(xp) = make_float4(xr[t][j][0], xr[t][j][1], xr[t][j][2], xr[t][j][3]);
+              *reinterpret_cast<float4*>(xp + 4) = make_float4(xr[t][j][4], xr[t][j][5], xr[t][j][6], xr[t][j][7]);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+          }
+        }
+      }
+      if (nrows > 0) {
+        if (!have_w) {
+          mbar_wait(&full[0], 0, abort_flag, a.ws.err);
+          have_w = true;
+        }
+        for (int j = 0; j < nrows; ++j) {
+          float v[NT];
+          row_dot<NT>(wsl + (size_t)j * d, xr, qbase, qpw, lane, v);
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            const float w = warp_sum(v[t]);
+            if (lane == 0) part[(j * kConsumerWarps + warp) * NT + t] = w;
+          }
+        }
+      }
+      consumer_sync();
+      for (int z = tid; z < nrows * nt; z += kConsumerThreads) {
+        const int j = z / nt, t = z % nt;
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) s += part[(j * kConsumerWarps + w) * NT + t];
+        a.ws.logits[(size_t)(t0 + t) * E + e0 + j] = s;
+      }
+      consumer_sync();
+    }
+  }
+  if (a.route_tables) {  // large-batch expert kernels: the last CTA builds the routing tables
+    if (last_cta_s(&a.ws.counters[kCntRouter], &s_misc[1])) {
+      topk_route(a, scratch);
+      if (tid == 0) a.ws.counters[kCntRouter] = 0;
+    }
+  }
+}
+
+// =============================================================================
+// K3 (batch <= 2): routing per CTA, then expert gate/up + SiLU*mul
+//   Pairs (union expert u, row p) in flattened order; CTA c takes [q0, q1).  A stage is up to
+//   PS consecutive pairs of one expert: its gate rows and its up rows (two copies).
+// =============================================================================
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1) k_gateup_f(const LayerArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int G = gridDim.x, c = blockIdx.x;
+  const int d = a.d, I = a.I, B = a.B;
+  const int S = a.k3.stages, PS = a.k3.rows_per_stage;  // pairs per stage
+  const uint32_t row_bytes = (uint32_t)d * 2u;
+  const size_t SB = al128((size_t)2 * PS * row_bytes);
+  const int PM = a.k3.rows_max;  // max pairs per CTA
+
+  unsigned char* ring = smem;
+  float* part = reinterpret_cast<float*>(ring + (size_t)S * SB);  // [PM][2][8][NT]
+  SmallRoute* rt = reinterpret_cast<SmallRoute*>(part + PM * 2 * kConsumerWarps * NT);
+  RouteScratch* sc = reinterpret_cast<RouteScratch*>(rt + 1);
+  float* fb = reinterpret_cast<float*>(sc + 1);  // fallback top-k scratch: 2 warps x 2 arrays
+  uint64_t* full = reinterpret_cast<uint64_t*>(
+      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + 2 * 2 * kCandStride) - smem)));
+  uint64_t* empty = full + S;
+  int* s_misc = reinterpret_cast<int*>(empty + S);
+  volatile int* abort_flag = s_misc;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  if (tid == 0) {
+    init_ring(full, empty, S);
+    s_misc[0] = 0;
+    fence_barrier_init();
+  }
+  pdl_wait();  // logits and x come from the router kernel
+  // Dependents may launch only now: the down kernel reads the logits before its own wait.
+  pdl_trigger();
+  route_small_cta(a, rt, sc, fb, c == 0);  // contains __syncthreads (also covers the init)
+
+  const int U = rt->U;
+  long long q0l, q1l;
+  split_range((long long)U * I, G, c, q0l, q1l);
+  const int q0 = (int)q0l, q1 = (int)q1l;
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int it = 0;
+      int u = q0 / I, p = q0 - u * I;
+      for (int q = q0; q < q1; ++it) {
+        const int np = min(min(PS, I - p), q1 - q);
+        if (!ring_acquire(empty, it, S, abort_flag, a.ws.err)) break;
+        const int s = it % S;
+        const uint16_t* base = a.w_gu + ((size_t)rt->un_e[u] * 2 * I + p) * d;
+        mbar_arrive_expect_tx(&full[s], 2u * np * row_bytes);
+        bulk_g2s(ring + s * SB, base, np * row_bytes, &full[s], pol);
+        bulk_g2s(ring + s * SB + (size_t)PS * row_bytes, base + (size_t)I * d, np * row_bytes, &full[s], pol);
+        q += np;
+        p += np;
+        if (p == I) { p = 0; ++u; }
+      }
+      ring_drain(full, it, S, a.ws.err);
+    }
+    return;
+  }
+
+  const int qpw = d / 64, qbase = warp * qpw;
+  float xr[NT][kCPLf][8];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int j = 0; j < kCPLf; ++j) {
+      if (t < B && cvalid(qpw, j, lane)) {
+        const float* xp = a.ws.x + (size_t)t * d + (size_t)(qbase + j * 32 + lane) * 8;
+        const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
+        xr[t][j][0] = x0.x; xr[t][j][1] = x0.y; xr[t][j][2] = x0.z; xr[t][j][3] = x0.w;
+        xr[t][j][4] = x1.x; xr[t][j][5] = x1.y; xr[t][j][6] = x1.z; xr[t][j][7] = x1.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+      }
+    }
+  int it = 0;
+  int p = q0 - (q0 / I) * I;
+  for (int q = q0; q < q1; ++it) {
+    const int np = min(min(PS, I - p), q1 - q), s = it % S;
+    mbar_wait(&full[s], (it / S) & 1, abort_flag, a.ws.err);
+    const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB);
+    for (int i = 0; i < 2 * np; ++i) {  // gate rows 0..np-1, then up rows
+      const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
+      float v[NT];
+      row_dot<NT>(st + (size_t)(gu * PS + pi) * d, xr, qbase, qpw, lane, v);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const float w = warp_sum(v[t]);
+        if (lane == 0) part[(((q - q0 + pi) * 2 + gu) * kConsumerWarps + warp) * NT + t] = w;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    q += np;
+    p += np;
+    if (p == I) p = 0;
+  }
+  consumer_sync();
+  for (int z = tid; z < (q1 - q0) * B; z += kConsumerThreads) {
+    const int pl = z / B, t = z % B;
+    float gs = 0.f, us = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      gs += part[((pl * 2 + 0) * kConsumerWarps + w) * NT + t];
+      us += part[((pl * 2 + 1) * kConsumerWarps + w) * NT + t];
+    }
+    const int qq = q0 + pl, u = qq / I, pp = qq - u * I;
+    for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+      if (rt->ent_tok[en] == t) a.ws.a[(size_t)en * I + pp] = gs / (1.0f + expf(-gs)) * us;
+  }
+}
+
+// =============================================================================
+// K4 (batch <= 2): routing per CTA, then expert down projection + combine
+//   CTA c owns output rows [i0, i1); a stage is those rows of one union expert (contiguous).
+//   Warp w owns rows w, w + 8, ...; lane l the elements [l*EPL, (l+1)*EPL) of each row.
+// =============================================================================
+template <int NT, int EPL>
+__global__ void __launch_bounds__(kThreads, 1) k_down_f(const LayerArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int kRPW = 7;  // rows per warp (rows_max <= 56)
+  const int G = gridDim.x, c = blockIdx.x;
+  const int d = a.d, I = a.I, B = a.B;
+  const int S = a.k4.stages, RM = a.k4.rows_max;
+  long long lo, hi;
+  split_range(d, G, c, lo, hi);
+  const int i0 = (int)lo, nrows = (int)(hi - lo);
+  const uint32_t row_bytes = (uint32_t)I * 2u;
+  const size_t SB = al128((size_t)RM * row_bytes);
+
+  unsigned char* ring = smem;
+  float* a_s = reinterpret_cast<float*>(ring + (size_t)S * SB);  // [n_ent][I], gate-scaled
+  SmallRoute* rt = reinterpret_cast<SmallRoute*>(a_s + (size_t)B * a.k * I);
+  RouteScratch* sc = reinterpret_cast<RouteScratch*>(rt + 1);
+  float* fb = reinterpret_cast<float*>(sc + 1);
+  uint64_t* full = reinterpret_cast<uint64_t*>(
+      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + 2 * 2 * kCandStride) - smem)));
+  uint64_t* empty = full + S;
+  int* s_misc = reinterpret_cast<int*>(empty + S);
+  volatile int* abort_flag = s_misc;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  if (tid == 0) {
+    init_ring(full, empty, S);
+    s_misc[0] = 0;
+    fence_barrier_init();
+  }
+  // The logits were complete before this grid could launch: the gate/up kernel allows its
+  // dependents to launch only after its own dependency wait, which returns once the router
+  // kernel has finished.
+  route_small_cta(a, rt, sc, fb, false);
+  const int U = rt->U;
+  pdl_trigger();
+
+  if (warp == kConsumerWarps) {
+    if (lane == 0 && nrows > 0) {  // W_down is static: stream it before the dependency wait
+      const uint64_t pol = policy_evict_first();
+      int it = 0;
+      for (int u = 0; u < U; ++u, ++it) {
+        if (!ring_acquire(empty, it, S, abort_flag, a.ws.err)) break;
+        const int s = it % S;
+        mbar_arrive_expect_tx(&full[s], nrows * row_bytes);
+        bulk_g2s(ring + s * SB, a.w_down + ((size_t)rt->un_e[u] * d + i0) * I, nrows * row_bytes, &full[s], pol);
+      }
+      ring_drain(full, it, S, a.ws.err);
+    }
+    return;
+  }
+
+  pdl_wait();  // the SwiGLU activations come from the gate/up kernel
+  const int nent = rt->n_ent;
+  for (int z = tid; z < nent * (I / 4); z += kConsumerThreads) {
+    const int en = z / (I / 4), cq = z % (I / 4);
+    const float g = rt->ent_gate[en];
+    const float4 v = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
+    *reinterpret_cast<float4*>(a_s + (size_t)en * I + cq * 4) = make_float4(g * v.x, g * v.y, g * v.z, g * v.w);
+  }
+  consumer_sync();
+
+  const int epl = (EPL > 0) ? EPL : I / 32;
+  float acc[kRPW][NT];
+#pragma unroll
+  for (int i = 0; i < kRPW; ++i)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[i][t] = 0.f;
+  for (int u = 0; u < U && nrows > 0; ++u) {
+    const int s = u % S;
+    mbar_wait(&full[s], (u / S) & 1, abort_flag, a.ws.err);
+    const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB);
+    for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en) {
+      const int t = rt->ent_tok[en];
+      float av[EPL > 0 ? EPL : 16];
+      const float* ap = a_s + (size_t)en * I + lane * epl;
+      if constexpr (EPL == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(ap);
+        av[0] = v.x; av[1] = v.y; av[2] = v.z; av[3] = v.w;
+      } else if constexpr (EPL == 8) {
+        const float4 v0 = *reinterpret_cast<const float4*>(ap), v1 = *reinterpret_cast<const float4*>(ap + 4);
+        av[0] = v0.x; av[1] = v0.y; av[2] = v0.z; av[3] = v0.w; av[4] = v1.x; av[5] = v1.y; av[6] = v1.z; av[7] = v1.w;
+      } else {
+#pragma unroll
+        for (int x = 0; x < 16; ++x) av[x] = (x < epl) ? ap[x] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kRPW; ++i) {
+        const int rl = warp + kConsumerWarps * i;
+        if (rl < nrows) {
+          const uint16_t* wr = st + (size_t)rl * I + lane * epl;
+          float sdot = 0.f;
+          if constexpr (EPL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(wr);
+            sdot = fmaf(bf16lo(w.x), av[0], sdot);
+            sdot = fmaf(bf16hi(w.x), av[1], sdot);
+            sdot = fmaf(bf16lo(w.y), av[2], sdot);
+            sdot = fmaf(bf16hi(w.y), av[3], sdot);
+          } else if constexpr (EPL == 8) {
+            const uint4 w = *reinterpret_cast<const uint4*>(wr);
+            float wf[8];
+            unpack8f(w, wf);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) sdot = fmaf(wf[x], av[x], sdot);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+              if (x < epl) sdot = fmaf(bf16f(wr[x]), av[x], sdot);
+          }
+#pragma unroll
+          for (int tt = 0; tt < NT; ++tt)
+            if (tt == t) acc[i][tt] += sdot;
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+#pragma unroll
+  for (int i = 0; i < kRPW; ++i) {
+    const int rl = warp + kConsumerWarps * i;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const float v = warp_sum(acc[i][t]);
+      if (lane == 0 && rl < nrows && t < B) {
+        const size_t o = (size_t)t * d + i0 + rl;
+        const __nv_bfloat16 bv = __float2bfloat16_rn(ld_act(&a.ws.h[o]) + v);
+        a.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
+      }
+    }
+  }
+}
+
+// =============================================================================
+// Host side
+// =============================================================================
+namespace {
+
+template <typename Kern>
+cudaError_t launch_f(Kern k, int grid, size_t smem, cudaStream_t s, bool pdl, const LayerArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, a);
+}
+
+size_t up128(size_t x) { return (x + 127) & ~size_t(127); }
+constexpr size_t kRouteBytes = sizeof(SmallRoute) + sizeof(RouteScratch) + 2 * 2 * kCandStride * 4 + 128;
+constexpr size_t kRingCap = 200 * 1024;
+
+}  // namespace
+
+bool plan_small(LayerArgs& a, int G, size_t optin) {
+  const size_t budget = optin - 1024 - 256;
+  const int NT = 2;
+  {  // K1: whole rows of W_o, ~32 KB stages
+    KTune& t = a.k1;
+    const size_t row = (size_t)a.d_o * 2;
+    t.rows_max = (a.d + G - 1) / G;
+    t.rows_per_stage = (int)std::max<size_t>(1, std::min<size_t>(32768 / row, (size_t)t.rows_max));
+    const size_t SB = up128((size_t)t.rows_per_stage * row);
+    const size_t extra = up128(((size_t)t.rows_max * kConsumerWarps * NT + (size_t)NT * t.rows_max) * 4) +
+                         2 * kMaxStages * 8 + 64;
+    t.stages = (int)std::min<size_t>(kMaxStages, (std::min(budget, kRingCap) - extra) / SB);
+    if (t.stages < 2) return false;
+    t.smem = (size_t)t.stages * SB + extra;
+  }
+  {  // K2: the whole router slice
+    KTune& t = a.k2;
+    t.rows_max = (a.E + G - 1) / G;
+    t.smem = up128((size_t)t.rows_max * a.d * 2) + up128((size_t)t.rows_max * kConsumerWarps * NT * 4 + 64 * 4) +
+             8 + 32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
+    if (t.smem > budget) return false;
+  }
+  {  // K3: pairs of gate/up rows
+    KTune& t = a.k3;
+    const size_t row = (size_t)a.d * 2;
+    const long long umax = std::min(a.E, std::max(a.B, 1) * a.k);
+    t.rows_max = (int)((umax * a.I + G - 1) / G);  // pairs per CTA
+    const size_t extra = (size_t)t.rows_max * 2 * kConsumerWarps * NT * 4 + kRouteBytes + 2 * kMaxStages * 8 + 64;
+    t.stages = 0;
+    for (int ps = 2; ps >= 1 && t.stages < 2; --ps) {
+      t.rows_per_stage = ps;
+      const size_t SB = up128((size_t)2 * ps * row);
+      t.stages = extra < budget ? (int)std::min<size_t>(kMaxStages, (budget - extra) / SB) : 0;
+      t.smem = (size_t)t.stages * SB + extra;
+    }
+    if (t.stages < 2) return false;
+  }
+  {  // K4: one expert's rows per stage
+    KTune& t = a.k4;
+    t.rows_max = (a.d + G - 1) / G;
+    if (t.rows_max > 7 * kConsumerWarps) return false;
+    const size_t SB = up128((size_t)t.rows_max * a.I * 2);
+    const size_t extra = (size_t)std::max(a.B, 1) * a.k * a.I * 4 + kRouteBytes + 2 * kMaxStages * 8 + 64;
+    t.stages = extra < budget ? (int)std::min<size_t>(kMaxStages, (budget - extra) / SB) : 0;
+    if (t.stages < 2) return false;
+    t.smem = (size_t)t.stages * SB + extra;
+  }
+  return true;
+}
+
+bool small_path_ok(const LayerArgs& a0, size_t optin) {
+  LayerArgs a = a0;
+  return a.B <= 2 && a.k <= 32 && a.d <= 8192 && a.d_o <= 8192 && plan_small(a, 148, optin);
+}
+
+bool oproj_small_ok(const LayerArgs& a, size_t optin) { return small_path_ok(a, optin); }
+
+bool router_ok(const LayerArgs& a0, size_t optin) {
+  LayerArgs a = a0;
+  const int G = 148;
+  KTune& t = a.k2;
+  t.rows_max = (a.E + G - 1) / G;
+  t.smem = up128((size_t)t.rows_max * a.d * 2) + up128((size_t)t.rows_max * kConsumerWarps * 2 * 4 + 64 * 4) + 8 +
+           32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
+  return a.d <= 8192 && t.smem <= optin - 1024 - 256;
+}
+
+cudaError_t set_small_attributes(size_t optin) {
+  const int v = (int)optin;
+  cudaError_t e = cudaSuccess;
+#define SETS(k)                                                                                              \
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, v); \
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100)
+  SETS(k_oproj_f<1>);
+  SETS(k_oproj_f<2>);
+  SETS(k_router_f<1>);
+  SETS(k_router_f<2>);
+  SETS(k_gateup_f<1>);
+  SETS(k_gateup_f<2>);
+  SETS((k_down_f<1, 4>));
+  SETS((k_down_f<2, 4>));
+  SETS((k_down_f<1, 8>));
+  SETS((k_down_f<2, 8>));
+  SETS((k_down_f<1, 0>));
+  SETS((k_down_f<2, 0>));
+#undef SETS
+  return e;
+}
+
+namespace {
+LayerArgs planned(const LayerArgs& a0, int grid, size_t optin) {
+  LayerArgs a = a0;
+  plan_small(a, grid, optin);
+  return a;
+}
+}  // namespace
+
+cudaError_t launch_oproj_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
+  const LayerArgs a = planned(a0, grid, optin);
+  return a.B == 1 ? launch_f(k_oproj_f<1>, grid, a.k1.smem, s, pdl, a) : launch_f(k_oproj_f<2>, grid, a.k1.smem, s, pdl, a);
+}
+
+cudaError_t launch_router_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
+  LayerArgs a = a0;
+  a.k2.rows_max = (a.E + grid - 1) / grid;
+  a.k2.smem = up128((size_t)a.k2.rows_max * a.d * 2) + up128((size_t)a.k2.rows_max * kConsumerWarps * 2 * 4 + 64 * 4) +
+              8 + 32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
+  (void)optin;
+  return a.B == 1 ? launch_f(k_router_f<1>, grid, a.k2.smem, s, pdl, a) : launch_f(k_router_f<2>, grid, a.k2.smem, s, pdl, a);
+}
+
+cudaError_t launch_gateup_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
+  const LayerArgs a = planned(a0, grid, optin);
+  return a.B == 1 ? launch_f(k_gateup_f<1>, grid, a.k3.smem, s, pdl, a) : launch_f(k_gateup_f<2>, grid, a.k3.smem, s, pdl, a);
+}
+
+cudaError_t launch_down_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
+  const LayerArgs a = planned(a0, grid, optin);
+  const int epl = a.I / 32;
+  if (epl == 4)
+    return a.B == 1 ? launch_f(k_down_f<1, 4>, grid, a.k4.smem, s, pdl, a) : launch_f(k_down_f<2, 4>, grid, a.k4.smem, s, pdl, a);
+  if (epl == 8)
+    return a.B == 1 ? launch_f(k_down_f<1, 8>, grid, a.k4.smem, s, pdl, a) : launch_f(k_down_f<2, 8>, grid, a.k4.smem, s, pdl, a);
+  return a.B == 1 ? launch_f(k_down_f<1, 0>, grid, a.k4.smem, s, pdl, a) : launch_f(k_down_f<2, 0>, grid, a.k4.smem, s, pdl, a);
+}
+
+}  // namespace moe

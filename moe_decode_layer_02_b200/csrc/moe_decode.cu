@@ -57,7 +57,7 @@ struct moe_decode_handle {
   uint16_t* resid_pp[2] = {nullptr, nullptr};
   // staging for moe_decode_step_host
   void *h_attn = nullptr, *h_resid = nullptr, *h_out = nullptr, *h_idx = nullptr, *h_gate = nullptr;
-  LayerArgs plan_small{}, plan_splitk{};
+  LayerArgs plan_splitk{};
   bool has_splitk = false;
   cudaStream_t cap = nullptr, side = nullptr;
   std::vector<cudaEvent_t> events;
@@ -118,12 +118,26 @@ bool use_splitk(const moe_decode_handle* h, int B) {
   return h->cfg.force_variant == 2;               // small-matrix kernels at batch one or two
 }
 
+// Kernel choice of one layer step.
+struct Variant {
+  bool oproj_small;   // whole-row o_proj (batch <= 2)
+  bool experts_small; // small-M gate/up and down with per-CTA routing (batch <= 2)
+};
+
+Variant variant_of(const moe_decode_handle* h, const LayerArgs& a) {
+  Variant v;
+  v.experts_small = !use_splitk(h, a.B) && small_path_ok(a, h->smem_optin);
+  v.oproj_small = v.experts_small && oproj_small_ok(a, h->smem_optin);
+  return v;
+}
+
 LayerArgs layer_args(const moe_decode_handle* h, int l, int B, const void* attn, const void* resid,
                      void* out, int32_t* idx, float* gate) {
   const moe_decode_config& c = h->cfg;
-  LayerArgs a = use_splitk(h, B) ? h->plan_splitk : h->plan_small;
+  LayerArgs a = h->plan_splitk;
   a.B = B;
   plan_layer(a, h->num_sms, h->smem_optin);  // validated for every batch size at create
+  a.route_tables = variant_of(h, a).experts_small ? 0 : 1;
   a.w_o = static_cast<const uint16_t*>(h->w[l].w_o);
   a.gamma = static_cast<const uint16_t*>(h->w[l].gamma);
   a.w_r = static_cast<const uint16_t*>(h->w[l].w_router);
@@ -137,6 +151,20 @@ LayerArgs layer_args(const moe_decode_handle* h, int l, int B, const void* attn,
   return a;
 }
 
+PrefetchArgs prefetch_args(const moe_decode_handle* h, int l) {
+  const moe_decode_config& c = h->cfg;
+  PrefetchArgs p{};
+  const moe_decode_layer_weights& nw = h->w[l];
+  p.ptr[0] = nw.w_router;
+  p.bytes[0] = (unsigned long long)c.n_experts * c.d * 2;
+  p.ptr[1] = nw.gamma;
+  p.bytes[1] = (unsigned long long)c.d * 2;
+  p.ptr[2] = nw.w_o;
+  p.bytes[2] = std::min<unsigned long long>(kPrefetchWoHead, (unsigned long long)c.d * c.d_o * 2);
+  p.n = 3;
+  return p;
+}
+
 // Records the whole step on h->cap (which is in capture mode).  Returns kernels launched.
 int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid, void* out,
                 int32_t* idx, float* gate, cudaError_t* err) {
@@ -148,30 +176,23 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
   bool forked = false;
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     LayerArgs a = layer_args(h, l, B, attn, resid, out, idx, gate);
-    e = launch_oproj(a, G, h->cap, l > 0);
-    if (e == cudaSuccess) e = launch_router(a, G, h->cap, true);
+    const Variant v = variant_of(h, a);
+    e = v.oproj_small ? launch_oproj_s(a, G, h->cap, l > 0, h->smem_optin) : launch_oproj(a, G, h->cap, l > 0);
+    if (e == cudaSuccess) e = launch_router_s(a, G, h->cap, true, h->smem_optin);
     kernels += 2;
     if (e == cudaSuccess && prefetch && l + 1 < c.n_layers) {
       // Fork: once this layer's router is done, warm L2 with the next layer's
       // router slice, RMSNorm scale and the head of its W_o.
       e = cudaEventRecord(h->events[ev], h->cap);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->events[ev++], 0);
-      PrefetchArgs p{};
-      const moe_decode_layer_weights& nw = h->w[l + 1];
-      p.ptr[0] = nw.w_router;
-      p.bytes[0] = (unsigned long long)c.n_experts * c.d * 2;
-      p.ptr[1] = nw.gamma;
-      p.bytes[1] = (unsigned long long)c.d * 2;
-      p.ptr[2] = nw.w_o;
-      p.bytes[2] = std::min<unsigned long long>(kPrefetchWoHead, (unsigned long long)c.d * c.d_o * 2);
-      p.n = 3;
+      PrefetchArgs p = prefetch_args(h, l + 1);
       if (e == cudaSuccess) e = launch_prefetch(p, G, h->side);
       ++kernels;
       forked = true;
     }
     if (e == cudaSuccess)
-      e = use_splitk(h, B) ? launch_gateup_splitk(a, G, h->cap, true) : launch_gateup_small(a, G, h->cap, true);
-    if (e == cudaSuccess) e = launch_down(a, G, h->cap, true);
+      e = v.experts_small ? launch_gateup_s(a, G, h->cap, true, h->smem_optin) : launch_gateup_splitk(a, G, h->cap, true);
+    if (e == cudaSuccess) e = v.experts_small ? launch_down_s(a, G, h->cap, true, h->smem_optin) : launch_down(a, G, h->cap, true);
     kernels += 2;
   }
   if (e == cudaSuccess && forked) {
@@ -263,21 +284,15 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   base.k = K;
   base.I = I;
   base.eps = cfg->rms_eps;
-  h->plan_small = base;
-  h->plan_small.k3.n_split = 0;
   h->plan_splitk = base;
   h->plan_splitk.k3.n_split = h->n_split;
   h->has_splitk = h->n_split > 0;
   bool ok = h->has_splitk;
   for (int B = 1; B <= maxB && ok; ++B) {
-    LayerArgs t = (B <= 2) ? h->plan_small : h->plan_splitk;
+    LayerArgs t = h->plan_splitk;
     t.B = B;
-    ok = plan_layer(t, G, h->smem_optin);
-    if (ok && B <= 2) {
-      LayerArgs u = h->plan_splitk;
-      u.B = B;
-      ok = plan_layer(u, G, h->smem_optin);
-    }
+    t.route_tables = 1;
+    ok = plan_layer(t, G, h->smem_optin) && router_ok(t, h->smem_optin);
   }
   if (!ok) {
     delete h;
@@ -328,13 +343,13 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   ws.err = (unsigned*)(b + o_err);
   h->resid_pp[0] = (uint16_t*)(b + o_r0);
   h->resid_pp[1] = (uint16_t*)(b + o_r1);
-  h->plan_small.ws = ws;
   h->plan_splitk.ws = ws;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(h->ws_base, 0, off, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e == cudaSuccess) e = set_kernel_attributes(h->smem_optin);
+  if (e == cudaSuccess) e = set_small_attributes(h->smem_optin);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
   for (int i = 0; i < 2 * cfg->n_layers + 2 && e == cudaSuccess; ++i) {
@@ -500,25 +515,21 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
   };
   for (int l = 0; l < c.n_layers; ++l) {
     LayerArgs a = layer_args(h, l, batch, attn_out, residual_in, out, topk_idx, topk_gate);
-    timed(1, s, [&](cudaStream_t st) { return launch_oproj(a, G, st, false); });
-    timed(2, s, [&](cudaStream_t st) { return launch_router(a, G, st, false); });
+    const Variant v = variant_of(h, a);
+    timed(1, s, [&](cudaStream_t st) {
+      return v.oproj_small ? launch_oproj_s(a, G, st, false, h->smem_optin) : launch_oproj(a, G, st, false);
+    });
+    timed(2, s, [&](cudaStream_t st) { return launch_router_s(a, G, st, false, h->smem_optin); });
     if (c.enable_prefetch && c.n_layers > 1 && l + 1 < c.n_layers) {
-      PrefetchArgs p{};
-      const moe_decode_layer_weights& nw = h->w[l + 1];
-      p.ptr[0] = nw.w_router;
-      p.bytes[0] = (unsigned long long)c.n_experts * c.d * 2;
-      p.ptr[1] = nw.gamma;
-      p.bytes[1] = (unsigned long long)c.d * 2;
-      p.ptr[2] = nw.w_o;
-      p.bytes[2] = std::min<unsigned long long>(kPrefetchWoHead, (unsigned long long)c.d * c.d_o * 2);
-      p.n = 3;
+      PrefetchArgs p = prefetch_args(h, l + 1);
       timed(6, s, [&](cudaStream_t st) { return launch_prefetch(p, G, st); });
     }
-    const bool sk = use_splitk(h, batch);
-    timed(sk ? 4 : 3, s, [&](cudaStream_t st) {
-      return sk ? launch_gateup_splitk(a, G, st, false) : launch_gateup_small(a, G, st, false);
+    timed(v.experts_small ? 3 : 4, s, [&](cudaStream_t st) {
+      return v.experts_small ? launch_gateup_s(a, G, st, false, h->smem_optin) : launch_gateup_splitk(a, G, st, false);
     });
-    timed(5, s, [&](cudaStream_t st) { return launch_down(a, G, st, false); });
+    timed(5, s, [&](cudaStream_t st) {
+      return v.experts_small ? launch_down_s(a, G, st, false, h->smem_optin) : launch_down(a, G, st, false);
+    });
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   for (int i = 0; i < k && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&kernel_ms[i], ev[2 * i], ev[2 * i + 1]);
