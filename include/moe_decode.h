@@ -153,8 +153,8 @@ MOE_API int moe_decode_kernels_per_step(moe_decode_handle* h, int batch);
  * `stream` with a CUDA event pair around every kernel, synchronises, and writes
  * each kernel's duration in milliseconds, in launch order, to kernel_ms (host,
  * max_kernels entries) and a short kernel name id to kernel_id (host, or NULL):
- * 1 o_proj+residual+RMS, 2 router+top-k, 3 gate/up small-M, 4 gate/up split-K,
- * 5 down+combine, 6 L2 prefetch (timed on the side stream).  Same buffers as
+ * 1 o_proj+residual+RMS, 2 router+top-k, 3 small-M expert kernel (gate/up and down),
+ * 4 gate/up split-K, 5 down+combine, 6 L2 prefetch.  Same buffers as
  * moe_decode_step.  Returns the number of kernels timed (or a negative code). */
 MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_out,
                                     const void* residual_in, void* out, int32_t* topk_idx,

@@ -5,6 +5,7 @@
 
 namespace moe {
 
+// Device counters: router ticket; expert-kernel grid barrier (count, generation).
 enum Counter { kCntOproj = 0, kCntRouter = 1, kCntGateUp = 2, kNumCounters = 4 };
 
 // Library-owned device workspace (one per handle).
@@ -77,8 +78,7 @@ bool router_ok(const LayerArgs& a, size_t smem_optin);       // router at this b
 cudaError_t set_small_attributes(size_t smem_optin);
 cudaError_t launch_oproj_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t launch_router_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
-cudaError_t launch_gateup_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
-cudaError_t launch_down_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
+cudaError_t launch_experts_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t set_kernel_attributes(size_t smem_optin);
 
 }  // namespace moe

@@ -17,11 +17,10 @@
 //   k_oproj_f    h = residual + W_o . attn_out, per-CTA sums of h^2            (batch <= 2)
 //   k_router_f   rstd, x = h * rstd * gamma, logits = W_r . x   (any batch; at batch >= 3
 //                the last CTA also builds the global routing tables)
-//   k_gateup_f   routing per CTA, then a = silu(W_g x) * (W_u x) for each (selected expert,
-//                row pair), each pair streamed once                            (batch <= 2)
-//   k_down_f     routing per CTA, then out = bf16(h + sum_j gate_j * W_down[e_j] . a_j);
-//                every lane accumulates its share of a row over all experts in registers
-//                and reduces once                                              (batch <= 2)
+//   k_experts_f  the expert kernel (batch <= 2): routing once per CTA; gate/up + SiLU*mul
+//                for each (selected expert, row pair), each pair streamed once; a grid
+//                barrier; then out = bf16(h + sum_j gate_j * W_down[e_j] . a_j), with W_down
+//                streaming into the freed ring while the barrier is open
 //
 // Weights are static, so producers issue their first copies before the programmatic-
 // launch dependency wait; activations are read only after it, with L2 loads.
@@ -299,41 +298,120 @@ __global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
 }
 
 // =============================================================================
-// K3 (batch <= 2): routing per CTA, then expert gate/up + SiLU*mul
-//   Pairs (union expert u, row p) in flattened order; CTA c takes [q0, q1).  A stage is up to
-//   PS consecutive pairs of one expert: its gate rows and its up rows (two copies).
+// Grid barrier for the expert kernel (cooperative launch: every CTA is resident).
+// Sense reversal: each CTA reads the generation before it arrives, the last arrival resets
+// the count and advances the generation, the others wait for the advance.  The wait is
+// bounded in time; on expiry the CTA records kErrTimeout and carries on (its results are
+// then meaningless, and the error word says so).  Called by the consumer warps only.
 // =============================================================================
-template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) k_gateup_f(const LayerArgs a) {
+namespace {
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ void grid_barrier(unsigned* count, unsigned* gen, volatile int* abort_flag, uint32_t* err) {
+  __threadfence();
+  consumer_sync();
+  if (threadIdx.x == 0) {
+    const unsigned g = ld_acquire_u32(gen);
+    const unsigned arrived = atomicAdd(count, 1u) + 1u;
+    if (arrived == gridDim.x) {
+      atomicExch(count, 0u);
+      __threadfence();
+      atomicExch(gen, g + 1u);
+    } else {
+      const unsigned long long t0 = globaltimer();
+      while (ld_acquire_u32(gen) == g) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicOr(err, kErrTimeout);
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+  }
+  consumer_sync();
+}
+
+}  // namespace
+
+// =============================================================================
+// K3 (batch <= 2): the expert kernel.  Routing once per CTA, then
+//   phase A  gate/up + SiLU*mul: pairs (union expert u, row p) in flattened order, CTA c takes
+//            [q0, q1); a stage is up to PS consecutive pairs of one expert (its gate rows and
+//            its up rows, two copies).  a goes to global memory.
+//   grid barrier (every a is needed by every CTA)
+//   phase B  down + combine: CTA c owns output rows [i0, i1); a stage is those rows of one
+//            union expert (one copy).  The producer streams phase B's weights into the freed
+//            ring while the barrier is still open.  Warp w owns rows w, w + 8, ...; lane l
+//            holds elements [l*EPL, (l+1)*EPL) of each row and accumulates over all experts
+//            in registers; one warp reduction per (row, token) at the end.
+// =============================================================================
+template <int NT, int EPL>
+__global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int kRPW = 7;  // rows per warp in phase B (rows_max <= 56)
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, I = a.I, B = a.B;
-  const int S = a.k3.stages, PS = a.k3.rows_per_stage;  // pairs per stage
-  const uint32_t row_bytes = (uint32_t)d * 2u;
-  const size_t SB = al128((size_t)2 * PS * row_bytes);
-  const int PM = a.k3.rows_max;  // max pairs per CTA
+  const int SA = a.k3.stages, PS = a.k3.rows_per_stage, PM = a.k3.rows_max;
+  const int SBn = a.k4.stages, RM = a.k4.rows_max;
+  const uint32_t row_bytes = (uint32_t)d * 2u, drow_bytes = (uint32_t)I * 2u;
+  const size_t SA_B = al128((size_t)2 * PS * row_bytes), SB_B = al128((size_t)RM * drow_bytes);
+  const size_t region = std::max((size_t)SA * SA_B, (size_t)SBn * SB_B);
+  const size_t scratch_f = std::max((size_t)PM * 2 * kConsumerWarps * NT, (size_t)B * a.k * I);  // floats
+  long long lo, hi;
+  split_range(d, G, c, lo, hi);
+  const int i0 = (int)lo, nrows = (int)(hi - lo);
 
   unsigned char* ring = smem;
-  float* part = reinterpret_cast<float*>(ring + (size_t)S * SB);  // [PM][2][8][NT]
-  SmallRoute* rt = reinterpret_cast<SmallRoute*>(part + PM * 2 * kConsumerWarps * NT);
+  float* part = reinterpret_cast<float*>(ring + region);  // phase A partials, then phase B's a
+  float* a_s = part;
+  SmallRoute* rt = reinterpret_cast<SmallRoute*>(part + scratch_f);
   RouteScratch* sc = reinterpret_cast<RouteScratch*>(rt + 1);
-  float* fb = reinterpret_cast<float*>(sc + 1);  // fallback top-k scratch: 2 warps x 2 arrays
-  uint64_t* full = reinterpret_cast<uint64_t*>(
+  float* fb = reinterpret_cast<float*>(sc + 1);
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(
       smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + 2 * 2 * kCandStride) - smem)));
-  uint64_t* empty = full + S;
-  int* s_misc = reinterpret_cast<int*>(empty + S);
+  uint64_t* emptyA = fullA + kMaxStages;
+  uint64_t* fullB = emptyA + kMaxStages;
+  uint64_t* emptyB = fullB + kMaxStages;
+  int* s_misc = reinterpret_cast<int*>(emptyB + kMaxStages);
   volatile int* abort_flag = s_misc;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   if (tid == 0) {
-    init_ring(full, empty, S);
+    init_ring(fullA, emptyA, SA);
+    init_ring(fullB, emptyB, SBn);
     s_misc[0] = 0;
     fence_barrier_init();
   }
   pdl_wait();  // logits and x come from the router kernel
-  // Dependents may launch only now: the down kernel reads the logits before its own wait.
   pdl_trigger();
-  route_small_cta(a, rt, sc, fb, c == 0);  // contains __syncthreads (also covers the init)
+
+  // x of every token, in registers (consumers; issued before routing to overlap it).
+  const int qpw = d / 64, qbase = warp * qpw;
+  float xr[NT][kCPLf][8];
+  if (warp < kConsumerWarps) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int j = 0; j < kCPLf; ++j) {
+        if (t < B && cvalid(qpw, j, lane)) {
+          const float* xp = a.ws.x + (size_t)t * d + (size_t)(qbase + j * 32 + lane) * 8;
+          const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
+          xr[t][j][0] = x0.x; xr[t][j][1] = x0.y; xr[t][j][2] = x0.z; xr[t][j][3] = x0.w;
+          xr[t][j][4] = x1.x; xr[t][j][5] = x1.y; xr[t][j][6] = x1.z; xr[t][j][7] = x1.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+        }
+      }
+  }
+  route_small_cta(a, rt, sc, fb, c == 0);  // barriers inside also publish the ring init
 
   const int U = rt->U;
   long long q0l, q1l;
@@ -343,139 +421,85 @@ __global__ void __launch_bounds__(kThreads, 1) k_gateup_f(const LayerArgs a) {
   if (warp == kConsumerWarps) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
+      // phase A: gate/up rows
       int it = 0;
       int u = q0 / I, p = q0 - u * I;
       for (int q = q0; q < q1; ++it) {
         const int np = min(min(PS, I - p), q1 - q);
-        if (!ring_acquire(empty, it, S, abort_flag, a.ws.err)) break;
-        const int s = it % S;
+        if (!ring_acquire(emptyA, it, SA, abort_flag, a.ws.err)) break;
+        const int s = it % SA;
         const uint16_t* base = a.w_gu + ((size_t)rt->un_e[u] * 2 * I + p) * d;
-        mbar_arrive_expect_tx(&full[s], 2u * np * row_bytes);
-        bulk_g2s(ring + s * SB, base, np * row_bytes, &full[s], pol);
-        bulk_g2s(ring + s * SB + (size_t)PS * row_bytes, base + (size_t)I * d, np * row_bytes, &full[s], pol);
+        mbar_arrive_expect_tx(&fullA[s], 2u * np * row_bytes);
+        bulk_g2s(ring + s * SA_B, base, np * row_bytes, &fullA[s], pol);
+        bulk_g2s(ring + s * SA_B + (size_t)PS * row_bytes, base + (size_t)I * d, np * row_bytes, &fullA[s], pol);
         q += np;
         p += np;
         if (p == I) { p = 0; ++u; }
       }
-      ring_drain(full, it, S, a.ws.err);
+      // The ring is reused by phase B only after every phase-A fill has landed and been read.
+      ring_drain(fullA, it, SA, a.ws.err);
+      for (int i = it - SA < 0 ? 0 : it - SA; i < it; ++i) mbar_drain(&emptyA[i % SA], (i / SA) & 1, a.ws.err);
+      // phase B: this CTA's rows of W_down for every union expert
+      if (nrows > 0) {
+        int jt = 0;
+        for (int uu = 0; uu < U; ++uu, ++jt) {
+          if (!ring_acquire(emptyB, jt, SBn, abort_flag, a.ws.err)) break;
+          const int s = jt % SBn;
+          mbar_arrive_expect_tx(&fullB[s], nrows * drow_bytes);
+          bulk_g2s(ring + s * SB_B, a.w_down + ((size_t)rt->un_e[uu] * d + i0) * I, nrows * drow_bytes, &fullB[s],
+                   pol);
+        }
+        ring_drain(fullB, jt, SBn, a.ws.err);
+      }
     }
     return;
   }
 
-  const int qpw = d / 64, qbase = warp * qpw;
-  float xr[NT][kCPLf][8];
+  // ---- phase A (consumers) ------------------------------------------------------------
+  {
+    int it = 0;
+    int p = q0 - (q0 / I) * I;
+    for (int q = q0; q < q1; ++it) {
+      const int np = min(min(PS, I - p), q1 - q), s = it % SA;
+      mbar_wait(&fullA[s], (it / SA) & 1, abort_flag, a.ws.err);
+      const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SA_B);
+      for (int i = 0; i < 2 * np; ++i) {  // gate rows 0..np-1, then up rows
+        const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
+        float v[NT];
+        row_dot<NT>(st + (size_t)(gu * PS + pi) * d, xr, qbase, qpw, lane, v);
 #pragma unroll
-  for (int t = 0; t < NT; ++t)
-#pragma unroll
-    for (int j = 0; j < kCPLf; ++j) {
-      if (t < B && cvalid(qpw, j, lane)) {
-        const float* xp = a.ws.x + (size_t)t * d + (size_t)(qbase + j * 32 + lane) * 8;
-        const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
-        xr[t][j][0] = x0.x; xr[t][j][1] = x0.y; xr[t][j][2] = x0.z; xr[t][j][3] = x0.w;
-        xr[t][j][4] = x1.x; xr[t][j][5] = x1.y; xr[t][j][6] = x1.z; xr[t][j][7] = x1.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+        for (int t = 0; t < NT; ++t) {
+          const float w = warp_sum(v[t]);
+          if (lane == 0) part[(((q - q0 + pi) * 2 + gu) * kConsumerWarps + warp) * NT + t] = w;
+        }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&emptyA[s]);
+      q += np;
+      p += np;
+      if (p == I) p = 0;
     }
-  int it = 0;
-  int p = q0 - (q0 / I) * I;
-  for (int q = q0; q < q1; ++it) {
-    const int np = min(min(PS, I - p), q1 - q), s = it % S;
-    mbar_wait(&full[s], (it / S) & 1, abort_flag, a.ws.err);
-    const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB);
-    for (int i = 0; i < 2 * np; ++i) {  // gate rows 0..np-1, then up rows
-      const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
-      float v[NT];
-      row_dot<NT>(st + (size_t)(gu * PS + pi) * d, xr, qbase, qpw, lane, v);
+    consumer_sync();
+    for (int z = tid; z < (q1 - q0) * B; z += kConsumerThreads) {
+      const int pl = z / B, t = z % B;
+      float gs = 0.f, us = 0.f;
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const float w = warp_sum(v[t]);
-        if (lane == 0) part[(((q - q0 + pi) * 2 + gu) * kConsumerWarps + warp) * NT + t] = w;
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        gs += part[((pl * 2 + 0) * kConsumerWarps + w) * NT + t];
+        us += part[((pl * 2 + 1) * kConsumerWarps + w) * NT + t];
       }
+      const int qq = q0 + pl, u = qq / I, pp = qq - u * I;
+      for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+        if (rt->ent_tok[en] == t) a.ws.a[(size_t)en * I + pp] = gs / (1.0f + expf(-gs)) * us;
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    q += np;
-    p += np;
-    if (p == I) p = 0;
-  }
-  consumer_sync();
-  for (int z = tid; z < (q1 - q0) * B; z += kConsumerThreads) {
-    const int pl = z / B, t = z % B;
-    float gs = 0.f, us = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      gs += part[((pl * 2 + 0) * kConsumerWarps + w) * NT + t];
-      us += part[((pl * 2 + 1) * kConsumerWarps + w) * NT + t];
-    }
-    const int qq = q0 + pl, u = qq / I, pp = qq - u * I;
-    for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
-      if (rt->ent_tok[en] == t) a.ws.a[(size_t)en * I + pp] = gs / (1.0f + expf(-gs)) * us;
-  }
-}
-
-// =============================================================================
-// K4 (batch <= 2): routing per CTA, then expert down projection + combine
-//   CTA c owns output rows [i0, i1); a stage is those rows of one union expert (contiguous).
-//   Warp w owns rows w, w + 8, ...; lane l the elements [l*EPL, (l+1)*EPL) of each row.
-// =============================================================================
-template <int NT, int EPL>
-__global__ void __launch_bounds__(kThreads, 1) k_down_f(const LayerArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kRPW = 7;  // rows per warp (rows_max <= 56)
-  const int G = gridDim.x, c = blockIdx.x;
-  const int d = a.d, I = a.I, B = a.B;
-  const int S = a.k4.stages, RM = a.k4.rows_max;
-  long long lo, hi;
-  split_range(d, G, c, lo, hi);
-  const int i0 = (int)lo, nrows = (int)(hi - lo);
-  const uint32_t row_bytes = (uint32_t)I * 2u;
-  const size_t SB = al128((size_t)RM * row_bytes);
-
-  unsigned char* ring = smem;
-  float* a_s = reinterpret_cast<float*>(ring + (size_t)S * SB);  // [n_ent][I], gate-scaled
-  SmallRoute* rt = reinterpret_cast<SmallRoute*>(a_s + (size_t)B * a.k * I);
-  RouteScratch* sc = reinterpret_cast<RouteScratch*>(rt + 1);
-  float* fb = reinterpret_cast<float*>(sc + 1);
-  uint64_t* full = reinterpret_cast<uint64_t*>(
-      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + 2 * 2 * kCandStride) - smem)));
-  uint64_t* empty = full + S;
-  int* s_misc = reinterpret_cast<int*>(empty + S);
-  volatile int* abort_flag = s_misc;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  if (tid == 0) {
-    init_ring(full, empty, S);
-    s_misc[0] = 0;
-    fence_barrier_init();
-  }
-  // The logits were complete before this grid could launch: the gate/up kernel allows its
-  // dependents to launch only after its own dependency wait, which returns once the router
-  // kernel has finished.
-  route_small_cta(a, rt, sc, fb, false);
-  const int U = rt->U;
-  pdl_trigger();
-
-  if (warp == kConsumerWarps) {
-    if (lane == 0 && nrows > 0) {  // W_down is static: stream it before the dependency wait
-      const uint64_t pol = policy_evict_first();
-      int it = 0;
-      for (int u = 0; u < U; ++u, ++it) {
-        if (!ring_acquire(empty, it, S, abort_flag, a.ws.err)) break;
-        const int s = it % S;
-        mbar_arrive_expect_tx(&full[s], nrows * row_bytes);
-        bulk_g2s(ring + s * SB, a.w_down + ((size_t)rt->un_e[u] * d + i0) * I, nrows * row_bytes, &full[s], pol);
-      }
-      ring_drain(full, it, S, a.ws.err);
-    }
-    return;
   }
 
-  pdl_wait();  // the SwiGLU activations come from the gate/up kernel
+  grid_barrier(&a.ws.counters[kCntGateUp], &a.ws.counters[kCntGateUp + 1], abort_flag, a.ws.err);
+
+  // ---- phase B (consumers) ------------------------------------------------------------
   const int nent = rt->n_ent;
   for (int z = tid; z < nent * (I / 4); z += kConsumerThreads) {
-    const int en = z / (I / 4), cq = z % (I / 4);
+    const int en = z / (I / 4), cq = z - en * (I / 4);
     const float g = rt->ent_gate[en];
     const float4 v = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
     *reinterpret_cast<float4*>(a_s + (size_t)en * I + cq * 4) = make_float4(g * v.x, g * v.y, g * v.z, g * v.w);
@@ -489,16 +513,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_down_f(const LayerArgs a) {
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[i][t] = 0.f;
   for (int u = 0; u < U && nrows > 0; ++u) {
-    const int s = u % S;
-    mbar_wait(&full[s], (u / S) & 1, abort_flag, a.ws.err);
-    const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB);
+    const int s = u % SBn;
+    mbar_wait(&fullB[s], (u / SBn) & 1, abort_flag, a.ws.err);
+    const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB_B);
     for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en) {
       const int t = rt->ent_tok[en];
       float av[EPL > 0 ? EPL : 16];
       const float* ap = a_s + (size_t)en * I + lane * epl;
       if constexpr (EPL == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(ap);
-        av[0] = v.x; av[1] = v.y; av[2] = v.z; av[3] = v.w;
+        const float4 vv = *reinterpret_cast<const float4*>(ap);
+        av[0] = vv.x; av[1] = vv.y; av[2] = vv.z; av[3] = vv.w;
       } else if constexpr (EPL == 8) {
         const float4 v0 = *reinterpret_cast<const float4*>(ap), v1 = *reinterpret_cast<const float4*>(ap + 4);
         av[0] = v0.x; av[1] = v0.y; av[2] = v0.z; av[3] = v0.w; av[4] = v1.x; av[5] = v1.y; av[6] = v1.z; av[7] = v1.w;
@@ -536,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_down_f(const LayerArgs a) {
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    if (lane == 0) mbar_arrive(&emptyB[s]);
   }
 #pragma unroll
   for (int i = 0; i < kRPW; ++i) {
@@ -559,17 +583,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_down_f(const LayerArgs a) {
 namespace {
 
 template <typename Kern>
-cudaError_t launch_f(Kern k, int grid, size_t smem, cudaStream_t s, bool pdl, const LayerArgs& a) {
+cudaError_t launch_f(Kern k, int grid, size_t smem, cudaStream_t s, bool pdl, const LayerArgs& a,
+                     bool cooperative = false) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cooperative) {  // the expert kernel's grid barrier needs every CTA resident
+    attr[n].id = cudaLaunchAttributeCooperative;
+    attr[n].val.cooperative = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, k, a);
 }
 
@@ -601,30 +635,29 @@ bool plan_small(LayerArgs& a, int G, size_t optin) {
              8 + 32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
     if (t.smem > budget) return false;
   }
-  {  // K3: pairs of gate/up rows
+  {  // K3 (phase A): pairs of gate/up rows; K4 fields: phase B of the same kernel
     KTune& t = a.k3;
+    KTune& t4 = a.k4;
     const size_t row = (size_t)a.d * 2;
     const long long umax = std::min(a.E, std::max(a.B, 1) * a.k);
     t.rows_max = (int)((umax * a.I + G - 1) / G);  // pairs per CTA
-    const size_t extra = (size_t)t.rows_max * 2 * kConsumerWarps * NT * 4 + kRouteBytes + 2 * kMaxStages * 8 + 64;
+    t4.rows_max = (a.d + G - 1) / G;                // output rows per CTA
+    if (t4.rows_max > 7 * kConsumerWarps) return false;
+    const size_t scratch_f = std::max((size_t)t.rows_max * 2 * kConsumerWarps * NT, (size_t)std::max(a.B, 1) * a.k * a.I);
+    const size_t extra = up128(scratch_f * 4) + kRouteBytes + 4 * kMaxStages * 8 + 64;
+    const size_t SBd = up128((size_t)t4.rows_max * a.I * 2);
     t.stages = 0;
     for (int ps = 2; ps >= 1 && t.stages < 2; --ps) {
       t.rows_per_stage = ps;
       const size_t SB = up128((size_t)2 * ps * row);
       t.stages = extra < budget ? (int)std::min<size_t>(kMaxStages, (budget - extra) / SB) : 0;
-      t.smem = (size_t)t.stages * SB + extra;
     }
     if (t.stages < 2) return false;
-  }
-  {  // K4: one expert's rows per stage
-    KTune& t = a.k4;
-    t.rows_max = (a.d + G - 1) / G;
-    if (t.rows_max > 7 * kConsumerWarps) return false;
-    const size_t SB = up128((size_t)t.rows_max * a.I * 2);
-    const size_t extra = (size_t)std::max(a.B, 1) * a.k * a.I * 4 + kRouteBytes + 2 * kMaxStages * 8 + 64;
-    t.stages = extra < budget ? (int)std::min<size_t>(kMaxStages, (budget - extra) / SB) : 0;
-    if (t.stages < 2) return false;
-    t.smem = (size_t)t.stages * SB + extra;
+    const size_t regionA = (size_t)t.stages * up128((size_t)2 * t.rows_per_stage * row);
+    t4.stages = (int)std::min<size_t>(kMaxStages, regionA / SBd);
+    if (t4.stages < 2) return false;
+    t.smem = std::max(regionA, (size_t)t4.stages * SBd) + extra;
+    t4.smem = t.smem;
   }
   return true;
 }
@@ -656,14 +689,12 @@ cudaError_t set_small_attributes(size_t optin) {
   SETS(k_oproj_f<2>);
   SETS(k_router_f<1>);
   SETS(k_router_f<2>);
-  SETS(k_gateup_f<1>);
-  SETS(k_gateup_f<2>);
-  SETS((k_down_f<1, 4>));
-  SETS((k_down_f<2, 4>));
-  SETS((k_down_f<1, 8>));
-  SETS((k_down_f<2, 8>));
-  SETS((k_down_f<1, 0>));
-  SETS((k_down_f<2, 0>));
+  SETS((k_experts_f<1, 4>));
+  SETS((k_experts_f<2, 4>));
+  SETS((k_experts_f<1, 8>));
+  SETS((k_experts_f<2, 8>));
+  SETS((k_experts_f<1, 0>));
+  SETS((k_experts_f<2, 0>));
 #undef SETS
   return e;
 }
@@ -690,19 +721,15 @@ cudaError_t launch_router_s(const LayerArgs& a0, int grid, cudaStream_t s, bool 
   return a.B == 1 ? launch_f(k_router_f<1>, grid, a.k2.smem, s, pdl, a) : launch_f(k_router_f<2>, grid, a.k2.smem, s, pdl, a);
 }
 
-cudaError_t launch_gateup_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
-  const LayerArgs a = planned(a0, grid, optin);
-  return a.B == 1 ? launch_f(k_gateup_f<1>, grid, a.k3.smem, s, pdl, a) : launch_f(k_gateup_f<2>, grid, a.k3.smem, s, pdl, a);
-}
-
-cudaError_t launch_down_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
+cudaError_t launch_experts_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   const LayerArgs a = planned(a0, grid, optin);
   const int epl = a.I / 32;
+  const size_t sm = a.k3.smem;
   if (epl == 4)
-    return a.B == 1 ? launch_f(k_down_f<1, 4>, grid, a.k4.smem, s, pdl, a) : launch_f(k_down_f<2, 4>, grid, a.k4.smem, s, pdl, a);
+    return a.B == 1 ? launch_f(k_experts_f<1, 4>, grid, sm, s, pdl, a, true) : launch_f(k_experts_f<2, 4>, grid, sm, s, pdl, a, true);
   if (epl == 8)
-    return a.B == 1 ? launch_f(k_down_f<1, 8>, grid, a.k4.smem, s, pdl, a) : launch_f(k_down_f<2, 8>, grid, a.k4.smem, s, pdl, a);
-  return a.B == 1 ? launch_f(k_down_f<1, 0>, grid, a.k4.smem, s, pdl, a) : launch_f(k_down_f<2, 0>, grid, a.k4.smem, s, pdl, a);
+    return a.B == 1 ? launch_f(k_experts_f<1, 8>, grid, sm, s, pdl, a, true) : launch_f(k_experts_f<2, 8>, grid, sm, s, pdl, a, true);
+  return a.B == 1 ? launch_f(k_experts_f<1, 0>, grid, sm, s, pdl, a, true) : launch_f(k_experts_f<2, 0>, grid, sm, s, pdl, a, true);
 }
 
 }  // namespace moe

@@ -190,10 +190,14 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
       ++kernels;
       forked = true;
     }
-    if (e == cudaSuccess)
-      e = v.experts_small ? launch_gateup_s(a, G, h->cap, true, h->smem_optin) : launch_gateup_splitk(a, G, h->cap, true);
-    if (e == cudaSuccess) e = v.experts_small ? launch_down_s(a, G, h->cap, true, h->smem_optin) : launch_down(a, G, h->cap, true);
-    kernels += 2;
+    if (v.experts_small) {
+      if (e == cudaSuccess) e = launch_experts_s(a, G, h->cap, true, h->smem_optin);
+      kernels += 1;
+    } else {
+      if (e == cudaSuccess) e = launch_gateup_splitk(a, G, h->cap, true);
+      if (e == cudaSuccess) e = launch_down(a, G, h->cap, true);
+      kernels += 2;
+    }
   }
   if (e == cudaSuccess && forked) {
     e = cudaEventRecord(h->events[ev], h->side);
@@ -485,7 +489,11 @@ int moe_decode_get_intermediate(moe_decode_handle* h, int which, void* dst, size
 int moe_decode_kernels_per_step(moe_decode_handle* h, int batch) {
   if (!h || !is_live(h) || batch < 1 || batch > h->cfg.max_batch) return MOE_ERR_INVALID_ARG;
   const int L = h->cfg.n_layers;
-  return 4 * L + ((h->cfg.enable_prefetch && L > 1) ? L - 1 : 0);
+  LayerArgs a = h->plan_splitk;
+  a.B = batch;
+  plan_layer(a, h->num_sms, h->smem_optin);
+  const int per_layer = variant_of(h, a).experts_small ? 3 : 4;
+  return per_layer * L + ((h->cfg.enable_prefetch && L > 1) ? L - 1 : 0);
 }
 
 int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_out, const void* residual_in,
@@ -524,12 +532,12 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
       PrefetchArgs p = prefetch_args(h, l + 1);
       timed(6, s, [&](cudaStream_t st) { return launch_prefetch(p, G, st); });
     }
-    timed(v.experts_small ? 3 : 4, s, [&](cudaStream_t st) {
-      return v.experts_small ? launch_gateup_s(a, G, st, false, h->smem_optin) : launch_gateup_splitk(a, G, st, false);
-    });
-    timed(5, s, [&](cudaStream_t st) {
-      return v.experts_small ? launch_down_s(a, G, st, false, h->smem_optin) : launch_down(a, G, st, false);
-    });
+    if (v.experts_small) {
+      timed(3, s, [&](cudaStream_t st) { return launch_experts_s(a, G, st, false, h->smem_optin); });
+    } else {
+      timed(4, s, [&](cudaStream_t st) { return launch_gateup_splitk(a, G, st, false); });
+      timed(5, s, [&](cudaStream_t st) { return launch_down(a, G, st, false); });
+    }
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   for (int i = 0; i < k && e == cudaSuccess; ++i) e = cudaEventElapsedTime(&kernel_ms[i], ev[2 * i], ev[2 * i + 1]);

@@ -311,13 +311,13 @@ __device__ void route_small(const LayerArgs& a, SmallRoute* rt, float* cand, boo
 
 namespace moe {
 
-// CTA-wide routing of a batch of at most 2 tokens (every thread calls it; 5 barriers).
+// CTA-wide routing of a batch of at most 2 tokens (every thread calls it; 7 barriers).
 // Selection with few dependent steps: each thread loads its strided share of the logits;
 // quarter-warp maxima (36 per token at 288 threads) give the lower bound T = their K-th
 // largest value (K groups hold an element >= T, so the K-th largest logit is >= T); the
 // logits >= T are compacted and ranked exactly in parallel.  Entries are then sorted by
-// (expert, token) and the union of experts marked.  Falls back to a warp arg-max
-// selection when more than kCandMax logits reach the bound.
+// (expert, token) and the union of experts indexed in the same pass.  Falls back to a warp
+// arg-max selection when more than kCandMax logits reach the bound.
 struct RouteScratch {
   float gmax[2][64];
   float T[2];
@@ -326,6 +326,8 @@ struct RouteScratch {
   int ci[2][kCandMax];
   float sel_v[2][32];
   int sel_i[2][32];
+  int key[64];
+  unsigned emask[32];  // experts selected by token 0
 };
 
 namespace {
@@ -349,7 +351,8 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
       }
       v[t][i] = x;
     }
-  if (tid < 4) sc->cnt[tid & 1] = 0;
+  if (tid < 2) sc->cnt[tid] = 0;
+  if (tid < 32) sc->emask[tid] = 0u;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     float m = -INFINITY;
@@ -360,11 +363,12 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
     if ((lane & 7) == 0 && t < B) sc->gmax[t][tid >> 3] = m;
   }
   __syncthreads();
-  // T[t] = K-th largest group maximum (ties by group index).
+  // (2) T[t] = K-th largest group maximum (ties by group index).
   if (tid < B * ngroups) {
-    const int t = tid / ngroups, gi = tid % ngroups;
+    const int t = tid / ngroups, gi = tid - t * ngroups;
     const float m = sc->gmax[t][gi];
     int r = 0;
+#pragma unroll 4
     for (int o = 0; o < ngroups; ++o) {
       const float x = sc->gmax[t][o];
       r += (x > m) || (x == m && o < gi);
@@ -372,6 +376,7 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
     if (r == K - 1) sc->T[t] = m;
   }
   __syncthreads();
+  // (3) candidates: logits >= T.
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     if (t >= B) break;
@@ -389,23 +394,26 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
     }
   }
   __syncthreads();
-  // Exact ranks among the candidates (= ranks among all experts).
+  // (4) exact ranks among the candidates (= ranks among all experts).
   for (int z = tid; z < 2 * kCandMax; z += nth) {
-    const int t = z / kCandMax, c = z % kCandMax;
-    if (t < B && c < sc->cnt[t] && sc->cnt[t] <= kCandMax) {
-      const float x = sc->cv[t][c];
-      const int xi = sc->ci[t][c];
+    const int t = z / kCandMax, c = z - t * kCandMax;
+    if (t < B) {
       const int C = sc->cnt[t];
-      int r = 0;
-      for (int o = 0; o < C; ++o) r += better(sc->cv[t][o], sc->ci[t][o], x, xi);
-      if (r < K) {
-        sc->sel_v[t][r] = x;
-        sc->sel_i[t][r] = xi;
+      if (c < C && C <= kCandMax) {
+        const float x = sc->cv[t][c];
+        const int xi = sc->ci[t][c];
+        int r = 0;
+#pragma unroll 4
+        for (int o = 0; o < C; ++o) r += better(sc->cv[t][o], sc->ci[t][o], x, xi);
+        if (r < K) {
+          sc->sel_v[t][r] = x;
+          sc->sel_i[t][r] = xi;
+        }
       }
     }
   }
   __syncthreads();
-  // Gates (warp t for token t); overflow tokens take the warp arg-max selection instead.
+  // (5) gates (warp t for token t; overflow tokens take the warp arg-max selection).
   if (warp < B) {
     float my_v = 0.f;
     int my_i = 0;
@@ -423,6 +431,8 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
       if (e != my_i) atomicOr(a.ws.err, kErrBounds);
       rt->idx[warp][lane] = e;
       rt->gate[warp][lane] = gte;
+      sc->key[warp * K + lane] = e * 2 + warp;
+      if (warp == 0) atomicOr(&sc->emask[e >> 5], 1u << (e & 31));
       if (write_user) {
         if (a.user_idx) a.user_idx[warp * K + lane] = e;
         if (a.user_gate) a.user_gate[warp * K + lane] = gte;
@@ -430,36 +440,34 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
     }
   }
   __syncthreads();
-  // Entries sorted by (expert, token): key = expert * 2 + token is unique.
+  // (6) entries sorted by key = expert * 2 + token (unique); an entry opens a union expert
+  // when its token is 0 or token 0 did not select that expert.
   const int n = B * K;
+  bool opens = false;
   if (tid < n) {
-    const int t = tid / K, j = tid % K;
-    const int key = rt->idx[t][j] * 2 + t;
-    int r = 0;
-    for (int o = 0; o < n; ++o) r += (rt->idx[o / K][o % K] * 2 + o / K) < key;
+    const int key = sc->key[tid], e = key >> 1, t = key & 1;
+    int r = 0, u = 0;
+#pragma unroll 4
+    for (int o = 0; o < n; ++o) {
+      const int k2 = sc->key[o], e2 = k2 >> 1;
+      r += k2 < key;
+      const bool op2 = (k2 & 1) == 0 || !((sc->emask[e2 >> 5] >> (e2 & 31)) & 1u);
+      u += (op2 && e2 < e);
+    }
+    opens = (t == 0) || !((sc->emask[e >> 5] >> (e & 31)) & 1u);
     rt->key[r] = key;
     rt->ent_tok[r] = t;
-    rt->ent_gate[r] = rt->gate[t][j];
+    rt->ent_gate[r] = rt->gate[t][tid - t * K];
+    if (opens) {
+      rt->un_e[u] = e;
+      rt->un_off[u] = r;
+    }
   }
-  __syncthreads();
-  if (warp == 0) {
-    int base = 0;
-    for (int p0 = 0; p0 < n; p0 += 32) {
-      const int p = p0 + lane;
-      const bool first = p < n && (p == 0 || (rt->key[p - 1] >> 1) != (rt->key[p] >> 1));
-      const unsigned m = __ballot_sync(0xffffffffu, first);
-      if (first) {
-        const int u = base + __popc(m & ((1u << lane) - 1u));
-        rt->un_e[u] = rt->key[p] >> 1;
-        rt->un_off[u] = p;
-      }
-      base += __popc(m);
-    }
-    if (lane == 0) {
-      rt->U = base;
-      rt->n_ent = n;
-      rt->un_off[base] = n;
-    }
+  const int U = __syncthreads_count(opens);
+  if (tid == 0) {
+    rt->U = U;
+    rt->n_ent = n;
+    rt->un_off[U] = n;
   }
   __syncthreads();
 }

@@ -98,7 +98,8 @@ def test_step_argument_checks():
             md.moe_decode_get_intermediate(h, 9, out, 16)
         md.moe_decode_step(h, 2, attn, res, out)
         assert md.moe_decode_sync_status(h) == 0
-        assert md.moe_decode_kernels_per_step(h, 2) == 4
+        assert md.moe_decode_kernels_per_step(h, 2) == 3  # small path: o_proj, router, experts
+        assert md.moe_decode_kernels_per_step(h, 4) == 4  # split-K path: o_proj, router, gate/up, down
     finally:
         assert md.moe_decode_destroy(h) == 0
     assert md.moe_decode_destroy(h) == md.MOE_ERR_INVALID_ARG  # destroyed twice: rejected
