@@ -61,7 +61,8 @@ enum {
   MOE_ERR_OOM = -4,                /* workspace allocation failed                   */
   MOE_ERR_CUDA = -5,               /* a CUDA runtime call failed                    */
   MOE_ERR_DEVICE_TIMEOUT = -6,     /* a kernel's bounded wait ran out               */
-  MOE_ERR_DEVICE_BOUNDS = -7       /* a kernel met an out-of-range index and skipped it */
+  MOE_ERR_DEVICE_BOUNDS = -7,      /* a kernel met an out-of-range index and skipped it */
+  MOE_ERR_SCRATCH_LIMIT = -8       /* moe_decode_step_static: scratch need above MOE_STATIC_SCRATCH_BYTES */
 };
 
 /* Layer shapes and options, fixed at create time.
@@ -160,6 +161,39 @@ MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void*
                                     const void* residual_in, void* out, int32_t* topk_idx,
                                     float* topk_gate, void* stream, float* kernel_ms,
                                     int* kernel_id, int max_kernels);
+
+/* Capacity of the static scratch array used by moe_decode_step_static (256 KiB per device). */
+#define MOE_STATIC_SCRATCH_BYTES (256u * 1024u)
+
+/* One layer step for batch 1 or 2 that allocates no device memory.  The pages have no
+ * counterpart of this entry point; it exists for callers that may not allocate when they
+ * run a step (an engine that has reserved nearly all device memory for its own pool, a
+ * process under a hard memory cap).
+ * It runs the same kernels as moe_decode_step's batch <= 2 path, launched directly on
+ * `stream` (no graph, no handle), with every intermediate in one static device array of
+ * MOE_STATIC_SCRATCH_BYTES that is part of the loaded library (one per device).
+ *   cfg          layer shapes as for moe_decode_create (host); n_layers must be 1 and
+ *                force_variant 0 or 1; enable_prefetch is ignored
+ *   w            the layer's weights (host struct of device pointers, as for create)
+ *   batch        1 or 2, and <= cfg->max_batch
+ *   attn_out     [batch][d_o] bf16, residual_in [batch][d] bf16, out [batch][d] bf16 (device)
+ *   topk_idx     [batch][top_k] int32 or NULL; topk_gate [batch][top_k] fp32 or NULL (device)
+ *   err_word     device uint32 (4-byte aligned) or NULL: receives this call's kernel error
+ *                bits (0 none, 1 a bounded wait ran out, 2 an index out of range)
+ * Errors: MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_CONFIG / MOE_ERR_ALIGNMENT as for
+ * create and step; MOE_ERR_SCRATCH_LIMIT when the scratch for (cfg, batch) exceeds
+ * MOE_STATIC_SCRATCH_BYTES (e.g. d = 8192 with top_k * inter = 16384 at batch 2); nothing is
+ * launched then.  MOE_ERR_CUDA on a failed CUDA call.
+ * The first call on each device, with that device current, looks up the array's address
+ * (cudaGetSymbolAddress) and sets kernel attributes; make that first call before any stream
+ * capture begins.  Each call zeroes the barrier counter and error word at the head of the
+ * array before its kernels run; nothing else needs a starting value.
+ * All calls on a device share the array: calls whose executions overlap (different streams,
+ * or threads without ordering) race on it and corrupt each other's results.  Outputs are
+ * valid once `stream` has been synchronised. */
+MOE_API int moe_decode_step_static(const moe_decode_config* cfg, const moe_decode_layer_weights* w, int batch,
+                                   const void* attn_out, const void* residual_in, void* out,
+                                   int32_t* topk_idx, float* topk_gate, uint32_t* err_word, void* stream);
 
 /* Frees the graphs and the workspace; weights are not touched.  NULL is a no-op. */
 MOE_API int moe_decode_destroy(moe_decode_handle* h);

@@ -22,10 +22,12 @@ MOE_ERR_OOM = -4
 MOE_ERR_CUDA = -5
 MOE_ERR_DEVICE_TIMEOUT = -6
 MOE_ERR_DEVICE_BOUNDS = -7
+MOE_ERR_SCRATCH_LIMIT = -8
+MOE_STATIC_SCRATCH_BYTES = 256 * 1024
 
 EXPORTED = ("moe_decode_create", "moe_decode_step", "moe_decode_step_host", "moe_decode_sync_status",
             "moe_decode_get_intermediate", "moe_decode_kernels_per_step", "moe_decode_profile_step",
-            "moe_decode_destroy", "moe_decode_strerror")
+            "moe_decode_step_static", "moe_decode_destroy", "moe_decode_strerror")
 
 KERNEL_NAMES = {1: "oproj_residual_rmsnorm", 2: "router_topk", 3: "experts_small_m", 4: "gateup_split_k",
                 5: "down_combine", 6: "prefetch_l2"}
@@ -70,6 +72,8 @@ def load(path: str = LIB_PATH):
     lib.moe_decode_get_intermediate.argtypes = [P, I, P, ctypes.c_size_t, P]
     lib.moe_decode_kernels_per_step.argtypes = [P, I]
     lib.moe_decode_profile_step.argtypes = [P, I, P, P, P, P, P, P, P, P, I]
+    lib.moe_decode_step_static.argtypes = [ctypes.POINTER(moe_decode_config),
+                                           ctypes.POINTER(moe_decode_layer_weights), I, P, P, P, P, P, P, P]
     lib.moe_decode_destroy.argtypes = [P]
     lib.moe_decode_strerror.argtypes = [I]
     lib.moe_decode_strerror.restype = ctypes.c_char_p
@@ -159,6 +163,21 @@ def moe_decode_profile_step(h: int, batch: int, attn_out, residual_in, out, topk
                                               _addr(topk_idx), _addr(topk_gate), _stream(stream), ms, ids,
                                               max_kernels), "moe_decode_profile_step")
     return [(KERNEL_NAMES.get(ids[i], str(ids[i])), ms[i]) for i in range(n)]
+
+
+def moe_decode_step_static(cfg: moe_decode_config, weights, batch: int, attn_out, residual_in, out,
+                           topk_idx=None, topk_gate=None, err_word=None, stream=None) -> None:
+    """One layer step (batch 1 or 2) with its scratch in the library's static device array."""
+    if isinstance(weights, moe_decode_layer_weights):
+        w = weights
+    elif isinstance(weights, dict):
+        w = moe_decode_layer_weights(*[_addr(weights[k]) for k in ("w_o", "gamma", "w_router", "w_gate_up",
+                                                                   "w_down")])
+    else:  # (w_o, gamma, w_router, w_gate_up, w_down)
+        w = moe_decode_layer_weights(*[_addr(t) for t in weights])
+    _check(load().moe_decode_step_static(ctypes.byref(cfg), ctypes.byref(w), batch, _addr(attn_out),
+                                         _addr(residual_in), _addr(out), _addr(topk_idx), _addr(topk_gate),
+                                         _addr(err_word), _stream(stream)), "moe_decode_step_static")
 
 
 def moe_decode_destroy(h: int) -> int:

@@ -575,6 +575,7 @@ const char* moe_decode_strerror(int code) {
     case MOE_ERR_CUDA: return "CUDA runtime error";
     case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case MOE_ERR_DEVICE_BOUNDS: return "device index out of range";
+    case MOE_ERR_SCRATCH_LIMIT: return "scratch need exceeds the static array";
     default: return "unknown error";
   }
 }
