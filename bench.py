@@ -51,7 +51,7 @@ WORKLOADS = {
     "tp8e64_b64": ("TP8E64", 64, 1, "indep"),
 }
 
-KERNEL_FILE = os.path.join(ROOT, "moe_decode_layer_02_b200", "csrc", "kernels.cu")
+KERNEL_DIR = os.path.join(ROOT, "moe_decode_layer_02_b200", "csrc")
 
 
 def peaks():
@@ -146,12 +146,25 @@ def algorithmic_bytes(dims, B, n_union):
         "router_topk": E * d * 2 + d * 2 + B * d * 4 + B * d * 4 + B * E * 4,
         "gateup": n_union * 2 * I * d * 2 + B * k * d * 4 + B * k * I * 4,
         "down_combine": n_union * d * I * 2 + B * k * I * 4 + B * d * 4 + B * d * 2,
+        # small-M expert kernel: gate/up and down weights of the union, x and h in, out
+        "experts_small_m": n_union * 3 * I * d * 2 + B * E * 4 + 2 * B * d * 4 + B * d * 2,
     }
 
 
 def weight_bytes(dims, n_union_per_layer):
     d, do, E, I = dims.d, dims.d_o, dims.E, dims.I
     return sum(d * do * 2 + d * 2 + E * d * 2 + u * (2 * I * d * 2 + d * I * 2) for u in n_union_per_layer)
+
+
+def kernels_sha():
+    """Hash of the kernel sources: ncu traffic figures are valid only for the code they were taken on."""
+    import hashlib
+    hs = hashlib.sha256()
+    for f in sorted(os.listdir(KERNEL_DIR)):
+        if f.endswith((".cu", ".cuh")):
+            hs.update(f.encode())
+            hs.update(open(os.path.join(KERNEL_DIR, f), "rb").read())
+    return hs.hexdigest()[:16]
 
 
 def traffic_for(kernel_name, B, workload):
@@ -161,7 +174,7 @@ def traffic_for(kernel_name, B, workload):
     if not os.path.exists(p):
         return None
     j = json.load(open(p))
-    h = hashlib.sha256(open(KERNEL_FILE, "rb").read()).hexdigest()[:16]
+    h = kernels_sha()
     ent = j.get(workload, {}).get(kernel_name)
     if not ent or ent.get("kernels_sha") != h:
         return None

@@ -5,7 +5,7 @@
 
 namespace moe {
 
-// Device counters: router ticket; expert-kernel grid barrier (count, generation).
+// Device counters: o_proj (unused), router ticket, expert-kernel grid barrier count, spare.
 enum Counter { kCntOproj = 0, kCntRouter = 1, kCntGateUp = 2, kNumCounters = 4 };
 
 // Library-owned device workspace (one per handle).

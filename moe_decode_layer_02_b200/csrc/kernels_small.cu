@@ -38,7 +38,16 @@ namespace moe {
 
 namespace {
 
-constexpr int kCPLf = 4;  // 8-element chunks per lane: K <= 8 warps * 32 lanes * 4 * 8 = 8192
+// 15 consumer warps + the producer = 16 warps, four per SM sub-partition, which leaves 128
+// registers per thread (a 17th warp would cut that to 96).  The dot products are latency-
+// bound chains of shared-memory loads and FMAs, so warps in flight are what keep the
+// consumers ahead of HBM.
+constexpr int kCW = 15;              // consumer warps
+constexpr int kCT = kCW * 32;        // consumer threads
+constexpr int kThreadsS = kCT + 32;  // + one producer warp
+constexpr int kCPLf = 3;             // 8-element chunks per lane: K <= 15 warps * 32 lanes * 3 * 8 = 11520
+
+__device__ __forceinline__ void csync() { asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory"); }
 
 __device__ __forceinline__ size_t al128(size_t x) { return (x + 127) & ~size_t(127); }
 
@@ -50,28 +59,39 @@ __device__ __forceinline__ void unpack8f(uint4 w, float* f) {
 // Chunk of lane `lane` in warp w's K slice: q = w * qpw + j * 32 + lane, valid if j*32+lane < qpw.
 __device__ __forceinline__ bool cvalid(int qpw, int j, int lane) { return j * 32 + lane < qpw; }
 
-// Dot of one bf16 row (shared memory) with NT register slices; two accumulators per token.
+// Dot of one bf16 row (shared memory) with NT register slices.  Eight independent FMA
+// chains per row (8 / NT accumulators per token) so consecutive FMAs never wait on each
+// other; all chunk loads are issued before the first FMA.
 template <int NT>
 __device__ __forceinline__ void row_dot(const uint16_t* row, const float (&x)[NT][kCPLf][8], int qbase, int qpw,
                                         int lane, float (&out)[NT]) {
-  float acc0[NT], acc1[NT];
+  constexpr int kA = 8 / NT;
+  uint4 w[kCPLf];
 #pragma unroll
-  for (int t = 0; t < NT; ++t) acc0[t] = acc1[t] = 0.f;
+  for (int j = 0; j < kCPLf; ++j)
+    w[j] = cvalid(qpw, j, lane) ? *reinterpret_cast<const uint4*>(row + (size_t)(qbase + j * 32 + lane) * 8)
+                                : make_uint4(0, 0, 0, 0);
+  float acc[NT][kA];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int e = 0; e < kA; ++e) acc[t][e] = 0.f;
 #pragma unroll
   for (int j = 0; j < kCPLf; ++j) {
-    if (!cvalid(qpw, j, lane)) continue;
-    const uint4 w = *reinterpret_cast<const uint4*>(row + (size_t)(qbase + j * 32 + lane) * 8);
     float wf[8];
-    unpack8f(w, wf);
+    unpack8f(w[j], wf);
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      float& acc = (j & 1) ? acc1[t] : acc0[t];
+    for (int t = 0; t < NT; ++t)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc = fmaf(wf[e], x[t][j][e], acc);
-    }
+      for (int e = 0; e < 8; ++e) acc[t][e % kA] = fmaf(wf[e], x[t][j][e], acc[t][e % kA]);
   }
 #pragma unroll
-  for (int t = 0; t < NT; ++t) out[t] = acc0[t] + acc1[t];
+  for (int t = 0; t < NT; ++t) {
+    float v = 0.f;
+#pragma unroll
+    for (int e = 0; e < kA; ++e) v += acc[t][e];
+    out[t] = v;
+  }
 }
 
 }  // namespace
@@ -81,7 +101,7 @@ __device__ __forceinline__ void row_dot(const uint16_t* row, const float (&x)[NT
 //   CTA c owns rows [r0, r1) of W_o (contiguous); a stage is RS whole rows (one copy).
 // =============================================================================
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) k_oproj_f(const LayerArgs a) {
+__global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, d_o = a.d_o, B = a.B;
@@ -94,8 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_oproj_f(const LayerArgs a) {
 
   unsigned char* ring = smem;
   float* part = reinterpret_cast<float*>(ring + (size_t)S * SB);  // [RM][8][NT]
-  float* sq = part + RM * kConsumerWarps * NT;                     // [NT][RM]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + al128((size_t)S * SB + ((size_t)RM * kConsumerWarps * NT +
+  float* sq = part + RM * kCW * NT;                     // [NT][RM]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + al128((size_t)S * SB + ((size_t)RM * kCW * NT +
                                                                               (size_t)NT * RM) * 4));
   uint64_t* empty = full + S;
   int* s_misc = reinterpret_cast<int*>(empty + S);
@@ -103,14 +123,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_oproj_f(const LayerArgs a) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   if (tid == 0) {
-    init_ring(full, empty, S);
+    init_ring(full, empty, S, kCW);
     s_misc[0] = 0;
     fence_barrier_init();
   }
   __syncthreads();
   pdl_trigger();
 
-  if (warp == kConsumerWarps) {
+  if (warp == kCW) {
     if (lane == 0) {  // W_o is static: stream it before the dependency resolves
       const uint64_t pol = policy_evict_first();
       int it = 0;
@@ -127,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_oproj_f(const LayerArgs a) {
   }
 
   pdl_wait();  // attn_out and residual may come from the previous kernel
-  const int qpw = d_o / 64, qbase = warp * qpw;
+  const int qbase = (d_o / 8) * warp / kCW, qpw = (d_o / 8) * (warp + 1) / kCW - qbase;
   float xa[NT][kCPLf][8];
 #pragma unroll
   for (int t = 0; t < NT; ++t)
@@ -148,24 +168,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_oproj_f(const LayerArgs a) {
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         const float w = warp_sum(v[t]);
-        if (lane == 0) part[((r - r0 + j) * kConsumerWarps + warp) * NT + t] = w;
+        if (lane == 0) part[((r - r0 + j) * kCW + warp) * NT + t] = w;
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
   }
-  consumer_sync();
-  for (int z = tid; z < rows * B; z += kConsumerThreads) {
+  csync();
+  for (int z = tid; z < rows * B; z += kCT) {
     const int rr = z / B, t = z % B;
     float sacc = 0.f;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) sacc += part[(rr * kConsumerWarps + w) * NT + t];
+    for (int w = 0; w < kCW; ++w) sacc += part[(rr * kCW + w) * NT + t];
     const size_t o = (size_t)t * d + r0 + rr;
     const float hv = bf16f(__ldcg(reinterpret_cast<const unsigned short*>(a.resid + o))) + sacc;
     a.ws.h[o] = hv;
     sq[t * RM + rr] = hv * hv;
   }
-  consumer_sync();
+  csync();
   if (warp < B) {  // per-CTA sum of h^2, fixed order
     float ss = 0.f;
     for (int rr = lane; rr < rows; rr += 32) ss += sq[warp * RM + rr];
@@ -180,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_oproj_f(const LayerArgs a) {
 //   the dependency wait.  x is exact fp32 in registers.
 // =============================================================================
 template <int NT>
-__global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
+__global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, E = a.E, B = a.B;
@@ -192,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
 
   uint16_t* wsl = reinterpret_cast<uint16_t*>(smem);                                 // [RM][d]
   float* part = reinterpret_cast<float*>(smem + al128((size_t)RM * row_bytes));    // [RM][8][NT]
-  float* rstd_s = part + RM * kConsumerWarps * NT;                                  // [64]
+  float* rstd_s = part + RM * kCW * NT;                                  // [64]
   uint64_t* full = reinterpret_cast<uint64_t*>(
       smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(rstd_s + 64) - smem)));
   int* s_misc = reinterpret_cast<int*>(full + 1);
@@ -209,14 +229,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
   __syncthreads();
   pdl_trigger();
 
-  if (warp == kConsumerWarps) {
+  if (warp == kCW) {
     if (lane == 0 && nrows > 0) {
       mbar_arrive_expect_tx(&full[0], nrows * row_bytes);
       bulk_g2s(wsl, a.w_r + (size_t)e0 * d, nrows * row_bytes, &full[0], policy_evict_first());
       mbar_drain(&full[0], 0, a.ws.err);
     }
   } else {
-    const int qpw = d / 64, qbase = warp * qpw;
+    const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
     float gam[kCPLf][8];
 #pragma unroll
     for (int j = 0; j < kCPLf; ++j) {
@@ -225,7 +245,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
       unpack8f(u, gam[j]);
     }
     pdl_wait();  // h and the sums of h^2 come from the o_proj kernel
-    for (int t = warp; t < B; t += kConsumerWarps) {  // fixed order: same bits in every CTA
+    if (c == 0 && tid == 0) a.ws.counters[kCntGateUp] = 0;  // the expert kernel's grid barrier count
+    // h of the first token group, loaded while the sums of h^2 are reduced
+    float xr[NT][kCPLf][8];
+    auto load_h = [&](int t0, int nt) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int j = 0; j < kCPLf; ++j) {
+          if (t < nt && cvalid(qpw, j, lane)) {
+            const float* hp = a.ws.h + (size_t)(t0 + t) * d + (size_t)(qbase + j * 32 + lane) * 8;
+            const float4 h0 = ld_act4(hp), h1 = ld_act4(hp + 4);
+            xr[t][j][0] = h0.x; xr[t][j][1] = h0.y; xr[t][j][2] = h0.z; xr[t][j][3] = h0.w;
+            xr[t][j][4] = h1.x; xr[t][j][5] = h1.y; xr[t][j][6] = h1.z; xr[t][j][7] = h1.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+          }
+        }
+    };
+    load_h(0, min(NT, B));
+    for (int t = warp; t < B; t += kCW) {  // fixed order: same bits in every CTA
       float ss = 0.f;
       for (int cc = lane; cc < G; cc += 32) ss += ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]);
       ss = warp_sum(ss);
@@ -235,31 +275,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
         if (c == 0) a.ws.rstd[t] = r;
       }
     }
-    consumer_sync();
+    csync();
     bool have_w = false;
     for (int t0 = 0; t0 < B; t0 += NT) {
       const int nt = min(NT, B - t0);
-      float xr[NT][kCPLf][8];
+      if (t0 > 0) load_h(t0, nt);
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         const float r = (t < nt) ? rstd_s[t0 + t] : 0.f;
 #pragma unroll
         for (int j = 0; j < kCPLf; ++j) {
           const int q = qbase + j * 32 + lane;
-          if (t < nt && cvalid(qpw, j, lane)) {
-            const float* hp = a.ws.h + (size_t)(t0 + t) * d + (size_t)q * 8;
-            const float4 h0 = ld_act4(hp), h1 = ld_act4(hp + 4);
-            const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) xr[t][j][e] = hv[e] * r * gam[j][e];
-            if (q % G == c) {  // each chunk of x is written to global memory by exactly one CTA
-              float* xp = a.ws.x + (size_t)(t0 + t) * d + (size_t)q * 8;
-              *reinterpret_cast<float4*>(xp) = make_float4(xr[t][j][0], xr[t][j][1], xr[t][j][2], xr[t][j][3]);
-              *reinterpret_cast<float4*>(xp + 4) = make_float4(xr[t][j][4], xr[t][j][5], xr[t][j][6], xr[t][j][7]);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+          for (int e = 0; e < 8; ++e) xr[t][j][e] = xr[t][j][e] * r * gam[j][e];
+          if (t < nt && cvalid(qpw, j, lane) && q % G == c) {  // each chunk of x is written by one CTA
+            float* xp = a.ws.x + (size_t)(t0 + t) * d + (size_t)q * 8;
+            *reinterpret_cast<float4*>(xp) = make_float4(xr[t][j][0], xr[t][j][1], xr[t][j][2], xr[t][j][3]);
+            *reinterpret_cast<float4*>(xp + 4) = make_float4(xr[t][j][4], xr[t][j][5], xr[t][j][6], xr[t][j][7]);
           }
         }
       }
@@ -274,19 +306,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
             const float w = warp_sum(v[t]);
-            if (lane == 0) part[(j * kConsumerWarps + warp) * NT + t] = w;
+            if (lane == 0) part[(j * kCW + warp) * NT + t] = w;
           }
         }
       }
-      consumer_sync();
-      for (int z = tid; z < nrows * nt; z += kConsumerThreads) {
+      csync();
+      for (int z = tid; z < nrows * nt; z += kCT) {
         const int j = z / nt, t = z % nt;
         float s = 0.f;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w) s += part[(j * kConsumerWarps + w) * NT + t];
+        for (int w = 0; w < kCW; ++w) s += part[(j * kCW + w) * NT + t];
         a.ws.logits[(size_t)(t0 + t) * E + e0 + j] = s;
       }
-      consumer_sync();
+      csync();
     }
   }
   if (a.route_tables) {  // large-batch expert kernels: the last CTA builds the routing tables
@@ -299,10 +331,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_router_f(const LayerArgs a) {
 
 // =============================================================================
 // Grid barrier for the expert kernel (cooperative launch: every CTA is resident).
-// Sense reversal: each CTA reads the generation before it arrives, the last arrival resets
-// the count and advances the generation, the others wait for the advance.  The wait is
-// bounded in time; on expiry the CTA records kErrTimeout and carries on (its results are
-// then meaningless, and the error word says so).  Called by the consumer warps only.
+// Each CTA adds one to a counter with release semantics and waits (acquire loads) until it
+// reaches the grid size.  The wait is bounded in time; on expiry the CTA records
+// kErrTimeout and carries on (its results are then meaningless, and the error word says
+// so).  Called by the consumer warps only.
 // =============================================================================
 namespace {
 
@@ -312,30 +344,32 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
-__device__ void grid_barrier(unsigned* count, unsigned* gen, volatile int* abort_flag, uint32_t* err) {
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// `count` is zero when the kernel starts (the router kernel clears it before its dependents
+// pass their dependency wait) and is used once per launch: the barrier opens when it reaches
+// gridDim.x, so the last arrival's add is the release (no second round trip).
+__device__ void grid_barrier(unsigned* count, volatile int* abort_flag, uint32_t* err) {
   __threadfence();
-  consumer_sync();
+  csync();
   if (threadIdx.x == 0) {
-    const unsigned g = ld_acquire_u32(gen);
-    const unsigned arrived = atomicAdd(count, 1u) + 1u;
-    if (arrived == gridDim.x) {
-      atomicExch(count, 0u);
-      __threadfence();
-      atomicExch(gen, g + 1u);
-    } else {
+    red_release_add(count, 1u);
+    const unsigned target = gridDim.x;
+    if (ld_acquire_u32(count) < target) {
       const unsigned long long t0 = globaltimer();
-      while (ld_acquire_u32(gen) == g) {
+      while (ld_acquire_u32(count) < target) {
         if (globaltimer() - t0 > kWaitLimitNs) {
           *abort_flag = 1;
           atomicOr(err, kErrTimeout);
           break;
         }
-        __nanosleep(64);
+        __nanosleep(32);
       }
     }
-    __threadfence();
   }
-  consumer_sync();
+  csync();
 }
 
 }  // namespace
@@ -353,9 +387,9 @@ __device__ void grid_barrier(unsigned* count, unsigned* gen, volatile int* abort
 //            in registers; one warp reduction per (row, token) at the end.
 // =============================================================================
 template <int NT, int EPL>
-__global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
+__global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kRPW = 7;  // rows per warp in phase B (rows_max <= 56)
+  constexpr int kRPW = 4;  // rows per warp in phase B (rows_max <= 64)
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, I = a.I, B = a.B;
   const int SA = a.k3.stages, PS = a.k3.rows_per_stage, PM = a.k3.rows_max;
@@ -363,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
   const uint32_t row_bytes = (uint32_t)d * 2u, drow_bytes = (uint32_t)I * 2u;
   const size_t SA_B = al128((size_t)2 * PS * row_bytes), SB_B = al128((size_t)RM * drow_bytes);
   const size_t region = std::max((size_t)SA * SA_B, (size_t)SBn * SB_B);
-  const size_t scratch_f = std::max((size_t)PM * 2 * kConsumerWarps * NT, (size_t)B * a.k * I);  // floats
+  const size_t scratch_f = std::max((size_t)PM * 2 * kCW * NT, (size_t)B * a.k * I);  // floats
   long long lo, hi;
   split_range(d, G, c, lo, hi);
   const int i0 = (int)lo, nrows = (int)(hi - lo);
@@ -384,18 +418,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   if (tid == 0) {
-    init_ring(fullA, emptyA, SA);
-    init_ring(fullB, emptyB, SBn);
+    init_ring(fullA, emptyA, SA, kCW);
+    init_ring(fullB, emptyB, SBn, kCW);
     s_misc[0] = 0;
     fence_barrier_init();
   }
   pdl_wait();  // logits and x come from the router kernel
   pdl_trigger();
 
-  // x of every token, in registers (consumers; issued before routing to overlap it).
-  const int qpw = d / 64, qbase = warp * qpw;
+  route_small_cta(a, rt, sc, fb, c == 0);  // barriers inside also publish the ring init
+  // x of every token, in registers (consumers).  Loaded after routing: the loads hit L2 and
+  // land before the first weight stage, and holding x across the routing code would spill.
+  const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
   float xr[NT][kCPLf][8];
-  if (warp < kConsumerWarps) {
+  if (warp < kCW) {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
@@ -411,20 +447,28 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
         }
       }
   }
-  route_small_cta(a, rt, sc, fb, c == 0);  // barriers inside also publish the ring init
 
   const int U = rt->U;
   long long q0l, q1l;
   split_range((long long)U * I, G, c, q0l, q1l);
   const int q0 = (int)q0l, q1 = (int)q1l;
 
-  if (warp == kConsumerWarps) {
+  if (warp == kCW) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
+      // This CTA's W_down blocks go to L2 once the ring is primed, so phase B reads them
+      // from L2 instead of waiting on HBM after the barrier.
+      bool prefetched = false;
+      auto prefetch_down = [&]() {
+        for (int uu = 0; uu < U && nrows > 0; ++uu)
+          bulk_prefetch_l2(a.w_down + ((size_t)rt->un_e[uu] * d + i0) * I, nrows * drow_bytes);
+        prefetched = true;
+      };
       // phase A: gate/up rows
       int it = 0;
       int u = q0 / I, p = q0 - u * I;
       for (int q = q0; q < q1; ++it) {
+        if (it == SA && !prefetched) prefetch_down();
         const int np = min(min(PS, I - p), q1 - q);
         if (!ring_acquire(emptyA, it, SA, abort_flag, a.ws.err)) break;
         const int s = it % SA;
@@ -436,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
         p += np;
         if (p == I) { p = 0; ++u; }
       }
+      if (!prefetched) prefetch_down();
       // The ring is reused by phase B only after every phase-A fill has landed and been read.
       ring_drain(fullA, it, SA, a.ws.err);
       for (int i = it - SA < 0 ? 0 : it - SA; i < it; ++i) mbar_drain(&emptyA[i % SA], (i / SA) & 1, a.ws.err);
@@ -470,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
           const float w = warp_sum(v[t]);
-          if (lane == 0) part[(((q - q0 + pi) * 2 + gu) * kConsumerWarps + warp) * NT + t] = w;
+          if (lane == 0) part[(((q - q0 + pi) * 2 + gu) * kCW + warp) * NT + t] = w;
         }
       }
       __syncwarp();
@@ -479,14 +524,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
       p += np;
       if (p == I) p = 0;
     }
-    consumer_sync();
-    for (int z = tid; z < (q1 - q0) * B; z += kConsumerThreads) {
+    csync();
+    for (int z = tid; z < (q1 - q0) * B; z += kCT) {
       const int pl = z / B, t = z % B;
       float gs = 0.f, us = 0.f;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        gs += part[((pl * 2 + 0) * kConsumerWarps + w) * NT + t];
-        us += part[((pl * 2 + 1) * kConsumerWarps + w) * NT + t];
+      for (int w = 0; w < kCW; ++w) {
+        gs += part[((pl * 2 + 0) * kCW + w) * NT + t];
+        us += part[((pl * 2 + 1) * kCW + w) * NT + t];
       }
       const int qq = q0 + pl, u = qq / I, pp = qq - u * I;
       for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
@@ -494,17 +539,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
     }
   }
 
-  grid_barrier(&a.ws.counters[kCntGateUp], &a.ws.counters[kCntGateUp + 1], abort_flag, a.ws.err);
+  grid_barrier(&a.ws.counters[kCntGateUp], abort_flag, a.ws.err);
 
   // ---- phase B (consumers) ------------------------------------------------------------
   const int nent = rt->n_ent;
-  for (int z = tid; z < nent * (I / 4); z += kConsumerThreads) {
+  for (int z = tid; z < nent * (I / 4); z += kCT) {
     const int en = z / (I / 4), cq = z - en * (I / 4);
     const float g = rt->ent_gate[en];
     const float4 v = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
     *reinterpret_cast<float4*>(a_s + (size_t)en * I + cq * 4) = make_float4(g * v.x, g * v.y, g * v.z, g * v.w);
   }
-  consumer_sync();
+  csync();
 
   const int epl = (EPL > 0) ? EPL : I / 32;
   float acc[kRPW][NT];
@@ -532,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
       }
 #pragma unroll
       for (int i = 0; i < kRPW; ++i) {
-        const int rl = warp + kConsumerWarps * i;
+        const int rl = warp + kCW * i;
         if (rl < nrows) {
           const uint16_t* wr = st + (size_t)rl * I + lane * epl;
           float sdot = 0.f;
@@ -564,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_experts_f(const LayerArgs a) {
   }
 #pragma unroll
   for (int i = 0; i < kRPW; ++i) {
-    const int rl = warp + kConsumerWarps * i;
+    const int rl = warp + kCW * i;
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       const float v = warp_sum(acc[i][t]);
@@ -587,7 +632,7 @@ cudaError_t launch_f(Kern k, int grid, size_t smem, cudaStream_t s, bool pdl, co
                      bool cooperative = false) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kThreadsS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
@@ -622,7 +667,7 @@ bool plan_small(LayerArgs& a, int G, size_t optin) {
     t.rows_max = (a.d + G - 1) / G;
     t.rows_per_stage = (int)std::max<size_t>(1, std::min<size_t>(32768 / row, (size_t)t.rows_max));
     const size_t SB = up128((size_t)t.rows_per_stage * row);
-    const size_t extra = up128(((size_t)t.rows_max * kConsumerWarps * NT + (size_t)NT * t.rows_max) * 4) +
+    const size_t extra = up128(((size_t)t.rows_max * kCW * NT + (size_t)NT * t.rows_max) * 4) +
                          2 * kMaxStages * 8 + 64;
     t.stages = (int)std::min<size_t>(kMaxStages, (std::min(budget, kRingCap) - extra) / SB);
     if (t.stages < 2) return false;
@@ -631,7 +676,7 @@ bool plan_small(LayerArgs& a, int G, size_t optin) {
   {  // K2: the whole router slice
     KTune& t = a.k2;
     t.rows_max = (a.E + G - 1) / G;
-    t.smem = up128((size_t)t.rows_max * a.d * 2) + up128((size_t)t.rows_max * kConsumerWarps * NT * 4 + 64 * 4) +
+    t.smem = up128((size_t)t.rows_max * a.d * 2) + up128((size_t)t.rows_max * kCW * NT * 4 + 64 * 4) +
              8 + 32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
     if (t.smem > budget) return false;
   }
@@ -642,8 +687,8 @@ bool plan_small(LayerArgs& a, int G, size_t optin) {
     const long long umax = std::min(a.E, std::max(a.B, 1) * a.k);
     t.rows_max = (int)((umax * a.I + G - 1) / G);  // pairs per CTA
     t4.rows_max = (a.d + G - 1) / G;                // output rows per CTA
-    if (t4.rows_max > 7 * kConsumerWarps) return false;
-    const size_t scratch_f = std::max((size_t)t.rows_max * 2 * kConsumerWarps * NT, (size_t)std::max(a.B, 1) * a.k * a.I);
+    if (t4.rows_max > 4 * kCW) return false;
+    const size_t scratch_f = std::max((size_t)t.rows_max * 2 * kCW * NT, (size_t)std::max(a.B, 1) * a.k * a.I);
     const size_t extra = up128(scratch_f * 4) + kRouteBytes + 4 * kMaxStages * 8 + 64;
     const size_t SBd = up128((size_t)t4.rows_max * a.I * 2);
     t.stages = 0;
@@ -674,7 +719,7 @@ bool router_ok(const LayerArgs& a0, size_t optin) {
   const int G = 148;
   KTune& t = a.k2;
   t.rows_max = (a.E + G - 1) / G;
-  t.smem = up128((size_t)t.rows_max * a.d * 2) + up128((size_t)t.rows_max * kConsumerWarps * 2 * 4 + 64 * 4) + 8 +
+  t.smem = up128((size_t)t.rows_max * a.d * 2) + up128((size_t)t.rows_max * kCW * 2 * 4 + 64 * 4) + 8 +
            32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
   return a.d <= 8192 && t.smem <= optin - 1024 - 256;
 }
@@ -715,7 +760,7 @@ cudaError_t launch_oproj_s(const LayerArgs& a0, int grid, cudaStream_t s, bool p
 cudaError_t launch_router_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   LayerArgs a = a0;
   a.k2.rows_max = (a.E + grid - 1) / grid;
-  a.k2.smem = up128((size_t)a.k2.rows_max * a.d * 2) + up128((size_t)a.k2.rows_max * kConsumerWarps * 2 * 4 + 64 * 4) +
+  a.k2.smem = up128((size_t)a.k2.rows_max * a.d * 2) + up128((size_t)a.k2.rows_max * kCW * 2 * 4 + 64 * 4) +
               8 + 32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
   (void)optin;
   return a.B == 1 ? launch_f(k_router_f<1>, grid, a.k2.smem, s, pdl, a) : launch_f(k_router_f<2>, grid, a.k2.smem, s, pdl, a);

@@ -319,7 +319,7 @@ namespace moe {
 // (expert, token) and the union of experts indexed in the same pass.  Falls back to a warp
 // arg-max selection when more than kCandMax logits reach the bound.
 struct RouteScratch {
-  float gmax[2][64];
+  float gmax[2][128];  // quarter-warp maxima (blockDim.x <= 1024)
   float T[2];
   int cnt[2];
   float cv[2][kCandMax];
@@ -336,7 +336,7 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
                                 bool write_user) {
   const int B = a.B, E = a.E, K = a.k;
   const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kPer = 8;  // logits per thread per token (E <= kPer * nth)
+  constexpr int kPer = 2;  // logits per thread per token (E <= kPer * nth: 1024 at 512 threads)
   const int ngroups = nth / 8;  // quarter-warp groups
   float v[2][kPer];
 #pragma unroll
