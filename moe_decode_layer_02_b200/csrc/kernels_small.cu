@@ -29,6 +29,7 @@
 // kernels", section "How the specialised decode path works" (small-matrix kernels at
 // batch one or two; o_proj fused with the residual step; 16 of 896 experts per token).
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -45,6 +46,7 @@ namespace {
 constexpr int kCW = 15;              // consumer warps
 constexpr int kCT = kCW * 32;        // consumer threads
 constexpr int kThreadsS = kCT + 32;  // + one producer warp
+static_assert(kThreadsS == kRouteThreads, "the expert kernel routes with all of its threads");
 constexpr int kCPLf = 3;             // 8-element chunks per lane: K <= 15 warps * 32 lanes * 3 * 8 = 11520
 
 __device__ __forceinline__ void csync() { asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory"); }
@@ -56,42 +58,93 @@ __device__ __forceinline__ void unpack8f(uint4 w, float* f) {
   f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
 }
 
+// Phase B experts per stage for EPL elements per lane (registers bound it).
+__host__ __device__ constexpr int experts_per_stage(int epl) { return epl == 4 ? 4 : (epl == 8 ? 2 : 1); }
+
 // Chunk of lane `lane` in warp w's K slice: q = w * qpw + j * 32 + lane, valid if j*32+lane < qpw.
 __device__ __forceinline__ bool cvalid(int qpw, int j, int lane) { return j * 32 + lane < qpw; }
 
-// Dot of one bf16 row (shared memory) with NT register slices.  Eight independent FMA
-// chains per row (8 / NT accumulators per token) so consecutive FMAs never wait on each
-// other; all chunk loads are issued before the first FMA.
-template <int NT>
-__device__ __forceinline__ void row_dot(const uint16_t* row, const float (&x)[NT][kCPLf][8], int qbase, int qpw,
-                                        int lane, float (&out)[NT]) {
-  constexpr int kA = 8 / NT;
-  uint4 w[kCPLf];
+// Per-lane partial dots of R bf16 rows (shared memory) with NT register slices of the
+// activations: out[r * NT + t].  Rows r >= nr contribute zeros.  All chunk loads of all
+// rows are issued before the first FMA, and the R * NT * kA accumulators are independent
+// FMA chains (kA per row and token), so a warp's pass over a stage is one short chain
+// instead of R dependent ones.
+template <int NT, int R>
+__device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr, const float (&x)[NT][kCPLf][8],
+                                         int qbase, int qpw, int lane, float (&out)[R * NT]) {
+  constexpr int kA = (R * NT >= 8) ? 1 : 8 / (R * NT);
+  uint4 w[R][kCPLf];
 #pragma unroll
-  for (int j = 0; j < kCPLf; ++j)
-    w[j] = cvalid(qpw, j, lane) ? *reinterpret_cast<const uint4*>(row + (size_t)(qbase + j * 32 + lane) * 8)
-                                : make_uint4(0, 0, 0, 0);
-  float acc[NT][kA];
+  for (int r = 0; r < R; ++r)
 #pragma unroll
-  for (int t = 0; t < NT; ++t)
+    for (int j = 0; j < kCPLf; ++j)
+      w[r][j] = (r < nr && cvalid(qpw, j, lane))
+                    ? *reinterpret_cast<const uint4*>(rp[r] + (size_t)(qbase + j * 32 + lane) * 8)
+                    : make_uint4(0, 0, 0, 0);
+  float acc[R][NT][kA];
 #pragma unroll
-    for (int e = 0; e < kA; ++e) acc[t][e] = 0.f;
-#pragma unroll
-  for (int j = 0; j < kCPLf; ++j) {
-    float wf[8];
-    unpack8f(w[j], wf);
+  for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[t][e % kA] = fmaf(wf[e], x[t][j][e], acc[t][e % kA]);
-  }
+      for (int e = 0; e < kA; ++e) acc[r][t][e] = 0.f;
 #pragma unroll
-  for (int t = 0; t < NT; ++t) {
-    float v = 0.f;
+  for (int j = 0; j < kCPLf; ++j)
 #pragma unroll
-    for (int e = 0; e < kA; ++e) v += acc[t][e];
-    out[t] = v;
+    for (int r = 0; r < R; ++r) {
+      float wf[8];
+      unpack8f(w[r][j], wf);
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[r][t][e % kA] = fmaf(wf[e], x[t][j][e], acc[r][t][e % kA]);
+    }
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float v = 0.f;
+#pragma unroll
+      for (int e = 0; e < kA; ++e) v += acc[r][t][e];
+      out[r * NT + t] = v;
+    }
+}
+
+// Warp sums of V per-lane values (V a power of two <= 32) with V - 1 + 5 - log2(V) shuffles
+// instead of 5 V: each halving step sends one value of every pair across the current lane
+// bit and keeps the other.  Every lane returns the total of value multi_index<V>(lane).
+template <int V>
+__device__ __forceinline__ float warp_reduce_multi(float (&v)[V], int lane) {
+  static_assert(V >= 1 && V <= 32 && (V & (V - 1)) == 0, "V must be a power of two <= 32");
+#pragma unroll
+  for (int o = 16, c = V; c > 1; o >>= 1, c >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < c / 2; ++j) {
+      const float send = up ? v[2 * j] : v[2 * j + 1];
+      const float keep = up ? v[2 * j + 1] : v[2 * j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
   }
+  float s = v[0];
+#pragma unroll
+  for (int o = 16 / V; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
+}
+
+// Value index held by `lane` after warp_reduce_multi<V>: bit k of the index is lane bit 4 - k.
+template <int V>
+__device__ __forceinline__ int multi_index(int lane) {
+  int idx = 0;
+#pragma unroll
+  for (int k = 0, c = V; c > 1; ++k, c >>= 1) idx |= ((lane >> (4 - k)) & 1) << k;
+  return idx;
+}
+
+// One lane per group of 32 / V holds each total.
+template <int V>
+__device__ __forceinline__ bool multi_writer(int lane) {
+  return (lane & (32 / V - 1)) == 0;
 }
 
 }  // namespace
@@ -147,6 +200,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
   }
 
   pdl_wait();  // attn_out and residual may come from the previous kernel
+  constexpr int kRI = 2;  // rows per interleaved pass (a stage is two rows at d_o = 8192)
   const int qbase = (d_o / 8) * warp / kCW, qpw = (d_o / 8) * (warp + 1) / kCW - qbase;
   float xa[NT][kCPLf][8];
 #pragma unroll
@@ -162,14 +216,15 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
     const int n = min(RS, r1 - r), s = it % S;
     mbar_wait(&full[s], (it / S) & 1, abort_flag, a.ws.err);
     const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB);
-    for (int j = 0; j < n; ++j) {
-      float v[NT];
-      row_dot<NT>(st + (size_t)j * d_o, xa, qbase, qpw, lane, v);
+    for (int j0 = 0; j0 < n; j0 += kRI) {
+      const uint16_t* rp[kRI];
 #pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        const float w = warp_sum(v[t]);
-        if (lane == 0) part[((r - r0 + j) * kCW + warp) * NT + t] = w;
-      }
+      for (int k = 0; k < kRI; ++k) rp[k] = st + (size_t)min(j0 + k, n - 1) * d_o;
+      float v[kRI * NT];
+      rows_dot<NT, kRI>(rp, n - j0, xa, qbase, qpw, lane, v);
+      const float tot = warp_reduce_multi<kRI * NT>(v, lane);
+      const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
+      if (multi_writer<kRI * NT>(lane) && j < n) part[((r - r0 + j) * kCW + warp) * NT + t] = tot;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -267,7 +322,16 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
     load_h(0, min(NT, B));
     for (int t = warp; t < B; t += kCW) {  // fixed order: same bits in every CTA
       float ss = 0.f;
-      for (int cc = lane; cc < G; cc += 32) ss += ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]);
+      for (int c0 = 0; c0 < G; c0 += 8 * 32) {  // eight independent loads per lane in flight
+        float pv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int cc = c0 + k * 32 + lane;
+          pv[k] = cc < G ? ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss += pv[k];
+      }
       ss = warp_sum(ss);
       if (lane == 0) {
         const float r = 1.0f / sqrtf(ss / (float)d + a.eps);
@@ -300,14 +364,16 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
           mbar_wait(&full[0], 0, abort_flag, a.ws.err);
           have_w = true;
         }
-        for (int j = 0; j < nrows; ++j) {
-          float v[NT];
-          row_dot<NT>(wsl + (size_t)j * d, xr, qbase, qpw, lane, v);
+        constexpr int kRI = 4 / NT;  // rows per interleaved pass
+        for (int j0 = 0; j0 < nrows; j0 += kRI) {
+          const uint16_t* rp[kRI];
 #pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            const float w = warp_sum(v[t]);
-            if (lane == 0) part[(j * kCW + warp) * NT + t] = w;
-          }
+          for (int k = 0; k < kRI; ++k) rp[k] = wsl + (size_t)min(j0 + k, nrows - 1) * d;
+          float v[kRI * NT];
+          rows_dot<NT, kRI>(rp, nrows - j0, xr, qbase, qpw, lane, v);
+          const float tot = warp_reduce_multi<kRI * NT>(v, lane);
+          const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
+          if (multi_writer<kRI * NT>(lane) && j < nrows) part[(j * kCW + warp) * NT + t] = tot;
         }
       }
       csync();
@@ -352,9 +418,9 @@ __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
 // pass their dependency wait) and is used once per launch: the barrier opens when it reaches
 // gridDim.x, so the last arrival's add is the release (no second round trip).
 __device__ void grid_barrier(unsigned* count, volatile int* abort_flag, uint32_t* err) {
-  __threadfence();
-  csync();
+  csync();  // the CTA's writes happen before thread 0's release (cumulative through the barrier)
   if (threadIdx.x == 0) {
+    __threadfence();
     red_release_add(count, 1u);
     const unsigned target = gridDim.x;
     if (ld_acquire_u32(count) < target) {
@@ -389,15 +455,17 @@ __device__ void grid_barrier(unsigned* count, volatile int* abort_flag, uint32_t
 template <int NT, int EPL>
 __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kRPW = 4;  // rows per warp in phase B (rows_max <= 64)
+  constexpr int kRPW = 4;  // rows per warp in phase B (rows_max <= 60)
+  constexpr int kEPS = experts_per_stage(EPL);
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, I = a.I, B = a.B;
   const int SA = a.k3.stages, PS = a.k3.rows_per_stage, PM = a.k3.rows_max;
   const int SBn = a.k4.stages, RM = a.k4.rows_max;
   const uint32_t row_bytes = (uint32_t)d * 2u, drow_bytes = (uint32_t)I * 2u;
-  const size_t SA_B = al128((size_t)2 * PS * row_bytes), SB_B = al128((size_t)RM * drow_bytes);
+  const size_t SA_B = al128((size_t)2 * PS * row_bytes), SB_B = al128((size_t)kEPS * RM * drow_bytes);
   const size_t region = std::max((size_t)SA * SA_B, (size_t)SBn * SB_B);
-  const size_t scratch_f = std::max((size_t)PM * 2 * kCW * NT, (size_t)B * a.k * I);  // floats
+  const size_t scratch_f =
+      std::max((size_t)PM * 2 * kCW * NT, (size_t)std::min(a.E, B * a.k) * NT * I);  // floats
   long long lo, hi;
   split_range(d, G, c, lo, hi);
   const int i0 = (int)lo, nrows = (int)(hi - lo);
@@ -405,7 +473,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   unsigned char* ring = smem;
   float* part = reinterpret_cast<float*>(ring + region);  // phase A partials, then phase B's a
   float* a_s = part;
-  SmallRoute* rt = reinterpret_cast<SmallRoute*>(part + scratch_f);
+  SmallRoute* rt = reinterpret_cast<SmallRoute*>(smem + al128(region + scratch_f * sizeof(float)));
   RouteScratch* sc = reinterpret_cast<RouteScratch*>(rt + 1);
   float* fb = reinterpret_cast<float*>(sc + 1);
   uint64_t* fullA = reinterpret_cast<uint64_t*>(
@@ -486,13 +554,16 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
       for (int i = it - SA < 0 ? 0 : it - SA; i < it; ++i) mbar_drain(&emptyA[i % SA], (i / SA) & 1, a.ws.err);
       // phase B: this CTA's rows of W_down for every union expert
       if (nrows > 0) {
+        const uint32_t blk = (uint32_t)nrows * drow_bytes;  // one expert's rows for this CTA
         int jt = 0;
-        for (int uu = 0; uu < U; ++uu, ++jt) {
+        for (int u0 = 0; u0 < U; u0 += kEPS, ++jt) {
+          const int ne = min(kEPS, U - u0);
           if (!ring_acquire(emptyB, jt, SBn, abort_flag, a.ws.err)) break;
           const int s = jt % SBn;
-          mbar_arrive_expect_tx(&fullB[s], nrows * drow_bytes);
-          bulk_g2s(ring + s * SB_B, a.w_down + ((size_t)rt->un_e[uu] * d + i0) * I, nrows * drow_bytes, &fullB[s],
-                   pol);
+          mbar_arrive_expect_tx(&fullB[s], ne * blk);
+          for (int e = 0; e < ne; ++e)
+            bulk_g2s(ring + s * SB_B + (size_t)e * blk, a.w_down + ((size_t)rt->un_e[u0 + e] * d + i0) * I, blk,
+                     &fullB[s], pol);
         }
         ring_drain(fullB, jt, SBn, a.ws.err);
       }
@@ -501,6 +572,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   }
 
   // ---- phase A (consumers) ------------------------------------------------------------
+  constexpr int kRI = 4 / NT;  // rows per interleaved pass
   {
     int it = 0;
     int p = q0 - (q0 / I) * I;
@@ -508,14 +580,21 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
       const int np = min(min(PS, I - p), q1 - q), s = it % SA;
       mbar_wait(&fullA[s], (it / SA) & 1, abort_flag, a.ws.err);
       const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SA_B);
-      for (int i = 0; i < 2 * np; ++i) {  // gate rows 0..np-1, then up rows
-        const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
-        float v[NT];
-        row_dot<NT>(st + (size_t)(gu * PS + pi) * d, xr, qbase, qpw, lane, v);
+      const int nrow = 2 * np;  // gate rows 0..np-1, then up rows
+      for (int i0 = 0; i0 < nrow; i0 += kRI) {
+        const uint16_t* rp[kRI];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const float w = warp_sum(v[t]);
-          if (lane == 0) part[(((q - q0 + pi) * 2 + gu) * kCW + warp) * NT + t] = w;
+        for (int k = 0; k < kRI; ++k) {
+          const int i = min(i0 + k, nrow - 1), pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
+          rp[k] = st + (size_t)(gu * PS + pi) * d;
+        }
+        float v[kRI * NT];
+        rows_dot<NT, kRI>(rp, nrow - i0, xr, qbase, qpw, lane, v);
+        const float tot = warp_reduce_multi<kRI * NT>(v, lane);
+        const int vi = multi_index<kRI * NT>(lane), i = i0 + vi / NT, t = vi % NT;
+        if (multi_writer<kRI * NT>(lane) && i < nrow) {
+          const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
+          part[(((q - q0 + pi) * 2 + gu) * kCW + warp) * NT + t] = tot;
         }
       }
       __syncwarp();
@@ -542,82 +621,110 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   grid_barrier(&a.ws.counters[kCntGateUp], abort_flag, a.ws.err);
 
   // ---- phase B (consumers) ------------------------------------------------------------
-  const int nent = rt->n_ent;
-  for (int z = tid; z < nent * (I / 4); z += kCT) {
-    const int en = z / (I / 4), cq = z - en * (I / 4);
-    const float g = rt->ent_gate[en];
-    const float4 v = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
-    *reinterpret_cast<float4*>(a_s + (size_t)en * I + cq * 4) = make_float4(g * v.x, g * v.y, g * v.z, g * v.w);
+  // a_s[u][t][:] = gate * a of (union expert u, token t), zero where t did not select u, so
+  // the accumulation below is branch-free.
+  for (int z = tid; z < U * NT * (I / 4); z += kCT) {
+    const int cq = z % (I / 4), ut = z / (I / 4), t = ut % NT, u = ut / NT;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+      if (rt->ent_tok[en] == t) {
+        const float g = rt->ent_gate[en];
+        const float4 x4 = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
+        v = make_float4(g * x4.x, g * x4.y, g * x4.z, g * x4.w);
+      }
+    *reinterpret_cast<float4*>(a_s + ((size_t)u * NT + t) * I + cq * 4) = v;
   }
   csync();
 
+  // A stage holds EPS experts' blocks of this CTA's rows; every load of a stage is issued
+  // before its FMAs.  Warp w owns rows w, w + 15, ...; lane l holds elements
+  // [l * epl, (l + 1) * epl) of each row and accumulates over all experts in registers.
   const int epl = (EPL > 0) ? EPL : I / 32;
   float acc[kRPW][NT];
 #pragma unroll
   for (int i = 0; i < kRPW; ++i)
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[i][t] = 0.f;
-  for (int u = 0; u < U && nrows > 0; ++u) {
-    const int s = u % SBn;
-    mbar_wait(&fullB[s], (u / SBn) & 1, abort_flag, a.ws.err);
+  int g = 0;
+  for (int u0 = 0; u0 < U && nrows > 0; u0 += kEPS, ++g) {
+    const int s = g % SBn, ne = min(kEPS, U - u0);
+    mbar_wait(&fullB[s], (g / SBn) & 1, abort_flag, a.ws.err);
     const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB_B);
-    for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en) {
-      const int t = rt->ent_tok[en];
-      float av[EPL > 0 ? EPL : 16];
-      const float* ap = a_s + (size_t)en * I + lane * epl;
-      if constexpr (EPL == 4) {
-        const float4 vv = *reinterpret_cast<const float4*>(ap);
-        av[0] = vv.x; av[1] = vv.y; av[2] = vv.z; av[3] = vv.w;
-      } else if constexpr (EPL == 8) {
-        const float4 v0 = *reinterpret_cast<const float4*>(ap), v1 = *reinterpret_cast<const float4*>(ap + 4);
-        av[0] = v0.x; av[1] = v0.y; av[2] = v0.z; av[3] = v0.w; av[4] = v1.x; av[5] = v1.y; av[6] = v1.z; av[7] = v1.w;
-      } else {
+    if constexpr (EPL == 4 || EPL == 8) {
+      using WT = typename std::conditional<EPL == 4, uint2, uint4>::type;
+      float av[kEPS][NT][EPL];
+      WT wv[kEPS][kRPW];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) av[x] = (x < epl) ? ap[x] : 0.f;
+      for (int e = 0; e < kEPS; ++e) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const float* ap = a_s + ((size_t)(u0 + min(e, ne - 1)) * NT + t) * I + lane * EPL;
+#pragma unroll
+          for (int x = 0; x < EPL; x += 4) {
+            const float4 f = (e < ne) ? *reinterpret_cast<const float4*>(ap + x) : make_float4(0.f, 0.f, 0.f, 0.f);
+            av[e][t][x] = f.x; av[e][t][x + 1] = f.y; av[e][t][x + 2] = f.z; av[e][t][x + 3] = f.w;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kRPW; ++i) {
+          const int rl = warp + kCW * i;
+          WT w{};
+          if (e < ne && rl < nrows) w = *reinterpret_cast<const WT*>(st + ((size_t)e * nrows + rl) * I + lane * EPL);
+          wv[e][i] = w;
+        }
       }
+#pragma unroll
+      for (int e = 0; e < kEPS; ++e)
+#pragma unroll
+        for (int i = 0; i < kRPW; ++i) {
+          float wf[8];
+          if constexpr (EPL == 4) {
+            wf[0] = bf16lo(wv[e][i].x); wf[1] = bf16hi(wv[e][i].x);
+            wf[2] = bf16lo(wv[e][i].y); wf[3] = bf16hi(wv[e][i].y);
+          } else {
+            unpack8f(reinterpret_cast<const uint4&>(wv[e][i]), wf);
+          }
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            float sdot = 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) sdot = fmaf(wf[x], av[e][t][x], sdot);
+            acc[i][t] += sdot;
+          }
+        }
+    } else {  // any other I: one expert per stage, epl <= 16 elements per lane
+      const float* ap = a_s + (size_t)u0 * NT * I + lane * epl;
 #pragma unroll
       for (int i = 0; i < kRPW; ++i) {
         const int rl = warp + kCW * i;
         if (rl < nrows) {
           const uint16_t* wr = st + (size_t)rl * I + lane * epl;
-          float sdot = 0.f;
-          if constexpr (EPL == 4) {
-            const uint2 w = *reinterpret_cast<const uint2*>(wr);
-            sdot = fmaf(bf16lo(w.x), av[0], sdot);
-            sdot = fmaf(bf16hi(w.x), av[1], sdot);
-            sdot = fmaf(bf16lo(w.y), av[2], sdot);
-            sdot = fmaf(bf16hi(w.y), av[3], sdot);
-          } else if constexpr (EPL == 8) {
-            const uint4 w = *reinterpret_cast<const uint4*>(wr);
-            float wf[8];
-            unpack8f(w, wf);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) sdot = fmaf(wf[x], av[x], sdot);
-          } else {
+          for (int t = 0; t < NT; ++t) {
+            float sdot = 0.f;
 #pragma unroll
             for (int x = 0; x < 16; ++x)
-              if (x < epl) sdot = fmaf(bf16f(wr[x]), av[x], sdot);
+              if (x < epl) sdot = fmaf(bf16f(wr[x]), ap[(size_t)t * I + x], sdot);
+            acc[i][t] += sdot;
           }
-#pragma unroll
-          for (int tt = 0; tt < NT; ++tt)
-            if (tt == t) acc[i][tt] += sdot;
         }
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&emptyB[s]);
   }
+  {
+    float v[kRPW * NT];
 #pragma unroll
-  for (int i = 0; i < kRPW; ++i) {
-    const int rl = warp + kCW * i;
+    for (int i = 0; i < kRPW; ++i)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      const float v = warp_sum(acc[i][t]);
-      if (lane == 0 && rl < nrows && t < B) {
-        const size_t o = (size_t)t * d + i0 + rl;
-        const __nv_bfloat16 bv = __float2bfloat16_rn(ld_act(&a.ws.h[o]) + v);
-        a.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
-      }
+      for (int t = 0; t < NT; ++t) v[i * NT + t] = acc[i][t];
+    const float tot = warp_reduce_multi<kRPW * NT>(v, lane);
+    const int vi = multi_index<kRPW * NT>(lane), i = vi / NT, t = vi % NT, rl = warp + kCW * i;
+    if (multi_writer<kRPW * NT>(lane) && rl < nrows && t < B) {
+      const size_t o = (size_t)t * d + i0 + rl;
+      const __nv_bfloat16 bv = __float2bfloat16_rn(ld_act(&a.ws.h[o]) + tot);
+      a.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
     }
   }
 }
@@ -688,9 +795,11 @@ bool plan_small(LayerArgs& a, int G, size_t optin) {
     t.rows_max = (int)((umax * a.I + G - 1) / G);  // pairs per CTA
     t4.rows_max = (a.d + G - 1) / G;                // output rows per CTA
     if (t4.rows_max > 4 * kCW) return false;
-    const size_t scratch_f = std::max((size_t)t.rows_max * 2 * kCW * NT, (size_t)std::max(a.B, 1) * a.k * a.I);
+    const int eps = experts_per_stage(a.I / 32);
+    t4.rows_per_stage = eps;
+    const size_t scratch_f = std::max((size_t)t.rows_max * 2 * kCW * NT, (size_t)umax * NT * a.I);
     const size_t extra = up128(scratch_f * 4) + kRouteBytes + 4 * kMaxStages * 8 + 64;
-    const size_t SBd = up128((size_t)t4.rows_max * a.I * 2);
+    const size_t SBd = up128((size_t)eps * t4.rows_max * a.I * 2);
     t.stages = 0;
     for (int ps = 2; ps >= 1 && t.stages < 2; --ps) {
       t.rows_per_stage = ps;

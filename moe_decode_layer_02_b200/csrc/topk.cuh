@@ -7,6 +7,7 @@
 // (16 of 896 experts per token); the renormalised softmax over the selected experts is
 // the layer's stated gate function.
 #pragma once
+#include <cstddef>
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -234,116 +235,61 @@ __device__ void topk_route(const LayerArgs& a, unsigned char* scratch) {
 }  // namespace
 
 // Per-CTA routing of a batch of at most 2 tokens (shared memory only).
-struct SmallRoute {
+struct alignas(16) SmallRoute {
   int U, n_ent;
-  int un_e[64];
-  int un_off[65];
-  int ent_tok[64];
-  float ent_gate[64];
-  int key[64];
-  int idx[2][32];
+  int un_e[64];        // union experts, ascending
+  int un_off[65];      // entries of union expert u: [un_off[u], un_off[u + 1])
+  int ent_tok[64];     // token of each entry (tokens ascending within an expert)
+  float ent_gate[64];  // gate of each entry
+  int idx[2][32];      // per-token selection, descending logit
   float gate[2][32];
 };
 
-namespace {
+// Threads of the CTA that runs route_small_cta.
+constexpr int kRouteThreads = 512;
+constexpr int kRouteGroups = kRouteThreads / 8;  // quarter-warp groups
 
-// Every thread of the CTA calls it (two __syncthreads).  Warps 0..B-1 select; warp 0 sorts
-// the entries by (expert, token) and marks the union.  write_user: store idx / gates to the
-// caller's buffers.
-__device__ void route_small(const LayerArgs& a, SmallRoute* rt, float* cand, bool write_user) {
-  const int B = a.B, E = a.E, K = a.k;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < B) {
-    float* cv = cand + warp * 2 * kCandStride;
-    int* ci = reinterpret_cast<int*>(cv + kCandStride);
-    float my_v = 0.f;
-    int my_i = 0;
-    warp_topk(a.ws.logits + (size_t)warp * E, E, K, cv, ci, lane, my_v, my_i);
-    const float gte = warp_gate(my_v, lane, K);
-    if (lane < K) {
-      const int e = (my_i >= 0 && my_i < E) ? my_i : 0;
-      if (e != my_i) atomicOr(a.ws.err, kErrBounds);
-      rt->idx[warp][lane] = e;
-      rt->gate[warp][lane] = gte;
-      if (write_user) {
-        if (a.user_idx) a.user_idx[warp * K + lane] = e;
-        if (a.user_gate) a.user_gate[warp * K + lane] = gte;
-      }
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const int n = B * K;  // <= 64, keys unique (a token selects an expert at most once)
-    for (int p = lane; p < n; p += 32) {
-      const int t = p / K, j = p % K;
-      const int key = rt->idx[t][j] * 2 + t;
-      int r = 0;
-      for (int o = 0; o < n; ++o) r += (rt->idx[o / K][o % K] * 2 + o / K) < key;
-      rt->key[r] = key;
-      rt->ent_tok[r] = t;
-      rt->ent_gate[r] = rt->gate[t][j];
-    }
-    __syncwarp();
-    int base = 0;
-    for (int p0 = 0; p0 < n; p0 += 32) {
-      const int p = p0 + lane;
-      const bool first = p < n && (p == 0 || (rt->key[p - 1] >> 1) != (rt->key[p] >> 1));
-      const unsigned m = __ballot_sync(0xffffffffu, first);
-      if (first) {
-        const int u = base + __popc(m & ((1u << lane) - 1u));
-        rt->un_e[u] = rt->key[p] >> 1;
-        rt->un_off[u] = p;
-      }
-      base += __popc(m);
-    }
-    if (lane == 0) {
-      rt->U = base;
-      rt->n_ent = n;
-      rt->un_off[base] = n;
-    }
-  }
-  __syncthreads();
-}
-
-}  // namespace
-
-}  // namespace moe
-
-namespace moe {
-
-// CTA-wide routing of a batch of at most 2 tokens (every thread calls it; 7 barriers).
-// Selection with few dependent steps: each thread loads its strided share of the logits;
-// quarter-warp maxima (36 per token at 288 threads) give the lower bound T = their K-th
-// largest value (K groups hold an element >= T, so the K-th largest logit is >= T); the
-// logits >= T are compacted and ranked exactly in parallel.  Entries are then sorted by
-// (expert, token) and the union of experts indexed in the same pass.  Falls back to a warp
-// arg-max selection when more than kCandMax logits reach the bound.
-struct RouteScratch {
-  float gmax[2][128];  // quarter-warp maxima (blockDim.x <= 1024)
-  float T[2];
-  int cnt[2];
-  float cv[2][kCandMax];
-  int ci[2][kCandMax];
-  float sel_v[2][32];
+// Scratch of route_small_cta.  Arrays read with 16-byte vector loads are 16-byte aligned.
+struct alignas(16) RouteScratch {
+  alignas(16) float cv[2][kCandMax];         // candidate logits
+  alignas(16) int ci[2][kCandMax];           // candidate experts
+  alignas(16) float gmax[2][kRouteGroups];   // quarter-warp maxima
+  float sel_v[2][32];                        // selection in rank order
   int sel_i[2][32];
-  int key[64];
-  unsigned emask[32];  // experts selected by token 0
+  unsigned bm[2][32];                        // selected-expert bitmaps (E <= 1024)
+  float T[2];                                // candidate bound per token
+  int cnt[2];                                // candidates per token
 };
+static_assert(offsetof(RouteScratch, cv) % 16 == 0 && offsetof(RouteScratch, ci) % 16 == 0 &&
+                  offsetof(RouteScratch, gmax) % 16 == 0,
+              "vector-loaded routing arrays must be 16-byte aligned");
+static_assert(sizeof(SmallRoute) % 16 == 0, "RouteScratch follows SmallRoute");
 
 namespace {
 
+// CTA-wide routing of a batch of at most 2 tokens (all kRouteThreads threads call it;
+// 5 barriers).
+//  1. each thread loads its strided share of the logits (E <= 2 * kRouteThreads);
+//     quarter-warp maxima go to shared memory;
+//  2. T = the k-th largest of a token's group maxima (each group maximum ranked against
+//     the others in parallel): k groups hold a logit >= T, so the k-th largest logit is >= T;
+//  3. the logits >= T are compacted (one shared atomic per warp);
+//  4. warp t ranks token t's candidates exactly (through shuffles when there are at most 32,
+//     else through shared memory; with more than kCandMax, e.g. mass ties, it selects by
+//     repeated arg-max instead), computes the gates and marks the selection in a bitmap;
+//  5. warp 0 scans the bitmaps (word = lane) and places every entry: its union index and
+//     its position in the (expert, token)-sorted entry list are a scan value plus a popcount.
 __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch* sc, float* fallback_cand,
                                 bool write_user) {
   const int B = a.B, E = a.E, K = a.k;
-  const int tid = threadIdx.x, nth = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kPer = 2;  // logits per thread per token (E <= kPer * nth: 1024 at 512 threads)
-  const int ngroups = nth / 8;  // quarter-warp groups
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kPer = 2;  // logits per thread per token
   float v[2][kPer];
 #pragma unroll
   for (int t = 0; t < 2; ++t)
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-      const int e = tid + i * nth;
+      const int e = tid + i * kRouteThreads;
       float x = -INFINITY;
       if (t < B && e < E) {
         x = ld_act(a.ws.logits + (size_t)t * E + e);
@@ -352,40 +298,47 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
       v[t][i] = x;
     }
   if (tid < 2) sc->cnt[tid] = 0;
-  if (tid < 32) sc->emask[tid] = 0u;
+  if (tid < 64) (&sc->bm[0][0])[tid] = 0u;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) m = fmaxf(m, v[t][i]);
+    float m = fmaxf(v[t][0], v[t][1]);
 #pragma unroll
     for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((lane & 7) == 0 && t < B) sc->gmax[t][tid >> 3] = m;
   }
   __syncthreads();
-  // (2) T[t] = K-th largest group maximum (ties by group index).
-  if (tid < B * ngroups) {
-    const int t = tid / ngroups, gi = tid - t * ngroups;
+  // (2) bound
+  if (tid < B * kRouteGroups) {
+    const int t = tid / kRouteGroups, gi = tid - t * kRouteGroups;
     const float m = sc->gmax[t][gi];
-    int r = 0;
-#pragma unroll 4
-    for (int o = 0; o < ngroups; ++o) {
-      const float x = sc->gmax[t][o];
-      r += (x > m) || (x == m && o < gi);
+    int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+#pragma unroll
+    for (int o = 0; o < kRouteGroups; o += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(&sc->gmax[t][o]);
+      r0 += (x.x > m) || (x.x == m && o < gi);
+      r1 += (x.y > m) || (x.y == m && o + 1 < gi);
+      r2 += (x.z > m) || (x.z == m && o + 2 < gi);
+      r3 += (x.w > m) || (x.w == m && o + 3 < gi);
     }
-    if (r == K - 1) sc->T[t] = m;
+    if ((r0 + r1) + (r2 + r3) == K - 1) sc->T[t] = m;
   }
   __syncthreads();
-  // (3) candidates: logits >= T.
+  // (3) candidates
+  const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     if (t >= B) break;
     const float T = sc->T[t];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-      const int e = tid + i * nth;
-      if (e < E && v[t][i] >= T) {
-        const int slot = atomicAdd(&sc->cnt[t], 1);
+      const int e = tid + i * kRouteThreads;
+      const bool isc = e < E && v[t][i] >= T;
+      const unsigned m = __ballot_sync(0xffffffffu, isc);
+      int base = 0;
+      if (lane == 0 && m) base = atomicAdd(&sc->cnt[t], __popc(m));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (isc) {
+        const int slot = base + __popc(m & lt);
         if (slot < kCandMax) {
           sc->cv[t][slot] = v[t][i];
           sc->ci[t][slot] = e;
@@ -394,80 +347,103 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
     }
   }
   __syncthreads();
-  // (4) exact ranks among the candidates (= ranks among all experts).
-  for (int z = tid; z < 2 * kCandMax; z += nth) {
-    const int t = z / kCandMax, c = z - t * kCandMax;
-    if (t < B) {
-      const int C = sc->cnt[t];
-      if (c < C && C <= kCandMax) {
+  // (4) selection and gates, warp t for token t
+  if (warp < B) {
+    const int t = warp, C = sc->cnt[t];
+    if (C <= 32) {
+      const float x = (lane < C) ? sc->cv[t][lane] : -INFINITY;
+      const int xi = (lane < C) ? sc->ci[t][lane] : 0x7FFFFFFF;  // empty lanes rank last
+      int r = 0;
+#pragma unroll
+      for (int o = 0; o < 32; ++o) r += better(__shfl_sync(0xffffffffu, x, o), __shfl_sync(0xffffffffu, xi, o), x, xi);
+      if (lane < C && r < K) {
+        sc->sel_v[t][r] = x;
+        sc->sel_i[t][r] = xi;
+      }
+    } else if (C <= kCandMax) {
+      for (int c = lane; c < C; c += 32) {
         const float x = sc->cv[t][c];
         const int xi = sc->ci[t][c];
-        int r = 0;
-#pragma unroll 4
-        for (int o = 0; o < C; ++o) r += better(sc->cv[t][o], sc->ci[t][o], x, xi);
+        int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+        for (int o = 0; o < C; o += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(&sc->cv[t][o]);
+          const int4 i4 = *reinterpret_cast<const int4*>(&sc->ci[t][o]);
+          r0 += better(v4.x, i4.x, x, xi);
+          r1 += (o + 1 < C) && better(v4.y, i4.y, x, xi);
+          r2 += (o + 2 < C) && better(v4.z, i4.z, x, xi);
+          r3 += (o + 3 < C) && better(v4.w, i4.w, x, xi);
+        }
+        const int r = (r0 + r1) + (r2 + r3);
         if (r < K) {
           sc->sel_v[t][r] = x;
           sc->sel_i[t][r] = xi;
         }
       }
     }
-  }
-  __syncthreads();
-  // (5) gates (warp t for token t; overflow tokens take the warp arg-max selection).
-  if (warp < B) {
+    __syncwarp();
     float my_v = 0.f;
     int my_i = 0;
-    if (sc->cnt[warp] > kCandMax) {
-      float* cvv = fallback_cand + warp * 2 * kCandStride;
-      warp_topk(a.ws.logits + (size_t)warp * E, E, K, cvv, reinterpret_cast<int*>(cvv + kCandStride), lane, my_v,
+    if (C > kCandMax) {
+      float* cvv = fallback_cand + t * 2 * kCandStride;
+      warp_topk(a.ws.logits + (size_t)t * E, E, K, cvv, reinterpret_cast<int*>(cvv + kCandStride), lane, my_v,
                 my_i);
     } else if (lane < K) {
-      my_v = sc->sel_v[warp][lane];
-      my_i = sc->sel_i[warp][lane];
+      my_v = sc->sel_v[t][lane];
+      my_i = sc->sel_i[t][lane];
     }
     const float gte = warp_gate(my_v, lane, K);
     if (lane < K) {
       const int e = (my_i >= 0 && my_i < E) ? my_i : 0;
       if (e != my_i) atomicOr(a.ws.err, kErrBounds);
-      rt->idx[warp][lane] = e;
-      rt->gate[warp][lane] = gte;
-      sc->key[warp * K + lane] = e * 2 + warp;
-      if (warp == 0) atomicOr(&sc->emask[e >> 5], 1u << (e & 31));
+      rt->idx[t][lane] = e;
+      rt->gate[t][lane] = gte;
+      atomicOr(&sc->bm[t][e >> 5], 1u << (e & 31));
       if (write_user) {
-        if (a.user_idx) a.user_idx[warp * K + lane] = e;
-        if (a.user_gate) a.user_gate[warp * K + lane] = gte;
+        if (a.user_idx) a.user_idx[t * K + lane] = e;
+        if (a.user_gate) a.user_gate[t * K + lane] = gte;
       }
     }
   }
   __syncthreads();
-  // (6) entries sorted by key = expert * 2 + token (unique); an entry opens a union expert
-  // when its token is 0 or token 0 did not select that expert.
-  const int n = B * K;
-  bool opens = false;
-  if (tid < n) {
-    const int key = sc->key[tid], e = key >> 1, t = key & 1;
-    int r = 0, u = 0;
-#pragma unroll 4
-    for (int o = 0; o < n; ++o) {
-      const int k2 = sc->key[o], e2 = k2 >> 1;
-      r += k2 < key;
-      const bool op2 = (k2 & 1) == 0 || !((sc->emask[e2 >> 5] >> (e2 & 31)) & 1u);
-      u += (op2 && e2 < e);
+  // (5) entries sorted by (expert, token); union experts ascending (warp 0)
+  if (warp == 0) {
+    const unsigned b0 = sc->bm[0][lane], b1 = sc->bm[1][lane];
+    const int own = __popc(b0) | (__popc(b1) << 8) | (__popc(b0 | b1) << 16);  // totals <= 64
+    int inc = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
     }
-    opens = (t == 0) || !((sc->emask[e >> 5] >> (e & 31)) & 1u);
-    rt->key[r] = key;
-    rt->ent_tok[r] = t;
-    rt->ent_gate[r] = rt->gate[t][tid - t * K];
-    if (opens) {
-      rt->un_e[u] = e;
-      rt->un_off[u] = r;
+    const int base = inc - own;
+    const int n = B * K;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int p = lane + 32 * h;
+      const int t = (p < n) ? p / K : 0, j = (p < n) ? p - t * K : 0;
+      const int e = rt->idx[t][j], w = e >> 5;
+      const unsigned below = (1u << (e & 31)) - 1u;
+      const int bs = __shfl_sync(0xffffffffu, base, w);
+      const unsigned w0 = __shfl_sync(0xffffffffu, b0, w), w1 = __shfl_sync(0xffffffffu, b1, w);
+      if (p < n) {
+        const int p0 = (bs & 0xFF) + __popc(w0 & below), p1 = ((bs >> 8) & 0xFF) + __popc(w1 & below);
+        const int pu = ((bs >> 16) & 0xFF) + __popc((w0 | w1) & below);
+        const bool t0_has = (w0 >> (e & 31)) & 1u;
+        const int pe = p0 + p1 + ((t == 1 && t0_has) ? 1 : 0);
+        rt->ent_tok[pe] = t;
+        rt->ent_gate[pe] = rt->gate[t][j];
+        if (t == 0 || !t0_has) {  // first entry of expert e
+          rt->un_e[pu] = e;
+          rt->un_off[pu] = pe;
+        }
+      }
     }
-  }
-  const int U = __syncthreads_count(opens);
-  if (tid == 0) {
-    rt->U = U;
-    rt->n_ent = n;
-    rt->un_off[U] = n;
+    if (lane == 31) {
+      const int u = (inc >> 16) & 0xFF;
+      rt->U = u;
+      rt->n_ent = n;
+      rt->un_off[u] = n;
+    }
   }
   __syncthreads();
 }
