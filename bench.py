@@ -1,9 +1,11 @@
 #!/usr/bin/env python
 """Benchmark of the MoE decode-layer step on B200: one JSON line on rank 0.
 
-Metric: microseconds per decode layer-step (device time, L2 flushed before every
-timed step) and the weight bytes the step touched per second as a fraction of the
-measured HBM peak.  A "step" is one call of moe_decode_step: every kernel of the
+Metric: microseconds per decode layer-step (device time; no step finds its weights in
+L2: a one-layer step cycles over 4 independently seeded weight copies, a stack streams
+more than twice the L2 per step) and the weight bytes the step touched per second as a
+fraction of the measured HBM peak.  Secondary figures: the same weights back to back
+(warm) and a 256 MiB L2 flush before each step.  A "step" is one call of moe_decode_step: every kernel of the
 layer (or of the 8-layer stack) on one batch of seeded synthetic inputs.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--prefetch 0|1]
@@ -71,6 +73,11 @@ def dims_of(name):
 def seed_of(dname, L):
     import synth
     return synth.config_seed({"TP16": 1, "TP8": 3, "TP16E64": 21, "TP8E64": 23}[dname] + (10 if L > 1 else 0))
+
+
+def rotation(L):
+    """Weight copies a single-layer step cycles over (4 x >= 218 MB > 2 x the 126 MB L2)."""
+    return 4 if L == 1 else 1
 
 
 def token_inputs(seed, dims, B, L, mode):
@@ -199,14 +206,18 @@ def run_ours(args, rank, world):
     dims = dims_of(dname)
     seed = seed_of(dname, L)
     sz = dims.sizes()
-    weights = []
-    for l in range(L):
-        t = {}
-        for kind in (synth.W_O, synth.GAMMA, synth.W_R, synth.W_GU, synth.W_DOWN):
-            x = torch.empty(sz[kind], dtype=torch.bfloat16, device="cuda")
-            synth.device_fill(x, seed, kind, layer=l)
-            t[kind] = x
-        weights.append((t[synth.W_O], t[synth.GAMMA], t[synth.W_R], t[synth.W_GU], t[synth.W_DOWN]))
+    R = rotation(L)
+    weight_sets = []
+    for r in range(R):  # independently seeded copies; a timed step uses copy i % R
+        weights = []
+        for l in range(L):
+            t = {}
+            for kind in (synth.W_O, synth.GAMMA, synth.W_R, synth.W_GU, synth.W_DOWN):
+                x = torch.empty(sz[kind], dtype=torch.bfloat16, device="cuda")
+                synth.device_fill(x, seed + 1000 * r, kind, layer=l)
+                t[kind] = x
+            weights.append((t[synth.W_O], t[synth.GAMMA], t[synth.W_R], t[synth.W_GU], t[synth.W_DOWN]))
+        weight_sets.append(weights)
     attn_np, resid_np = token_inputs(seed, dims, B, L, mode)
     attn = torch.from_numpy(attn_np.view(np.int16)).cuda().view(torch.bfloat16)
     resid = torch.from_numpy(resid_np.view(np.int16)).cuda().view(torch.bfloat16)
@@ -215,31 +226,38 @@ def run_ours(args, rank, world):
     gate = torch.empty((L, B, dims.k), dtype=torch.float32, device="cuda")
     cfg = md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, max(B, 1), L, enable_prefetch=args.prefetch)
     s = torch.cuda.current_stream()
-    h = md.moe_decode_create(cfg, weights, s)
+    hs = [md.moe_decode_create(cfg, w, s) for w in weight_sets]
+    h = hs[0]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # 256 MiB > 126 MB L2
     kps = md.moe_decode_kernels_per_step(h, B)
 
-    def step():
-        md.moe_decode_step(h, B, attn, resid, out, idx, gate, s)
+    def step(i=0):
+        md.moe_decode_step(hs[i % R], B, attn, resid, out, idx, gate, s)
 
-    for _ in range(max(args.warmup, 3)):
-        step()
+    for i in range(max(args.warmup, 3) * R):
+        step(i)
     if args.profile_run:
         # Profiling mode (for ncu): a few plain graph replays, no timing.
-        for _ in range(args.profile_run):
-            step()
-        rc = md.moe_decode_sync_status(h, s)
-        md.moe_decode_destroy(h)
+        for i in range(args.profile_run):
+            step(i)
+        rc = max(abs(md.moe_decode_sync_status(x, s)) for x in hs)
+        for x in hs:
+            md.moe_decode_destroy(x)
+        if rc:
+            raise RuntimeError(md.strerror(-rc))
+        return None
+    n_union = []
+    for r in range(R):
+        step(r)
+        rc = md.moe_decode_sync_status(hs[r], s)
         if rc:
             raise RuntimeError(md.strerror(rc))
-        return None
-    rc = md.moe_decode_sync_status(h, s)
-    if rc:
-        raise RuntimeError(md.strerror(rc))
-    idx_np = idx.cpu().numpy()
-    n_union = [len(np.unique(idx_np[l])) for l in range(L)]
+        idx_np = idx.cpu().numpy()
+        n_union += [len(np.unique(idx_np[l])) for l in range(L)]
 
-    # ---- timed region: K steps, L2 flushed before each (outside the event pair) --------------
+    # ---- timed region: K steps; no step reuses weights that can still be in L2 -----------------
+    # (one layer: the step cycles over R weight copies, R x bytes per step > 2 x L2; a stack of
+    # layers streams more than 2 x L2 per step by itself)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
@@ -247,24 +265,25 @@ def run_ours(args, rank, world):
     with Clocks(dev) as clk:
         time.sleep(0.3)
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
             ev[i][0].record(s)
-            step()
+            step(i)
             ev[i][1].record(s)
         torch.cuda.synchronize()
         time.sleep(0.2)
     if world > 1:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    rc = md.moe_decode_sync_status(h, s)
+    rc = max(abs(md.moe_decode_sync_status(x, s)) for x in hs)
     if rc:
-        raise RuntimeError(md.strerror(rc))
+        raise RuntimeError(md.strerror(-rc))
     tot = torch.tensor([sum(step_ms)], dtype=torch.float64, device="cuda")
     if world > 1:
         dist.all_reduce(tot, op=dist.ReduceOp.MAX)
     t_max_ms = float(tot.item())
 
-    # ---- warm back-to-back (secondary) -----------------------------------------------------------
+    # ---- secondary: the same weights back to back (warm L2), and a 256 MiB L2 flush before each
+    # step instead of the rotation (the flush leaves dirty lines whose write-back lands inside
+    # the next step, so it overstates a cold step)
     w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     w0.record(s)
     for _ in range(args.steps):
@@ -272,6 +291,16 @@ def run_ours(args, rank, world):
     w1.record(s)
     torch.cuda.synchronize()
     warm_us = w0.elapsed_time(w1) * 1000 / (args.steps * L)
+    fl = []
+    for i in range(min(args.steps, 20)):
+        flush.fill_(i & 0xFF)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(s)
+        step()
+        f1.record(s)
+        torch.cuda.synchronize()
+        fl.append(f0.elapsed_time(f1))
+    flushed_us = statistics.median(fl) * 1000 / L
 
     # ---- end to end through the host-buffer entry point (pinned host memory) -----------------
     a_h = torch.from_numpy(attn_np.view(np.int16)).pin_memory()
@@ -279,30 +308,30 @@ def run_ours(args, rank, world):
     o_h = torch.empty((B, dims.d), dtype=torch.int16).pin_memory()
     i_h = torch.empty((L, B, dims.k), dtype=torch.int32).pin_memory()
     g_h = torch.empty((L, B, dims.k), dtype=torch.float32).pin_memory()
-    for _ in range(2):
-        md.moe_decode_step_host(h, B, a_h, r_h, o_h, i_h, g_h, s)
+    for x in hs:
+        md.moe_decode_step_host(x, B, a_h, r_h, o_h, i_h, g_h, s)
     e_ms = []
     for i in range(args.steps):
-        flush.fill_(i & 0xFF)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s)
-        md.moe_decode_step_host(h, B, a_h, r_h, o_h, i_h, g_h, s)
+        md.moe_decode_step_host(hs[i % R], B, a_h, r_h, o_h, i_h, g_h, s)
         e1.record(s)
         e1.synchronize()
         e_ms.append(e0.elapsed_time(e1))
     h2d = attn_np.nbytes + resid_np.nbytes
     d2h = B * dims.d * 2 + 2 * L * B * dims.k * 4
 
-    # ---- per-kernel durations (eager, event-bracketed launches, L2 flushed) -------------------
+    # ---- per-kernel durations (eager, event-bracketed launches, weights rotated as above) ------
     per = {}
-    for i in range(max(5, min(args.steps, 20))):
-        flush.fill_(i & 0xFF)
+    for i in range(max(5, min(args.steps, 20)) * R):
         torch.cuda.synchronize()
-        for name, ms in md.moe_decode_profile_step(h, B, attn, resid, out, idx, gate, s):
+        for name, ms in md.moe_decode_profile_step(hs[i % R], B, attn, resid, out, idx, gate, s):
             per.setdefault(name, []).append(ms)
-    md.moe_decode_destroy(h)
-    return {"B": B, "L": L, "dims": dims, "step_ms": step_ms, "t_max_ms": t_max_ms, "warm_us": warm_us,
+    for x in hs:
+        md.moe_decode_destroy(x)
+    return {"B": B, "L": L, "R": R, "dims": dims, "step_ms": step_ms, "t_max_ms": t_max_ms, "warm_us": warm_us,
+            "flushed_us": flushed_us,
             "e2e_ms": e_ms, "h2d": h2d, "d2h": d2h, "per_kernel": per, "n_union": n_union,
             "clocks": clk.summary(), "kps": kps}
 
@@ -361,7 +390,9 @@ def main():
     dname, B, L, mode = WORKLOADS[args.workload]
     config = {"workload": args.workload, "batch": B, "layers": L, "shape": dname,
               "prefetch": bool(args.prefetch and L > 1),
-              "l2": "flushed before every timed step (256 MiB write outside the event pair)",
+              "l2": (f"inputs larger than L2: the step cycles over {rotation(L)} independently seeded weight "
+                     "copies, no flush" if rotation(L) > 1 else
+                     f"inputs larger than L2: {L} layers of distinct weights per step, no flush"),
               "parallelism": f"replicas x{args.gpus}"}
 
     if args.impl == "reference":
@@ -392,7 +423,7 @@ def main():
     dims = r["dims"]
     K = args.steps
     us_per_layer = r["t_max_ms"] * 1000 / (world * K * L)
-    wbytes = weight_bytes(dims, r["n_union"])
+    wbytes = weight_bytes(dims, r["n_union"]) / r["R"]  # n_union holds R copies x L layers
     per_step_ms = r["t_max_ms"] / K
     gbs = wbytes / (per_step_ms * 1e-3) / 1e9
     # dominant kernel by time share
@@ -419,6 +450,7 @@ def main():
                                            statistics.median(r["step_ms"]),
                                            sorted(r["step_ms"])[int(0.9 * (K - 1))])],
         "warm_us_per_layer_step": round(r["warm_us"], 3),
+        "l2_flushed_us_per_layer_step": round(r["flushed_us"], 3),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(ach / hbm, 4), "traffic": traffic_for(dom, B, args.workload),
                      "algorithmic_bytes": dom_bytes, "avg_launch_us": round(avg[dom] * 1000, 3),
