@@ -74,8 +74,10 @@ enum {
  *   max_batch  largest batch passed to step                          1 <= max_batch <= 64
  *   n_layers   layers run back to back by one step (residual chains)  1 <= n_layers <= 64
  *   rms_eps    RMSNorm epsilon (> 0; the layer uses 1e-6)
- *   enable_prefetch  1: a side stream prefetches layer l+1's router, RMSNorm scale and
- *                    the head of its W_o into L2 while layer l runs its experts
+ *   enable_prefetch  1: layer l's router kernel prefetches into L2 what layer l+1 reads
+ *                    first (its router matrix, RMSNorm scale and the leading 16 MB of
+ *                    its W_o, split by the CTA that reads them) while layer l's top-k
+ *                    and first expert bytes leave HBM idle; no extra kernel
  *   force_variant    0 or 1: expert gate/up kernel by batch size (small-M at B <= 2,
  *                    split-K above); 2: split-K at every batch size (testing)              */
 typedef struct {
@@ -154,8 +156,8 @@ MOE_API int moe_decode_kernels_per_step(moe_decode_handle* h, int batch);
  * `stream` with a CUDA event pair around every kernel, synchronises, and writes
  * each kernel's duration in milliseconds, in launch order, to kernel_ms (host,
  * max_kernels entries) and a short kernel name id to kernel_id (host, or NULL):
- * 1 o_proj+residual+RMS, 2 router+top-k, 3 small-M expert kernel (gate/up and down),
- * 4 gate/up split-K, 5 down+combine, 6 L2 prefetch.  Same buffers as
+ * 1 o_proj+residual+RMS, 2 router+top-k (and the next layer's L2 prefetch),
+ * 3 small-M expert kernel (gate/up and down), 4 gate/up split-K, 5 down+combine.  Same buffers as
  * moe_decode_step.  Returns the number of kernels timed (or a negative code). */
 MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_out,
                                     const void* residual_in, void* out, int32_t* topk_idx,

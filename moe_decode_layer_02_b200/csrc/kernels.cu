@@ -9,7 +9,6 @@
 //                        each expert (atomic ticket per expert, no spinning).
 //   K4 k_down_combine    out = bf16(h + sum_j gate_j * W_down[e_j] . a_j): rows of d split over
 //                        CTAs, experts streamed in ascending order, fixed reduction order.
-//   k_prefetch_l2        side-stream L2 prefetch of the next layer's weights.
 //
 // Sources: "vLLM speeds up Kimi K3 up to 1.9x on NVIDIA GB300 with agent-assisted
 // kernels", section "How the specialised decode path works" (kernels chosen by batch size,
@@ -493,29 +492,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_down_combine(const LayerArgs a)
 }
 
 // =============================================================================
-// Side-stream L2 prefetch of the next layer's weights (no shared memory, no outputs)
-// =============================================================================
-__global__ void k_prefetch_l2(const PrefetchArgs p) {
-  constexpr unsigned long long kChunk = 32768;
-  unsigned long long total = 0;
-  for (int i = 0; i < p.n; ++i) total += (p.bytes[i] + kChunk - 1) / kChunk;
-  for (unsigned long long q = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x; q < total;
-       q += (unsigned long long)gridDim.x * blockDim.x) {
-    unsigned long long rem = q;
-    for (int i = 0; i < p.n; ++i) {
-      const unsigned long long nch = (p.bytes[i] + kChunk - 1) / kChunk;
-      if (rem < nch) {
-        const unsigned long long off = rem * kChunk;
-        const unsigned long long len = min(kChunk, p.bytes[i] - off) & ~15ull;
-        if (len) bulk_prefetch_l2(static_cast<const unsigned char*>(p.ptr[i]) + off, (uint32_t)len);
-        break;
-      }
-      rem -= nch;
-    }
-  }
-}
-
-// =============================================================================
 // Host side: planning and launch
 // =============================================================================
 namespace {
@@ -628,11 +604,6 @@ cudaError_t launch_gateup_splitk(const LayerArgs& a, int grid, cudaStream_t s, b
 
 cudaError_t launch_down(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
   return launch_k(k_down_combine<0>, grid, a.k4.smem, s, pdl, a);
-}
-
-cudaError_t launch_prefetch(const PrefetchArgs& p, int grid, cudaStream_t s) {
-  k_prefetch_l2<<<grid, 128, 0, s>>>(p);
-  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -51,14 +51,11 @@ struct LayerArgs {
   int* user_idx;          // [B][k] or null
   float* user_gate;       // [B][k] or null
   int route_tables;       // the router's last CTA builds the global routing tables
+  // Next layer's weights for the router kernel's L2 prefetch (null: no prefetch)
+  const uint16_t *pf_w_o, *pf_w_r, *pf_gamma;
+  int pf_w_o_rows;        // leading rows of each CTA's share of the next W_o to prefetch
   Workspace ws;
   KTune k1, k2, k3, k4;
-};
-
-struct PrefetchArgs {
-  const void* ptr[4];
-  unsigned long long bytes[4];
-  int n;
 };
 
 // Host-side planning for a.B tokens (sets the KTune fields, returns false if unsupported).
@@ -68,7 +65,6 @@ bool plan_layer(LayerArgs& a, int num_sms, size_t smem_optin);
 cudaError_t launch_oproj(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_gateup_splitk(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
 cudaError_t launch_down(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
-cudaError_t launch_prefetch(const PrefetchArgs& p, int grid, cudaStream_t s);
 
 // Small-batch kernels and the router (kernels_small.cu): whole rows streamed by TMA.
 bool plan_small(LayerArgs& a, int grid, size_t smem_optin);

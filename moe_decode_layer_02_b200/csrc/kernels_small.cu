@@ -288,8 +288,26 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
     if (lane == 0 && nrows > 0) {
       mbar_arrive_expect_tx(&full[0], nrows * row_bytes);
       bulk_g2s(wsl, a.w_r + (size_t)e0 * d, nrows * row_bytes, &full[0], policy_evict_first());
-      mbar_drain(&full[0], 0, a.ws.err);
     }
+    if (lane == 0 && a.pf_w_o) {
+      // Next layer: warm L2 while this layer's router, top-k and first expert bytes leave HBM
+      // idle.  Each CTA prefetches what the same CTA of the next layer reads first: its router
+      // rows and the leading rows of its share of W_o.
+      if (nrows > 0) bulk_prefetch_l2(a.pf_w_r + (size_t)e0 * d, nrows * row_bytes);
+      if (c == 0) bulk_prefetch_l2(a.pf_gamma, (uint32_t)d * 2u);
+      long long o0, o1;
+      split_range(d, G, c, o0, o1);
+      const size_t orow = (size_t)a.d_o * 2;
+      size_t left = (size_t)min((long long)a.pf_w_o_rows, o1 - o0) * orow;
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(a.pf_w_o + (size_t)o0 * a.d_o);
+      for (size_t off = 0; left > 0;) {
+        const uint32_t n = (uint32_t)min(left, (size_t)65536);
+        bulk_prefetch_l2(src + off, n);
+        off += n;
+        left -= n;
+      }
+    }
+    if (lane == 0 && nrows > 0) mbar_drain(&full[0], 0, a.ws.err);
   } else {
     const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
     float gam[kCPLf][8];

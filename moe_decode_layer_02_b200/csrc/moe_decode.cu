@@ -5,9 +5,10 @@
 // CUDA graph: per layer K1 o_proj+residual+RMS stats -> K2 router+top-k+routing ->
 // K3 expert gate/up (small-M or split-K by batch) -> K4 down+combine, chained with
 // programmatic dependent launch so each kernel's CTAs start (and fetch their static
-// weights) while the previous kernel drains.  With prefetch on, a forked side stream
-// prefetches layer l+1's router, RMSNorm scale and the head of its W_o into L2 once
-// layer l's router is done; it joins the main stream at the end of the graph.
+// weights) while the previous kernel drains.  With prefetch on, layer l's router kernel
+// also prefetches into L2 what layer l+1 reads first (its router rows, RMSNorm scale and
+// the leading rows of its W_o), in the window where the router, top-k and the first
+// expert bytes leave HBM idle.
 //
 // Sources: "vLLM speeds up Kimi K3 up to 1.9x on NVIDIA GB300 with agent-assisted
 // kernels", section "How the specialised decode path works" (kernel choice by batch
@@ -41,7 +42,7 @@ struct GraphEntry {
   int kernels;
 };
 
-constexpr size_t kPrefetchWoHead = 24ull << 20;  // bytes of the next W_o prefetched into L2
+constexpr size_t kPrefetchWoBytes = 16ull << 20;  // bytes of the next W_o prefetched into L2
 constexpr int kGraphCacheMax = 16;
 
 }  // namespace
@@ -59,8 +60,7 @@ struct moe_decode_handle {
   void *h_attn = nullptr, *h_resid = nullptr, *h_out = nullptr, *h_idx = nullptr, *h_gate = nullptr;
   LayerArgs plan_splitk{};
   bool has_splitk = false;
-  cudaStream_t cap = nullptr, side = nullptr;
-  std::vector<cudaEvent_t> events;
+  cudaStream_t cap = nullptr;
   std::vector<GraphEntry> graphs;
   int last_batch = 0;
   bool poisoned = false;
@@ -104,12 +104,9 @@ void release(moe_decode_handle* h) {
   for (auto& g : h->graphs)
     if (g.exec) cudaGraphExecDestroy(g.exec);
   h->graphs.clear();
-  for (auto e : h->events) cudaEventDestroy(e);
-  h->events.clear();
   if (h->cap) cudaStreamDestroy(h->cap);
-  if (h->side) cudaStreamDestroy(h->side);
   if (h->ws_base) cudaFree(h->ws_base);
-  h->cap = h->side = nullptr;
+  h->cap = nullptr;
   h->ws_base = nullptr;
 }
 
@@ -148,21 +145,17 @@ LayerArgs layer_args(const moe_decode_handle* h, int l, int B, const void* attn,
   a.out = (l == c.n_layers - 1) ? static_cast<uint16_t*>(out) : h->resid_pp[l & 1];
   a.user_idx = idx ? idx + (size_t)l * B * c.top_k : nullptr;
   a.user_gate = gate ? gate + (size_t)l * B * c.top_k : nullptr;
+  a.pf_w_o = a.pf_w_r = a.pf_gamma = nullptr;
+  a.pf_w_o_rows = 0;
+  if (c.enable_prefetch && l + 1 < c.n_layers) {
+    const moe_decode_layer_weights& nw = h->w[l + 1];
+    a.pf_w_o = static_cast<const uint16_t*>(nw.w_o);
+    a.pf_w_r = static_cast<const uint16_t*>(nw.w_router);
+    a.pf_gamma = static_cast<const uint16_t*>(nw.gamma);
+    const size_t rows = kPrefetchWoBytes / ((size_t)c.d_o * 2) / (size_t)h->num_sms;
+    a.pf_w_o_rows = (int)std::max<size_t>(1, rows);
+  }
   return a;
-}
-
-PrefetchArgs prefetch_args(const moe_decode_handle* h, int l) {
-  const moe_decode_config& c = h->cfg;
-  PrefetchArgs p{};
-  const moe_decode_layer_weights& nw = h->w[l];
-  p.ptr[0] = nw.w_router;
-  p.bytes[0] = (unsigned long long)c.n_experts * c.d * 2;
-  p.ptr[1] = nw.gamma;
-  p.bytes[1] = (unsigned long long)c.d * 2;
-  p.ptr[2] = nw.w_o;
-  p.bytes[2] = std::min<unsigned long long>(kPrefetchWoHead, (unsigned long long)c.d * c.d_o * 2);
-  p.n = 3;
-  return p;
 }
 
 // Records the whole step on h->cap (which is in capture mode).  Returns kernels launched.
@@ -170,26 +163,14 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
                 int32_t* idx, float* gate, cudaError_t* err) {
   const moe_decode_config& c = h->cfg;
   const int G = h->num_sms;
-  const bool prefetch = c.enable_prefetch && c.n_layers > 1;
-  int kernels = 0, ev = 0;
+  int kernels = 0;
   cudaError_t e = cudaSuccess;
-  bool forked = false;
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     LayerArgs a = layer_args(h, l, B, attn, resid, out, idx, gate);
     const Variant v = variant_of(h, a);
     e = v.oproj_small ? launch_oproj_s(a, G, h->cap, l > 0, h->smem_optin) : launch_oproj(a, G, h->cap, l > 0);
     if (e == cudaSuccess) e = launch_router_s(a, G, h->cap, true, h->smem_optin);
     kernels += 2;
-    if (e == cudaSuccess && prefetch && l + 1 < c.n_layers) {
-      // Fork: once this layer's router is done, warm L2 with the next layer's
-      // router slice, RMSNorm scale and the head of its W_o.
-      e = cudaEventRecord(h->events[ev], h->cap);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->events[ev++], 0);
-      PrefetchArgs p = prefetch_args(h, l + 1);
-      if (e == cudaSuccess) e = launch_prefetch(p, G, h->side);
-      ++kernels;
-      forked = true;
-    }
     if (v.experts_small) {
       if (e == cudaSuccess) e = launch_experts_s(a, G, h->cap, true, h->smem_optin);
       kernels += 1;
@@ -198,10 +179,6 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
       if (e == cudaSuccess) e = launch_down(a, G, h->cap, true);
       kernels += 2;
     }
-  }
-  if (e == cudaSuccess && forked) {
-    e = cudaEventRecord(h->events[ev], h->side);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(h->cap, h->events[ev++], 0);
   }
   *err = e;
   return kernels;
@@ -355,12 +332,6 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   if (e == cudaSuccess) e = set_kernel_attributes(h->smem_optin);
   if (e == cudaSuccess) e = set_small_attributes(h->smem_optin);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
-  for (int i = 0; i < 2 * cfg->n_layers + 2 && e == cudaSuccess; ++i) {
-    cudaEvent_t ev;
-    e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
-    if (e == cudaSuccess) h->events.push_back(ev);
-  }
   if (e != cudaSuccess) {
     cudaGetLastError();
     release(h);
@@ -493,7 +464,7 @@ int moe_decode_kernels_per_step(moe_decode_handle* h, int batch) {
   a.B = batch;
   plan_layer(a, h->num_sms, h->smem_optin);
   const int per_layer = variant_of(h, a).experts_small ? 3 : 4;
-  return per_layer * L + ((h->cfg.enable_prefetch && L > 1) ? L - 1 : 0);
+  return per_layer * L;
 }
 
 int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_out, const void* residual_in,
@@ -528,10 +499,6 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
       return v.oproj_small ? launch_oproj_s(a, G, st, false, h->smem_optin) : launch_oproj(a, G, st, false);
     });
     timed(2, s, [&](cudaStream_t st) { return launch_router_s(a, G, st, false, h->smem_optin); });
-    if (c.enable_prefetch && c.n_layers > 1 && l + 1 < c.n_layers) {
-      PrefetchArgs p = prefetch_args(h, l + 1);
-      timed(6, s, [&](cudaStream_t st) { return launch_prefetch(p, G, st); });
-    }
     if (v.experts_small) {
       timed(3, s, [&](cudaStream_t st) { return launch_experts_s(a, G, st, false, h->smem_optin); });
     } else {
