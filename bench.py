@@ -151,8 +151,8 @@ def algorithmic_bytes(dims, B, n_union):
     return {
         "oproj_residual_rmsnorm": d * do * 2 + B * do * 2 + B * d * 2 + B * d * 4,
         "router_topk": E * d * 2 + d * 2 + B * d * 4 + B * d * 4 + B * E * 4,
-        "gateup": n_union * 2 * I * d * 2 + B * k * d * 4 + B * k * I * 4,
-        "down_combine": n_union * d * I * 2 + B * k * I * 4 + B * d * 4 + B * d * 2,
+        "gateup_rows": n_union * 2 * I * d * 2 + B * k * d * 4 + B * k * I * 4,
+        "down_rows": n_union * d * I * 2 + B * k * I * 4 + B * d * 4 + B * d * 2,
         # small-M expert kernel: gate/up and down weights of the union, x and h in, out
         "experts_small_m": n_union * 3 * I * d * 2 + B * E * 4 + 2 * B * d * 4 + B * d * 2,
     }
@@ -431,7 +431,7 @@ def main():
     tot = sum(avg.values())
     dom = max(avg, key=avg.get)
     ab = algorithmic_bytes(dims, B, statistics.mean(r["n_union"]))
-    key = "gateup" if dom.startswith("gateup") else dom
+    key = dom
     dom_bytes = ab.get(key, 0)
     ach = dom_bytes / (avg[dom] * 1e-3) / 1e9
     e2e_us = statistics.mean(r["e2e_ms"]) * 1000 / L

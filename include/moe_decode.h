@@ -78,8 +78,9 @@ enum {
  *                    first (its router matrix, RMSNorm scale and the leading 16 MB of
  *                    its W_o, split by the CTA that reads them) while layer l's top-k
  *                    and first expert bytes leave HBM idle; no extra kernel
- *   force_variant    0 or 1: expert gate/up kernel by batch size (small-M at B <= 2,
- *                    split-K above); 2: split-K at every batch size (testing)              */
+ *   force_variant    0 or 1: expert kernels by batch size (the fused small-M kernel at
+ *                    B <= 2, separate large-batch gate/up and down kernels above);
+ *                    2: the large-batch kernels at every batch size (testing)             */
 typedef struct {
   int d, d_o, n_experts, top_k, inter, max_batch, n_layers;
   float rms_eps;
@@ -157,7 +158,8 @@ MOE_API int moe_decode_kernels_per_step(moe_decode_handle* h, int batch);
  * each kernel's duration in milliseconds, in launch order, to kernel_ms (host,
  * max_kernels entries) and a short kernel name id to kernel_id (host, or NULL):
  * 1 o_proj+residual+RMS, 2 router+top-k (and the next layer's L2 prefetch),
- * 3 small-M expert kernel (gate/up and down), 4 gate/up split-K, 5 down+combine.  Same buffers as
+ * 3 small-M expert kernel (gate/up and down), 4 large-batch gate/up, 5 large-batch
+ * down+combine.  Same buffers as
  * moe_decode_step.  Returns the number of kernels timed (or a negative code). */
 MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_out,
                                     const void* residual_in, void* out, int32_t* topk_idx,

@@ -29,8 +29,8 @@ EXPORTED = ("moe_decode_create", "moe_decode_step", "moe_decode_step_host", "moe
             "moe_decode_get_intermediate", "moe_decode_kernels_per_step", "moe_decode_profile_step",
             "moe_decode_step_static", "moe_decode_destroy", "moe_decode_strerror")
 
-KERNEL_NAMES = {1: "oproj_residual_rmsnorm", 2: "router_topk", 3: "experts_small_m", 4: "gateup_split_k",
-                5: "down_combine"}
+KERNEL_NAMES = {1: "oproj_residual_rmsnorm", 2: "router_topk", 3: "experts_small_m", 4: "gateup_rows",
+                5: "down_rows"}
 
 
 class moe_decode_config(ctypes.Structure):

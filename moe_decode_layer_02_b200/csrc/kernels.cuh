@@ -23,8 +23,6 @@ struct Workspace {
   int* entry_tok;    // [maxB*k]    token of each entry (ascending within an expert)
   int* entry_slot;   // [maxB*k]    slot j of that token's top-k list
   float* a;          // [maxB*k][I] SwiGLU activations per entry
-  float* gu_part;    // split-K partials [maxB*k][n_split][2I]
-  unsigned* gu_tick; // [E]         split-K per-union-expert tickets
   unsigned* counters;  // [kNumCounters]
   unsigned* err;       // error word (kErrTimeout | kErrBounds)
 };
@@ -33,11 +31,9 @@ struct KTune {
   int stages = 0;          // ring stages
   int rows_per_stage = 0;  // weight rows (or row pairs) per stage (CUDA-core kernels)
   int rows_max = 0;        // max rows owned by one CTA
-  int n_split = 0;         // split-K factor (gate/up large-batch variant)
   int kc = 0;              // K chunk of one MMA stage (multiple of 64)
   int nch = 0;             // K chunks per row (K = kc * nch)
-  int tok_group = 0;       // tokens per pass over the weights
-  int a_in_smem = 0;       // down kernel: all SwiGLU activations staged in shared memory
+  int tok_group = 0;       // tokens per pass over the weights (down kernel: entries staged per stage)
   size_t smem = 0;         // dynamic shared memory bytes
 };
 
@@ -63,8 +59,6 @@ bool plan_layer(LayerArgs& a, int num_sms, size_t smem_optin);
 
 // Launchers (pdl: launch with programmatic stream serialisation).
 cudaError_t launch_oproj(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
-cudaError_t launch_gateup_splitk(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
-cudaError_t launch_down(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
 
 // Small-batch kernels and the router (kernels_small.cu): whole rows streamed by TMA.
 bool plan_small(LayerArgs& a, int grid, size_t smem_optin);
@@ -76,5 +70,11 @@ cudaError_t launch_oproj_s(const LayerArgs& a, int grid, cudaStream_t s, bool pd
 cudaError_t launch_router_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t launch_experts_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t set_kernel_attributes(size_t smem_optin);
+
+// Expert kernels above batch 2 (kernels_large.cu): whole rows, tokens grouped per expert.
+bool plan_large(LayerArgs& a, int grid, size_t smem_optin);
+cudaError_t set_large_attributes(size_t smem_optin);
+cudaError_t launch_gateup_rows(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
+cudaError_t launch_down_rows(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 
 }  // namespace moe

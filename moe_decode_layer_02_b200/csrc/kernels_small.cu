@@ -33,119 +33,17 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "rowdot.cuh"
 #include "topk.cuh"
 
 namespace moe {
 
 namespace {
 
-// 15 consumer warps + the producer = 16 warps, four per SM sub-partition, which leaves 128
-// registers per thread (a 17th warp would cut that to 96).  The dot products are latency-
-// bound chains of shared-memory loads and FMAs, so warps in flight are what keep the
-// consumers ahead of HBM.
-constexpr int kCW = 15;              // consumer warps
-constexpr int kCT = kCW * 32;        // consumer threads
-constexpr int kThreadsS = kCT + 32;  // + one producer warp
 static_assert(kThreadsS == kRouteThreads, "the expert kernel routes with all of its threads");
-constexpr int kCPLf = 3;             // 8-element chunks per lane: K <= 15 warps * 32 lanes * 3 * 8 = 11520
-
-__device__ __forceinline__ void csync() { asm volatile("bar.sync 1, %0;" ::"n"(kCT) : "memory"); }
-
-__device__ __forceinline__ size_t al128(size_t x) { return (x + 127) & ~size_t(127); }
-
-__device__ __forceinline__ void unpack8f(uint4 w, float* f) {
-  f[0] = bf16lo(w.x); f[1] = bf16hi(w.x); f[2] = bf16lo(w.y); f[3] = bf16hi(w.y);
-  f[4] = bf16lo(w.z); f[5] = bf16hi(w.z); f[6] = bf16lo(w.w); f[7] = bf16hi(w.w);
-}
 
 // Phase B experts per stage for EPL elements per lane (registers bound it).
 __host__ __device__ constexpr int experts_per_stage(int epl) { return epl == 4 ? 4 : (epl == 8 ? 2 : 1); }
-
-// Chunk of lane `lane` in warp w's K slice: q = w * qpw + j * 32 + lane, valid if j*32+lane < qpw.
-__device__ __forceinline__ bool cvalid(int qpw, int j, int lane) { return j * 32 + lane < qpw; }
-
-// Per-lane partial dots of R bf16 rows (shared memory) with NT register slices of the
-// activations: out[r * NT + t].  Rows r >= nr contribute zeros.  All chunk loads of all
-// rows are issued before the first FMA, and the R * NT * kA accumulators are independent
-// FMA chains (kA per row and token), so a warp's pass over a stage is one short chain
-// instead of R dependent ones.
-template <int NT, int R>
-__device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr, const float (&x)[NT][kCPLf][8],
-                                         int qbase, int qpw, int lane, float (&out)[R * NT]) {
-  constexpr int kA = (R * NT >= 8) ? 1 : 8 / (R * NT);
-  uint4 w[R][kCPLf];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int j = 0; j < kCPLf; ++j)
-      w[r][j] = (r < nr && cvalid(qpw, j, lane))
-                    ? *reinterpret_cast<const uint4*>(rp[r] + (size_t)(qbase + j * 32 + lane) * 8)
-                    : make_uint4(0, 0, 0, 0);
-  float acc[R][NT][kA];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int t = 0; t < NT; ++t)
-#pragma unroll
-      for (int e = 0; e < kA; ++e) acc[r][t][e] = 0.f;
-#pragma unroll
-  for (int j = 0; j < kCPLf; ++j)
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      float wf[8];
-      unpack8f(w[r][j], wf);
-#pragma unroll
-      for (int t = 0; t < NT; ++t)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][t][e % kA] = fmaf(wf[e], x[t][j][e], acc[r][t][e % kA]);
-    }
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int t = 0; t < NT; ++t) {
-      float v = 0.f;
-#pragma unroll
-      for (int e = 0; e < kA; ++e) v += acc[r][t][e];
-      out[r * NT + t] = v;
-    }
-}
-
-// Warp sums of V per-lane values (V a power of two <= 32) with V - 1 + 5 - log2(V) shuffles
-// instead of 5 V: each halving step sends one value of every pair across the current lane
-// bit and keeps the other.  Every lane returns the total of value multi_index<V>(lane).
-template <int V>
-__device__ __forceinline__ float warp_reduce_multi(float (&v)[V], int lane) {
-  static_assert(V >= 1 && V <= 32 && (V & (V - 1)) == 0, "V must be a power of two <= 32");
-#pragma unroll
-  for (int o = 16, c = V; c > 1; o >>= 1, c >>= 1) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int j = 0; j < c / 2; ++j) {
-      const float send = up ? v[2 * j] : v[2 * j + 1];
-      const float keep = up ? v[2 * j + 1] : v[2 * j];
-      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  float s = v[0];
-#pragma unroll
-  for (int o = 16 / V; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  return s;
-}
-
-// Value index held by `lane` after warp_reduce_multi<V>: bit k of the index is lane bit 4 - k.
-template <int V>
-__device__ __forceinline__ int multi_index(int lane) {
-  int idx = 0;
-#pragma unroll
-  for (int k = 0, c = V; c > 1; ++k, c >>= 1) idx |= ((lane >> (4 - k)) & 1) << k;
-  return idx;
-}
-
-// One lane per group of 32 / V holds each total.
-template <int V>
-__device__ __forceinline__ bool multi_writer(int lane) {
-  return (lane & (32 / V - 1)) == 0;
-}
 
 }  // namespace
 

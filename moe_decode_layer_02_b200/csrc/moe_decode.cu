@@ -2,8 +2,9 @@
 // capture of the per-layer kernel chain, and the host-buffer variant of the step.
 //
 // A step of n_layers layers is captured once per (batch, buffer addresses) into one
-// CUDA graph: per layer K1 o_proj+residual+RMS stats -> K2 router+top-k+routing ->
-// K3 expert gate/up (small-M or split-K by batch) -> K4 down+combine, chained with
+// CUDA graph: per layer K1 o_proj+residual+RMS stats -> K2 router (+ routing tables above
+// batch 2) -> the expert kernel(s): one fused gate/up + down kernel with per-CTA routing at
+// batch <= 2, separate gate/up and down kernels above, chained with
 // programmatic dependent launch so each kernel's CTAs start (and fetch their static
 // weights) while the previous kernel drains.  With prefetch on, layer l's router kernel
 // also prefetches into L2 what layer l+1 reads first (its router rows, RMSNorm scale and
@@ -52,14 +53,12 @@ struct moe_decode_handle {
   std::vector<moe_decode_layer_weights> w;
   int device = 0, num_sms = 0;
   size_t smem_optin = 0;
-  int n_split = 0;  // split-K factor, 0 if the shape has none
   Workspace ws{};
   void* ws_base = nullptr;
   uint16_t* resid_pp[2] = {nullptr, nullptr};
   // staging for moe_decode_step_host
   void *h_attn = nullptr, *h_resid = nullptr, *h_out = nullptr, *h_idx = nullptr, *h_gate = nullptr;
-  LayerArgs plan_splitk{};
-  bool has_splitk = false;
+  LayerArgs plan_base{};
   cudaStream_t cap = nullptr;
   std::vector<GraphEntry> graphs;
   int last_batch = 0;
@@ -92,12 +91,6 @@ int check_cfg(const moe_decode_config* c) {
   return MOE_OK;
 }
 
-int pick_split(int d) {
-  for (int ns = 1; ns <= d / 64; ++ns)
-    if (d % ns == 0 && (d / ns) % 64 == 0 && d / ns <= 1024) return ns;
-  return 0;
-}
-
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 void release(moe_decode_handle* h) {
@@ -110,8 +103,8 @@ void release(moe_decode_handle* h) {
   h->ws_base = nullptr;
 }
 
-bool use_splitk(const moe_decode_handle* h, int B) {
-  if (B >= 3) return true;                        // split-K above batch two
+bool use_large(const moe_decode_handle* h, int B) {
+  if (B >= 3) return true;                        // separate large-batch kernels above batch two
   return h->cfg.force_variant == 2;               // small-matrix kernels at batch one or two
 }
 
@@ -123,7 +116,7 @@ struct Variant {
 
 Variant variant_of(const moe_decode_handle* h, const LayerArgs& a) {
   Variant v;
-  v.experts_small = !use_splitk(h, a.B) && small_path_ok(a, h->smem_optin);
+  v.experts_small = !use_large(h, a.B) && small_path_ok(a, h->smem_optin);
   v.oproj_small = v.experts_small && oproj_small_ok(a, h->smem_optin);
   return v;
 }
@@ -131,7 +124,7 @@ Variant variant_of(const moe_decode_handle* h, const LayerArgs& a) {
 LayerArgs layer_args(const moe_decode_handle* h, int l, int B, const void* attn, const void* resid,
                      void* out, int32_t* idx, float* gate) {
   const moe_decode_config& c = h->cfg;
-  LayerArgs a = h->plan_splitk;
+  LayerArgs a = h->plan_base;
   a.B = B;
   plan_layer(a, h->num_sms, h->smem_optin);  // validated for every batch size at create
   a.route_tables = variant_of(h, a).experts_small ? 0 : 1;
@@ -175,8 +168,8 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
       if (e == cudaSuccess) e = launch_experts_s(a, G, h->cap, true, h->smem_optin);
       kernels += 1;
     } else {
-      if (e == cudaSuccess) e = launch_gateup_splitk(a, G, h->cap, true);
-      if (e == cudaSuccess) e = launch_down(a, G, h->cap, true);
+      if (e == cudaSuccess) e = launch_gateup_rows(a, G, h->cap, true, h->smem_optin);
+      if (e == cudaSuccess) e = launch_down_rows(a, G, h->cap, true, h->smem_optin);
       kernels += 2;
     }
   }
@@ -254,7 +247,6 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
     delete h;
     return MOE_ERR_UNSUPPORTED_CONFIG;
   }
-  h->n_split = pick_split(d);
 
   // ---- plans: every batch size 1..max_batch must fit ------------------------------------
   LayerArgs base{};
@@ -265,15 +257,13 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   base.k = K;
   base.I = I;
   base.eps = cfg->rms_eps;
-  h->plan_splitk = base;
-  h->plan_splitk.k3.n_split = h->n_split;
-  h->has_splitk = h->n_split > 0;
-  bool ok = h->has_splitk;
-  for (int B = 1; B <= maxB && ok; ++B) {
-    LayerArgs t = h->plan_splitk;
+  h->plan_base = base;
+  bool ok = true;
+  for (int B = 1; B <= maxB && ok; ++B) {  // the large-batch kernels must fit at every batch
+    LayerArgs t = h->plan_base;
     t.B = B;
     t.route_tables = 1;
-    ok = plan_layer(t, G, h->smem_optin) && router_ok(t, h->smem_optin);
+    ok = plan_layer(t, G, h->smem_optin) && router_ok(t, h->smem_optin) && plan_large(t, G, h->smem_optin);
   }
   if (!ok) {
     delete h;
@@ -281,7 +271,6 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   }
 
   // ---- workspace -----------------------------------------------------------------------
-  const int NS = std::max(h->n_split, 1);
   const size_t entries = (size_t)maxB * K;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -295,8 +284,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
                o_tg = take(sizeof(float) * entries), o_nu = take(sizeof(int)), o_ue = take(sizeof(int) * E),
                o_uo = take(sizeof(int) * (E + 1)), o_et = take(sizeof(int) * entries),
                o_es = take(sizeof(int) * entries), o_a = take(sizeof(float) * entries * I),
-               o_gp = take(h->has_splitk ? sizeof(float) * entries * NS * 2 * I : 16),
-               o_gt = take(sizeof(unsigned) * E), o_cnt = take(sizeof(unsigned) * kNumCounters),
+               o_cnt = take(sizeof(unsigned) * kNumCounters),
                o_err = take(sizeof(unsigned)), o_r0 = take(2ull * maxB * d), o_r1 = take(2ull * maxB * d);
   if (cudaMalloc(&h->ws_base, off) != cudaSuccess) {
     cudaGetLastError();
@@ -318,19 +306,18 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   ws.entry_tok = (int*)(b + o_et);
   ws.entry_slot = (int*)(b + o_es);
   ws.a = (float*)(b + o_a);
-  ws.gu_part = (float*)(b + o_gp);
-  ws.gu_tick = (unsigned*)(b + o_gt);
   ws.counters = (unsigned*)(b + o_cnt);
   ws.err = (unsigned*)(b + o_err);
   h->resid_pp[0] = (uint16_t*)(b + o_r0);
   h->resid_pp[1] = (uint16_t*)(b + o_r1);
-  h->plan_splitk.ws = ws;
+  h->plan_base.ws = ws;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(h->ws_base, 0, off, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e == cudaSuccess) e = set_kernel_attributes(h->smem_optin);
   if (e == cudaSuccess) e = set_small_attributes(h->smem_optin);
+  if (e == cudaSuccess) e = set_large_attributes(h->smem_optin);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -460,7 +447,7 @@ int moe_decode_get_intermediate(moe_decode_handle* h, int which, void* dst, size
 int moe_decode_kernels_per_step(moe_decode_handle* h, int batch) {
   if (!h || !is_live(h) || batch < 1 || batch > h->cfg.max_batch) return MOE_ERR_INVALID_ARG;
   const int L = h->cfg.n_layers;
-  LayerArgs a = h->plan_splitk;
+  LayerArgs a = h->plan_base;
   a.B = batch;
   plan_layer(a, h->num_sms, h->smem_optin);
   const int per_layer = variant_of(h, a).experts_small ? 3 : 4;
@@ -502,8 +489,8 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
     if (v.experts_small) {
       timed(3, s, [&](cudaStream_t st) { return launch_experts_s(a, G, st, false, h->smem_optin); });
     } else {
-      timed(4, s, [&](cudaStream_t st) { return launch_gateup_splitk(a, G, st, false); });
-      timed(5, s, [&](cudaStream_t st) { return launch_down(a, G, st, false); });
+      timed(4, s, [&](cudaStream_t st) { return launch_gateup_rows(a, G, st, false, h->smem_optin); });
+      timed(5, s, [&](cudaStream_t st) { return launch_down_rows(a, G, st, false, h->smem_optin); });
     }
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);

@@ -127,8 +127,6 @@ size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, Work
     ws->entry_tok = reinterpret_cast<int*>(et);
     ws->entry_slot = reinterpret_cast<int*>(es);
     ws->a = reinterpret_cast<float*>(act);
-    ws->gu_part = nullptr;  // split-K only; never launched from here
-    ws->gu_tick = nullptr;
   }
   return off;
 }
