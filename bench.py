@@ -51,6 +51,7 @@ WORKLOADS = {
     "tp16e64_b1": ("TP16E64", 1, 1, "indep"),
     "tp16e64_b2": ("TP16E64", 2, 1, "indep"),
     "tp8e64_b64": ("TP8E64", 64, 1, "indep"),
+    "tp8e224k4_b16": ("TP8E224K4", 16, 1, "indep"),
 }
 
 KERNEL_DIR = os.path.join(ROOT, "moe_decode_layer_02_b200", "csrc")
@@ -66,13 +67,15 @@ def peaks():
 
 def dims_of(name):
     import synth
-    small = {"TP16E64": synth.Dims(7168, 8192, 64, 16, 128), "TP8E64": synth.Dims(7168, 8192, 64, 16, 256)}
+    small = {"TP16E64": synth.Dims(7168, 8192, 64, 16, 128), "TP8E64": synth.Dims(7168, 8192, 64, 16, 256),
+             # batch 16 with the TP8 shard's tokens-per-expert (16 * 4 / 224 = 16 * 16 / 896) in 2.5 GB
+             "TP8E224K4": synth.Dims(7168, 8192, 224, 4, 256)}
     return small[name] if name in small else getattr(synth, name)
 
 
 def seed_of(dname, L):
     import synth
-    return synth.config_seed({"TP16": 1, "TP8": 3, "TP16E64": 21, "TP8E64": 23}[dname] + (10 if L > 1 else 0))
+    return synth.config_seed({"TP16": 1, "TP8": 3, "TP16E64": 21, "TP8E64": 23, "TP8E224K4": 25}[dname] + (10 if L > 1 else 0))
 
 
 def rotation(L):

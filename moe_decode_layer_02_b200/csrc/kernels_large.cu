@@ -174,6 +174,26 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
       }
       if (g0 == 0) mbar_wait(&full[s], (it / SA) & 1, abort_flag, a.ws.err);
       const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SA_B);
+      if (m - g0 == 1) {  // a single token: half the FMAs, four rows per pass
+        const float(&x1)[1][kCPLf][8] = reinterpret_cast<const float(&)[1][kCPLf][8]>(xr[0]);
+        for (int i0 = 0; i0 < nrow; i0 += 4) {
+          const uint16_t* rp[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int i = min(i0 + k, nrow - 1), pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
+            rp[k] = st + (size_t)(gu * PS + pi) * d;
+          }
+          float v[4];
+          rows_dot<1, 4>(rp, nrow - i0, x1, qbase, qpw, lane, v);
+          const float tot = warp_reduce_multi<4>(v, lane);
+          const int i = i0 + multi_index<4>(lane);
+          if (multi_writer<4>(lane) && i < nrow) {
+            const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
+            pb[((size_t)(gu * PS + pi) * B + g0) * kCW + warp] = tot;
+          }
+        }
+        continue;
+      }
       for (int i0 = 0; i0 < nrow; i0 += kRI) {
         const uint16_t* rp[kRI];
 #pragma unroll
@@ -195,15 +215,14 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     csync();  // every warp's partials of this stage are in pb (the other buffer is the next stage's)
-    for (int z = tid; z < np * m; z += kCT) {
-      const int pi = z / m, t = z - pi * m;
-      float gs = 0.f, us = 0.f;
+    // one warp per (pair, token): lanes 0..14 hold the gate partials, 16..30 the up partials
+    for (int z = warp; z < np * m; z += kCW) {
+      const int pi = z / m, t = z - pi * m, w = lane & 15;
+      float v = (w < kCW) ? pb[((size_t)((lane >> 4) * PS + pi) * B + t) * kCW + w] : 0.f;
 #pragma unroll
-      for (int w = 0; w < kCW; ++w) {
-        gs += pb[((size_t)pi * B + t) * kCW + w];
-        us += pb[((size_t)(PS + pi) * B + t) * kCW + w];
-      }
-      a.ws.a[(size_t)(off + t) * I + p + pi] = gs / (1.0f + expf(-gs)) * us;
+      for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      const float gs = __shfl_sync(0xffffffffu, v, 0), us = __shfl_sync(0xffffffffu, v, 16);
+      if (lane == 0) a.ws.a[(size_t)(off + t) * I + p + pi] = gs / (1.0f + expf(-gs)) * us;
     }
     q += np;
     p += np;
