@@ -29,6 +29,8 @@ namespace moe {
 
 namespace {
 
+constexpr int kGateUpChunk = 4;  // pairs per gate/up chunk: stages of four whole rows
+
 // Down-kernel experts per stage for EPL elements per lane (registers bound it).
 __host__ __device__ constexpr int down_experts_per_stage(int epl) { return epl == 4 ? 4 : (epl == 8 ? 2 : 1); }
 
@@ -72,6 +74,10 @@ __device__ __forceinline__ void load_tables(const LayerArgs& a, int U, int n_ent
 
 // =============================================================================
 // gate/up + SiLU*mul (batch >= 3)
+//   The CTA's pairs are taken in chunks of up to PC consecutive pairs of one expert; a chunk
+//   is two stages, its PC gate rows and then its PC up rows, each one contiguous bulk copy
+//   (fewer, larger copies stream faster).  The partial sums of a chunk are reduced once its
+//   up stage is done.
 // =============================================================================
 template <int NT>
 __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a) {
@@ -79,14 +85,14 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
   constexpr int kRI = 4 / NT;  // rows per interleaved pass
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, I = a.I, E = a.E, B = a.B;
-  const int SA = a.k3.stages, PS = a.k3.rows_per_stage;
+  const int SA = a.k3.stages, PC = a.k3.rows_per_stage;
   const int n_ent = B * a.k;
   const uint32_t row_bytes = (uint32_t)d * 2u;
-  const size_t SA_B = al128((size_t)2 * PS * row_bytes);
-  const size_t part_f = (size_t)2 * PS * B * kCW;  // floats of one partial buffer
+  const size_t SA_B = al128((size_t)PC * row_bytes);
+  const size_t part_f = (size_t)2 * PC * B * kCW;  // floats of one partial buffer
 
   unsigned char* ring = smem;
-  float* part = reinterpret_cast<float*>(ring + (size_t)SA * SA_B);  // [2][2 PS][B][kCW]
+  float* part = reinterpret_cast<float*>(ring + (size_t)SA * SA_B);  // [2][2 PC][B][kCW]
   SmemTables tb;
   tb.uoff = reinterpret_cast<int*>(part + 2 * part_f);             // [E + 1]
   tb.etok = tb.uoff + (E + 1);                                      // [n_ent]
@@ -117,14 +123,19 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
       const uint64_t pol = policy_evict_first();
       int it = 0, u = q0 / I, p = q0 - (q0 / I) * I;
       int e = (q0 < q1) ? clamp_expert(ld_act_i(&a.ws.union_e[u]), E, a.ws.err) : 0;
-      for (int q = q0; q < q1; ++it) {
-        const int np = min(min(PS, I - p), q1 - q);
-        if (!ring_acquire(empty, it, SA, abort_flag, a.ws.err)) break;
-        const int s = it % SA;
-        const uint16_t* base = a.w_gu + ((size_t)e * 2 * I + p) * d;
-        mbar_arrive_expect_tx(&full[s], 2u * np * row_bytes);
-        bulk_g2s(ring + s * SA_B, base, np * row_bytes, &full[s], pol);
-        bulk_g2s(ring + s * SA_B + (size_t)PS * row_bytes, base + (size_t)I * d, np * row_bytes, &full[s], pol);
+      bool ok = true;
+      for (int q = q0; q < q1 && ok;) {
+        const int np = min(min(PC, I - p), q1 - q);
+        for (int gu = 0; gu < 2; ++gu, ++it) {  // the chunk's gate rows, then its up rows
+          if (!ring_acquire(empty, it, SA, abort_flag, a.ws.err)) {
+            ok = false;
+            break;
+          }
+          const int s = it % SA;
+          mbar_arrive_expect_tx(&full[s], np * row_bytes);
+          bulk_g2s(ring + s * SA_B, a.w_gu + ((size_t)e * 2 * I + (size_t)gu * I + p) * d, np * row_bytes,
+                   &full[s], pol);
+        }
         q += np;
         p += np;
         if (p == I) {
@@ -144,81 +155,76 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
   const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
   float xr[NT][kCPLf][8];
   int cached_u = -1, cached_g = -1;
-  int it = 0, u = q0 / I, p = q0 - (q0 / I) * I;
-  for (int q = q0; q < q1; ++it) {
-    const int np = min(min(PS, I - p), q1 - q), s = it % SA;
+  int it = 0, ch = 0, u = q0 / I, p = q0 - (q0 / I) * I;
+  for (int q = q0; q < q1; ++ch) {
+    const int np = min(min(PC, I - p), q1 - q);
     const int off = tb.uoff[u];
     const int m = min(tb.uoff[u + 1] - off, B);
-    float* pb = part + (size_t)(it & 1) * part_f;
-    const int nrow = 2 * np;  // gate rows 0..np-1, then up rows
-    for (int g0 = 0; g0 < m; g0 += NT) {
-      if (u != cached_u || g0 != cached_g) {  // x of this group's tokens, in registers
+    float* pb = part + (size_t)(ch & 1) * part_f;
+    for (int gu = 0; gu < 2; ++gu, ++it) {
+      const int s = it % SA;
+      bool waited = false;
+      for (int g0 = 0; g0 < m; g0 += NT) {
+        if (u != cached_u || g0 != cached_g) {  // x of this group's tokens, in registers
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const int tok = (g0 + t < m) ? tb.etok[off + g0 + t] : -1;
+          for (int t = 0; t < NT; ++t) {
+            const int tok = (g0 + t < m) ? tb.etok[off + g0 + t] : -1;
 #pragma unroll
-          for (int j = 0; j < kCPLf; ++j) {
-            if (tok >= 0 && cvalid(qpw, j, lane)) {
-              const float* xp = a.ws.x + (size_t)tok * d + (size_t)(qbase + j * 32 + lane) * 8;
-              const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
-              xr[t][j][0] = x0.x; xr[t][j][1] = x0.y; xr[t][j][2] = x0.z; xr[t][j][3] = x0.w;
-              xr[t][j][4] = x1.x; xr[t][j][5] = x1.y; xr[t][j][6] = x1.z; xr[t][j][7] = x1.w;
-            } else {
+            for (int j = 0; j < kCPLf; ++j) {
+              if (tok >= 0 && cvalid(qpw, j, lane)) {
+                const float* xp = a.ws.x + (size_t)tok * d + (size_t)(qbase + j * 32 + lane) * 8;
+                const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
+                xr[t][j][0] = x0.x; xr[t][j][1] = x0.y; xr[t][j][2] = x0.z; xr[t][j][3] = x0.w;
+                xr[t][j][4] = x1.x; xr[t][j][5] = x1.y; xr[t][j][6] = x1.z; xr[t][j][7] = x1.w;
+              } else {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+                for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+              }
             }
           }
+          cached_u = u;
+          cached_g = g0;
         }
-        cached_u = u;
-        cached_g = g0;
-      }
-      if (g0 == 0) mbar_wait(&full[s], (it / SA) & 1, abort_flag, a.ws.err);
-      const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SA_B);
-      if (m - g0 == 1) {  // a single token: half the FMAs, four rows per pass
-        const float(&x1)[1][kCPLf][8] = reinterpret_cast<const float(&)[1][kCPLf][8]>(xr[0]);
-        for (int i0 = 0; i0 < nrow; i0 += 4) {
-          const uint16_t* rp[4];
+        if (!waited) {
+          mbar_wait(&full[s], (it / SA) & 1, abort_flag, a.ws.err);
+          waited = true;
+        }
+        const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SA_B);
+        if (m - g0 == 1) {  // a single token: half the FMAs, four rows per pass
+          const float(&x1)[1][kCPLf][8] = reinterpret_cast<const float(&)[1][kCPLf][8]>(xr[0]);
+          for (int i0 = 0; i0 < np; i0 += 4) {
+            const uint16_t* rp[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int i = min(i0 + k, nrow - 1), pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
-            rp[k] = st + (size_t)(gu * PS + pi) * d;
+            for (int k = 0; k < 4; ++k) rp[k] = st + (size_t)min(i0 + k, np - 1) * d;
+            float v[4];
+            rows_dot<1, 4>(rp, np - i0, x1, qbase, qpw, lane, v);
+            const float tot = warp_reduce_multi<4>(v, lane);
+            const int i = i0 + multi_index<4>(lane);
+            if (multi_writer<4>(lane) && i < np) pb[((size_t)(gu * PC + i) * B + g0) * kCW + warp] = tot;
           }
-          float v[4];
-          rows_dot<1, 4>(rp, nrow - i0, x1, qbase, qpw, lane, v);
-          const float tot = warp_reduce_multi<4>(v, lane);
-          const int i = i0 + multi_index<4>(lane);
-          if (multi_writer<4>(lane) && i < nrow) {
-            const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
-            pb[((size_t)(gu * PS + pi) * B + g0) * kCW + warp] = tot;
-          }
+          continue;
         }
-        continue;
-      }
-      for (int i0 = 0; i0 < nrow; i0 += kRI) {
-        const uint16_t* rp[kRI];
+        for (int i0 = 0; i0 < np; i0 += kRI) {
+          const uint16_t* rp[kRI];
 #pragma unroll
-        for (int k = 0; k < kRI; ++k) {
-          const int i = min(i0 + k, nrow - 1), pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
-          rp[k] = st + (size_t)(gu * PS + pi) * d;
-        }
-        float v[kRI * NT];
-        rows_dot<NT, kRI>(rp, nrow - i0, xr, qbase, qpw, lane, v);
-        const float tot = warp_reduce_multi<kRI * NT>(v, lane);
-        const int vi = multi_index<kRI * NT>(lane), i = i0 + vi / NT, t = vi % NT;
-        if (multi_writer<kRI * NT>(lane) && i < nrow && g0 + t < m) {
-          const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
-          pb[((size_t)(gu * PS + pi) * B + g0 + t) * kCW + warp] = tot;
+          for (int k = 0; k < kRI; ++k) rp[k] = st + (size_t)min(i0 + k, np - 1) * d;
+          float v[kRI * NT];
+          rows_dot<NT, kRI>(rp, np - i0, xr, qbase, qpw, lane, v);
+          const float tot = warp_reduce_multi<kRI * NT>(v, lane);
+          const int vi = multi_index<kRI * NT>(lane), i = i0 + vi / NT, t = vi % NT;
+          if (multi_writer<kRI * NT>(lane) && i < np && g0 + t < m)
+            pb[((size_t)(gu * PC + i) * B + g0 + t) * kCW + warp] = tot;
         }
       }
+      if (!waited) mbar_wait(&full[s], (it / SA) & 1, abort_flag, a.ws.err);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (m <= 0) mbar_wait(&full[s], (it / SA) & 1, abort_flag, a.ws.err);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    csync();  // every warp's partials of this stage are in pb (the other buffer is the next stage's)
+    csync();  // every warp's partials of this chunk are in pb (the other buffer is the next chunk's)
     // one warp per (pair, token): lanes 0..14 hold the gate partials, 16..30 the up partials
     for (int z = warp; z < np * m; z += kCW) {
       const int pi = z / m, t = z - pi * m, w = lane & 15;
-      float v = (w < kCW) ? pb[((size_t)((lane >> 4) * PS + pi) * B + t) * kCW + w] : 0.f;
+      float v = (w < kCW) ? pb[((size_t)((lane >> 4) * PC + pi) * B + t) * kCW + w] : 0.f;
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       const float gs = __shfl_sync(0xffffffffu, v, 0), us = __shfl_sync(0xffffffffu, v, 16);
@@ -402,10 +408,10 @@ size_t up128h(size_t x) { return (x + 127) & ~size_t(127); }
 bool plan_large(LayerArgs& a, int G, size_t optin) {
   const size_t budget = optin - 1024;
   const size_t bars = 2 * kMaxStages * 8 + 64;
-  {  // gate/up: two pairs per stage (2 gate + 2 up rows, one copy each)
+  {  // gate/up: chunks of up to PC pairs, two one-copy stages (gate rows, up rows) per chunk
     KTune& t = a.k3;
-    t.rows_per_stage = 2;
-    const size_t SA_B = up128h((size_t)2 * t.rows_per_stage * a.d * 2);
+    t.rows_per_stage = kGateUpChunk;
+    const size_t SA_B = up128h((size_t)t.rows_per_stage * a.d * 2);
     const size_t part = (size_t)2 * 2 * t.rows_per_stage * a.B * kCW * sizeof(float);
     const size_t extra = up128h(part + (size_t)(a.E + 1 + a.B * a.k) * sizeof(int)) + bars;
     t.stages = (budget > extra) ? (int)std::min<size_t>(kMaxStages, (budget - extra) / SA_B) : 0;
