@@ -29,15 +29,28 @@ __device__ __forceinline__ void unpack8f(uint4 w, float* f) {
 // Chunk of lane `lane` in warp w's K slice: q = w * qpw + j * 32 + lane, valid if j*32+lane < qpw.
 __device__ __forceinline__ bool cvalid(int qpw, int j, int lane) { return j * 32 + lane < qpw; }
 
+// d = a * b + d on a pair of fp32 lanes with one instruction (sm_100 packed FMA; each lane
+// rounds exactly like fmaf).
+__device__ __forceinline__ void ffma2(float2& d, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d.x), "+f"(d.y)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // Per-lane partial dots of R bf16 rows (shared memory) with NT register slices of the
 // activations: out[r * NT + t].  Rows r >= nr contribute zeros.  All chunk loads of all
-// rows are issued before the first FMA, and the R * NT * kA accumulators are independent
-// FMA chains (kA per row and token), so a warp's pass over a stage is one short chain
-// instead of R dependent ones.
+// rows are issued before the first FMA; the accumulators are independent chains of packed
+// FMAs (an even and an odd element per instruction, kA pairs per row and token), so a
+// warp's pass over a stage is one short chain instead of R dependent ones.
 template <int NT, int R>
 __device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr, const float (&x)[NT][kCPLf][8],
                                          int qbase, int qpw, int lane, float (&out)[R * NT]) {
-  constexpr int kA = (R * NT >= 8) ? 1 : 8 / (R * NT);
+  constexpr int kA = (R * NT >= 4) ? 1 : 4 / (R * NT);  // accumulator pairs per (row, token)
   uint4 w[R][kCPLf];
 #pragma unroll
   for (int r = 0; r < R; ++r)
@@ -46,13 +59,13 @@ __device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr,
       w[r][j] = (r < nr && cvalid(qpw, j, lane))
                     ? *reinterpret_cast<const uint4*>(rp[r] + (size_t)(qbase + j * 32 + lane) * 8)
                     : make_uint4(0, 0, 0, 0);
-  float acc[R][NT][kA];
+  float2 acc[R][NT][kA];
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
-      for (int e = 0; e < kA; ++e) acc[r][t][e] = 0.f;
+      for (int e = 0; e < kA; ++e) acc[r][t][e] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < kCPLf; ++j)
 #pragma unroll
@@ -62,7 +75,8 @@ __device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr,
 #pragma unroll
       for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[r][t][e % kA] = fmaf(wf[e], x[t][j][e], acc[r][t][e % kA]);
+        for (int e = 0; e < 4; ++e)
+          ffma2(acc[r][t][e % kA], wf[2 * e], wf[2 * e + 1], x[t][j][2 * e], x[t][j][2 * e + 1]);
     }
 #pragma unroll
   for (int r = 0; r < R; ++r)
@@ -70,7 +84,7 @@ __device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr,
     for (int t = 0; t < NT; ++t) {
       float v = 0.f;
 #pragma unroll
-      for (int e = 0; e < kA; ++e) v += acc[r][t][e];
+      for (int e = 0; e < kA; ++e) v += acc[r][t][e].x + acc[r][t][e].y;
       out[r * NT + t] = v;
     }
 }
