@@ -27,6 +27,12 @@ def top_gap(logits_row: np.ndarray, k: int) -> float:
     return float(np.min(s[:-1] - s[1:])) if s.size > 1 else np.inf
 
 
+def boundary_gap(logits_row: np.ndarray, k: int) -> float:
+    """Gap between the k-th and (k+1)-th largest values of one row (inf when k = E)."""
+    s = np.sort(np.asarray(logits_row, np.float64))[::-1][: k + 1]
+    return float(s[k - 1] - s[k]) if s.size > k else np.inf
+
+
 class LayerRef:
     """One layer's seeded weights on the host plus oracle calls over them."""
 
@@ -64,7 +70,7 @@ def token_resid(seed, dims, b, attempt):
 
 def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=None,
                min_gap: float = 1e-3, max_attempts: int = 200, resid0=None, attn0=None,
-               refs=None, moe_tokens=None) -> dict:
+               refs=None, moe_tokens=None, min_boundary_gap=None) -> dict:
     """Seeded inputs for a B-token, n_layers-deep step and the oracle's answers.
 
     ``checked`` lists the tokens the oracle follows through every layer (all
@@ -74,6 +80,9 @@ def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=N
     output (used by constructed batch-2 cases); fixed inputs are never redrawn.
     ``moe_tokens`` (one-layer cases only) limits the expert half of the oracle to a
     subset of the checked tokens; the others get indices and gates only.
+    ``min_boundary_gap`` (one value per layer) also asks of each checked token's draw
+    that the k-th and (k+1)-th largest logits lie that far apart, so that an input
+    perturbed within half of it still selects the same experts.
 
     Returns attn [L][B][d_o] and resid [B][d] (bf16 bits), the attempts used,
     and per layer the oracle's front results and outputs for checked tokens.
@@ -107,7 +116,10 @@ def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=N
                         cur[b] = token_resid(seed, dims, b, att)
                         resid[b] = cur[b]
                 f = ref.front(attn[l, b][None], cur[b][None])
-                if top_gap(f["logits64"][0], dims.k) >= min_gap:
+                ok = top_gap(f["logits64"][0], dims.k) >= min_gap
+                if ok and min_boundary_gap is not None:
+                    ok = boundary_gap(f["logits64"][0], dims.k) >= min_boundary_gap[l]
+                if ok:
                     break
                 if fixed0 and l == 0:
                     raise RuntimeError("fixed layer-0 inputs violate the gap rule")

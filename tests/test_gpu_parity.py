@@ -1,8 +1,9 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
 
 Every case uses seeded synthetic inputs; indices and their order must match
-exactly, gates and intermediates within fp32-vs-fp64 tolerances, the bf16
-output within the layer's bar (tests/harness.py).
+exactly (in a stack's later layers: any order the oracle's logits allow within
+the chains' divergence), gates and intermediates within fp32-vs-fp64 tolerances,
+the bf16 output within the layer's bar (tests/harness.py).
 """
 import gc
 
@@ -36,9 +37,12 @@ def check_case(stack: H.GpuStack, case: dict, sampled=None, check_intermediates=
     B = case["attn"].shape[1]
     for l, per in enumerate(case["layers"]):
         for b in per["idx"]:
-            assert np.array_equal(idx[l, b], per["idx"][b]), (l, b, idx[l, b], per["idx"][b])
-            tol = H.GATE_ATOL if l == 0 else H.GATE_ATOL_STACKED
-            assert np.allclose(gate[l, b], per["gate"][b], atol=tol, rtol=0), (l, b)
+            if l == 0:
+                assert np.array_equal(idx[l, b], per["idx"][b]), (l, b, idx[l, b], per["idx"][b])
+                assert np.allclose(gate[l, b], per["gate"][b], atol=H.GATE_ATOL, rtol=0), (l, b)
+            else:
+                H.check_route_stacked(idx[l, b], gate[l, b], per["idx"][b], per["gate"][b],
+                                      per["logits64"][b], H.stack_tau(l), where=(l, b))
     last = case["layers"][-1]
     toks = sorted(last["out_ref"]) if sampled is None else sampled
     res = []
@@ -194,7 +198,8 @@ def test_stack8(stack8, B, prefetch):
     st = H.GpuStack(seed, synth.TP16, n_layers=8, max_batch=64, prefetch=prefetch, weights=w)
     try:
         sampled = [0] if B == 1 else [0, 37]
-        case = build_case(seed, synth.TP16, B, n_layers=8, checked=sampled, refs=refs)
+        case = build_case(seed, synth.TP16, B, n_layers=8, checked=sampled, refs=refs,
+                          min_boundary_gap=[2 * H.stack_tau(l) for l in range(8)])
         check_case(st, case, sampled=sampled)
     finally:
         st.close()
