@@ -161,7 +161,9 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     LayerArgs a = layer_args(h, l, B, attn, resid, out, idx, gate);
     const Variant v = variant_of(h, a);
-    e = v.oproj_small ? launch_oproj_s(a, G, h->cap, l > 0, h->smem_optin) : launch_oproj(a, G, h->cap, l > 0);
+    e = v.oproj_small                         ? launch_oproj_s(a, G, h->cap, l > 0, h->smem_optin)
+        : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, h->cap, l > 0)
+                                            : launch_oproj(a, G, h->cap, l > 0);
     if (e == cudaSuccess) e = launch_router_s(a, G, h->cap, true, h->smem_optin);
     kernels += 2;
     if (v.experts_small) {
@@ -318,6 +320,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   if (e == cudaSuccess) e = set_kernel_attributes(h->smem_optin);
   if (e == cudaSuccess) e = set_small_attributes(h->smem_optin);
   if (e == cudaSuccess) e = set_large_attributes(h->smem_optin);
+  if (e == cudaSuccess) e = set_tc_attributes(h->smem_optin);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -483,7 +486,9 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
     LayerArgs a = layer_args(h, l, batch, attn_out, residual_in, out, topk_idx, topk_gate);
     const Variant v = variant_of(h, a);
     timed(1, s, [&](cudaStream_t st) {
-      return v.oproj_small ? launch_oproj_s(a, G, st, false, h->smem_optin) : launch_oproj(a, G, st, false);
+      return v.oproj_small                         ? launch_oproj_s(a, G, st, false, h->smem_optin)
+             : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, st, false)
+                                                 : launch_oproj(a, G, st, false);
     });
     timed(2, s, [&](cudaStream_t st) { return launch_router_s(a, G, st, false, h->smem_optin); });
     if (v.experts_small) {
