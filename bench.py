@@ -158,6 +158,9 @@ def algorithmic_bytes(dims, B, n_union):
         "down_rows": n_union * d * I * 2 + B * k * I * 4 + B * d * 4 + B * d * 2,
         # small-M expert kernel: gate/up and down weights of the union, x and h in, out
         "experts_small_m": n_union * 3 * I * d * 2 + B * E * 4 + 2 * B * d * 4 + B * d * 2,
+        # fused batch <= 2 layer kernel: every weight of the layer once, attn_out and the
+        # residual in, the output out (its h, x and logits stay in L2)
+        "layer_fused_small_m": d * do * 2 + E * d * 2 + d * 2 + n_union * 3 * I * d * 2 + B * (do * 2 + d * 4),
     }
 
 
@@ -227,7 +230,8 @@ def run_ours(args, rank, world):
     out = torch.empty((B, dims.d), dtype=torch.bfloat16, device="cuda")
     idx = torch.empty((L, B, dims.k), dtype=torch.int32, device="cuda")
     gate = torch.empty((L, B, dims.k), dtype=torch.float32, device="cuda")
-    cfg = md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, max(B, 1), L, enable_prefetch=args.prefetch)
+    cfg = md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, max(B, 1), L, enable_prefetch=args.prefetch,
+                    force_variant=args.force_variant)
     s = torch.cuda.current_stream()
     hs = [md.moe_decode_create(cfg, w, s) for w in weight_sets]
     h = hs[0]
@@ -382,6 +386,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="tp16_b1", choices=sorted(WORKLOADS))
     ap.add_argument("--prefetch", type=int, default=1)
+    ap.add_argument("--force-variant", type=int, default=0, choices=[0, 1, 2],
+                    help="kernel choice: 0 by batch size, 1 unfused batch <= 2 kernels, 2 large-batch "
+                         "kernels at every batch (comparison runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-run", type=int, default=0,
                     help="profiling mode: warm up, replay the step N times, print nothing")
@@ -393,6 +400,7 @@ def main():
     dname, B, L, mode = WORKLOADS[args.workload]
     config = {"workload": args.workload, "batch": B, "layers": L, "shape": dname,
               "prefetch": bool(args.prefetch and L > 1),
+              "force_variant": args.force_variant,
               "l2": (f"inputs larger than L2: the step cycles over {rotation(L)} independently seeded weight "
                      "copies, no flush" if rotation(L) > 1 else
                      f"inputs larger than L2: {L} layers of distinct weights per step, no flush"),

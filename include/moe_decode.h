@@ -74,12 +74,14 @@ enum {
  *   max_batch  largest batch passed to step                          1 <= max_batch <= 64
  *   n_layers   layers run back to back by one step (residual chains)  1 <= n_layers <= 64
  *   rms_eps    RMSNorm epsilon (> 0; the layer uses 1e-6)
- *   enable_prefetch  1: layer l's router kernel prefetches into L2 what layer l+1 reads
- *                    first (its router matrix, RMSNorm scale and the leading 16 MB of
- *                    its W_o, split by the CTA that reads them) while layer l's top-k
- *                    and first expert bytes leave HBM idle; no extra kernel
- *   force_variant    0 or 1: expert kernels by batch size (the fused small-M kernel at
- *                    B <= 2, separate large-batch gate/up and down kernels above);
+ *   enable_prefetch  1: layer l prefetches into L2 what layer l+1 reads first (its
+ *                    router matrix, RMSNorm scale and the leading 16 MB of its W_o,
+ *                    split by the CTA that reads them), issued once layer l's own
+ *                    router rows are in flight; no extra kernel
+ *   force_variant    0: kernels by batch size (B = 1: one fused layer kernel; B = 2:
+ *                    o_proj, router, small-M expert kernel; above: o_proj, router,
+ *                    gate/up, down);
+ *                    1: at B = 1 too the three small-batch kernels (testing);
  *                    2: the large-batch kernels at every batch size (testing)             */
 typedef struct {
   int d, d_o, n_experts, top_k, inter, max_batch, n_layers;
@@ -159,7 +161,7 @@ MOE_API int moe_decode_kernels_per_step(moe_decode_handle* h, int batch);
  * max_kernels entries) and a short kernel name id to kernel_id (host, or NULL):
  * 1 o_proj+residual+RMS, 2 router+top-k (and the next layer's L2 prefetch),
  * 3 small-M expert kernel (gate/up and down), 4 large-batch gate/up, 5 large-batch
- * down+combine.  Same buffers as
+ * down+combine, 6 fused batch <= 2 layer kernel (all of a layer).  Same buffers as
  * moe_decode_step.  Returns the number of kernels timed (or a negative code). */
 MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_out,
                                     const void* residual_in, void* out, int32_t* topk_idx,
@@ -190,7 +192,7 @@ MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void*
  * launched then.  MOE_ERR_CUDA on a failed CUDA call.
  * The first call on each device, with that device current, looks up the array's address
  * (cudaGetSymbolAddress) and sets kernel attributes; make that first call before any stream
- * capture begins.  Each call zeroes the barrier counter and error word at the head of the
+ * capture begins.  Each call zeroes the barrier counters and error word at the head of the
  * array before its kernels run; nothing else needs a starting value.
  * All calls on a device share the array: calls whose executions overlap (different streams,
  * or threads without ordering) race on it and corrupt each other's results.  Outputs are

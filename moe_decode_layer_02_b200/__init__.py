@@ -30,7 +30,7 @@ EXPORTED = ("moe_decode_create", "moe_decode_step", "moe_decode_step_host", "moe
             "moe_decode_step_static", "moe_decode_destroy", "moe_decode_strerror")
 
 KERNEL_NAMES = {1: "oproj_residual_rmsnorm", 2: "router_topk", 3: "experts_small_m", 4: "gateup_rows",
-                5: "down_rows"}
+                5: "down_rows", 6: "layer_fused_small_m"}
 
 
 class moe_decode_config(ctypes.Structure):

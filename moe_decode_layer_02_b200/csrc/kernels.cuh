@@ -5,8 +5,9 @@
 
 namespace moe {
 
-// Device counters: o_proj (unused), router ticket, expert-kernel grid barrier count, spare.
-enum Counter { kCntOproj = 0, kCntRouter = 1, kCntGateUp = 2, kNumCounters = 4 };
+// Device counters: fused layer kernel's exit ticket, router ticket, expert-kernel grid
+// barrier count, fused layer kernel's grid barrier count.  All are zero between launches.
+enum Counter { kCntLayerExit = 0, kCntRouter = 1, kCntGateUp = 2, kCntLayer = 3, kNumCounters = 4 };
 
 // Library-owned device workspace (one per handle).
 struct Workspace {
@@ -69,6 +70,10 @@ cudaError_t set_small_attributes(size_t smem_optin);
 cudaError_t launch_oproj_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t launch_router_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t launch_experts_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
+// The three small-batch kernels fused into one cooperative launch per layer (batch <= 2).
+bool plan_fused(LayerArgs& a, int grid, size_t smem_optin);
+bool layer_fused_ok(const LayerArgs& a, size_t smem_optin);
+cudaError_t launch_layer_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t set_kernel_attributes(size_t smem_optin);
 
 // o_proj above batch 2 on the tensor cores with 2-D TMA tiles (kernels_tc.cu).

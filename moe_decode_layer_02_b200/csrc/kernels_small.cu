@@ -330,15 +330,17 @@ __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// `count` is zero when the kernel starts (the router kernel clears it before its dependents
-// pass their dependency wait) and is used once per launch: the barrier opens when it reaches
-// gridDim.x, so the last arrival's add is the release (no second round trip).
-__device__ void grid_barrier(unsigned* count, volatile int* abort_flag, uint32_t* err) {
-  csync();  // the CTA's writes happen before thread 0's release (cumulative through the barrier)
+// `count` is zero when the kernel starts and only grows during a launch: the n-th barrier
+// of a launch opens when it reaches n * gridDim.x (`target`), so the last arrival's add is
+// the release (no second round trip).  Who clears it: for the expert kernel, the router
+// kernel before its dependents pass their dependency wait; for the fused layer kernel, its
+// own last CTA to finish (layer_exit).
+__device__ void grid_barrier(unsigned* count, unsigned target, volatile int* abort_flag, uint32_t* err) {
+  // The CTA's writes happen before thread 0's release add: bar.sync orders them before it
+  // and the release is cumulative, so no separate fence is needed.
+  csync();
   if (threadIdx.x == 0) {
-    __threadfence();
     red_release_add(count, 1u);
-    const unsigned target = gridDim.x;
     if (ld_acquire_u32(count) < target) {
       const unsigned long long t0 = globaltimer();
       while (ld_acquire_u32(count) < target) {
@@ -356,6 +358,108 @@ __device__ void grid_barrier(unsigned* count, volatile int* abort_flag, uint32_t
 
 }  // namespace
 
+// Phase B of the batch <= 2 expert kernels (consumer warps): out = bf16(h + sum over the
+// union experts of W_down[e] rows [i0, i0 + nrows) . a_s[e]), the W_down blocks arriving in
+// the B ring.  A stage holds EPS experts' blocks of this CTA's rows; every load of a stage is
+// issued before its FMAs.  Warp w owns rows w, w + 15, ...; lane l holds elements
+// [l * epl, (l + 1) * epl) of each row and accumulates over all experts in registers.
+template <int NT, int EPL>
+__device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned char* ring, size_t SB_B, int SBn,
+                                             uint64_t* fullB, uint64_t* emptyB, volatile int* abort_flag,
+                                             const float* a_s, int U, int i0, int nrows, int warp, int lane) {
+  constexpr int kRPW = 4;  // rows per warp (rows_max <= 60)
+  constexpr int kEPS = experts_per_stage(EPL);
+  const int d = a.d, I = a.I, B = a.B;
+  const int epl = (EPL > 0) ? EPL : I / 32;
+  float acc[kRPW][NT];
+#pragma unroll
+  for (int i = 0; i < kRPW; ++i)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[i][t] = 0.f;
+  int g = 0;
+  for (int u0 = 0; u0 < U && nrows > 0; u0 += kEPS, ++g) {
+    const int s = g % SBn, ne = min(kEPS, U - u0);
+    mbar_wait(&fullB[s], (g / SBn) & 1, abort_flag, a.ws.err);
+    const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB_B);
+    if constexpr (EPL == 4 || EPL == 8) {
+      using WT = typename std::conditional<EPL == 4, uint2, uint4>::type;
+      float av[kEPS][NT][EPL];
+      WT wv[kEPS][kRPW];
+#pragma unroll
+      for (int e = 0; e < kEPS; ++e) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const float* ap = a_s + ((size_t)(u0 + min(e, ne - 1)) * NT + t) * I + lane * EPL;
+#pragma unroll
+          for (int x = 0; x < EPL; x += 4) {
+            const float4 f = (e < ne) ? *reinterpret_cast<const float4*>(ap + x) : make_float4(0.f, 0.f, 0.f, 0.f);
+            av[e][t][x] = f.x; av[e][t][x + 1] = f.y; av[e][t][x + 2] = f.z; av[e][t][x + 3] = f.w;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kRPW; ++i) {
+          const int rl = warp + kCW * i;
+          WT w{};
+          if (e < ne && rl < nrows) w = *reinterpret_cast<const WT*>(st + ((size_t)e * nrows + rl) * I + lane * EPL);
+          wv[e][i] = w;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < kEPS; ++e)
+#pragma unroll
+        for (int i = 0; i < kRPW; ++i) {
+          float wf[8];
+          if constexpr (EPL == 4) {
+            wf[0] = bf16lo(wv[e][i].x); wf[1] = bf16hi(wv[e][i].x);
+            wf[2] = bf16lo(wv[e][i].y); wf[3] = bf16hi(wv[e][i].y);
+          } else {
+            unpack8f(reinterpret_cast<const uint4&>(wv[e][i]), wf);
+          }
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            float sdot = 0.f;
+#pragma unroll
+            for (int x = 0; x < EPL; ++x) sdot = fmaf(wf[x], av[e][t][x], sdot);
+            acc[i][t] += sdot;
+          }
+        }
+    } else {  // any other I: one expert per stage, epl <= 16 elements per lane
+      const float* ap = a_s + (size_t)u0 * NT * I + lane * epl;
+#pragma unroll
+      for (int i = 0; i < kRPW; ++i) {
+        const int rl = warp + kCW * i;
+        if (rl < nrows) {
+          const uint16_t* wr = st + (size_t)rl * I + lane * epl;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            float sdot = 0.f;
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+              if (x < epl) sdot = fmaf(bf16f(wr[x]), ap[(size_t)t * I + x], sdot);
+            acc[i][t] += sdot;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&emptyB[s]);
+  }
+  {
+    float v[kRPW * NT];
+#pragma unroll
+    for (int i = 0; i < kRPW; ++i)
+#pragma unroll
+      for (int t = 0; t < NT; ++t) v[i * NT + t] = acc[i][t];
+    const float tot = warp_reduce_multi<kRPW * NT>(v, lane);
+    const int vi = multi_index<kRPW * NT>(lane), i = vi / NT, t = vi % NT, rl = warp + kCW * i;
+    if (multi_writer<kRPW * NT>(lane) && rl < nrows && t < B) {
+      const size_t o = (size_t)t * d + i0 + rl;
+      const __nv_bfloat16 bv = __float2bfloat16_rn(ld_act(&a.ws.h[o]) + tot);
+      a.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
+    }
+  }
+}
+
 // =============================================================================
 // K3 (batch <= 2): the expert kernel.  Routing once per CTA, then
 //   phase A  gate/up + SiLU*mul: pairs (union expert u, row p) in flattened order, CTA c takes
@@ -371,7 +475,6 @@ __device__ void grid_barrier(unsigned* count, volatile int* abort_flag, uint32_t
 template <int NT, int EPL>
 __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kRPW = 4;  // rows per warp in phase B (rows_max <= 60)
   constexpr int kEPS = experts_per_stage(EPL);
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, I = a.I, B = a.B;
@@ -534,7 +637,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
     }
   }
 
-  grid_barrier(&a.ws.counters[kCntGateUp], abort_flag, a.ws.err);
+  grid_barrier(&a.ws.counters[kCntGateUp], gridDim.x, abort_flag, a.ws.err);
 
   // ---- phase B (consumers) ------------------------------------------------------------
   // a_s[u][t][:] = gate * a of (union expert u, token t), zero where t did not select u, so
@@ -552,97 +655,425 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   }
   csync();
 
-  // A stage holds EPS experts' blocks of this CTA's rows; every load of a stage is issued
-  // before its FMAs.  Warp w owns rows w, w + 15, ...; lane l holds elements
-  // [l * epl, (l + 1) * epl) of each row and accumulates over all experts in registers.
-  const int epl = (EPL > 0) ? EPL : I / 32;
-  float acc[kRPW][NT];
+  combine_down<NT, EPL>(a, ring, SB_B, SBn, fullB, emptyB, abort_flag, a_s, U, i0, nrows, warp, lane);
+}
+
+// =============================================================================
+// The fused layer kernel (batch <= 2): the three kernels above as one cooperative launch,
+// with grid barriers where a kernel boundary was:
+//   o_proj     h = residual + W_o . attn_out, per-CTA sums of h^2 (as k_oproj_f).  The
+//              producer streams this CTA's router rows into the same ring right after its
+//              W_o rows, so W_r leaves HBM while the o_proj tail computes.
+//   barrier 1  (every h and sum of h^2 written)
+//   router     rstd from the 148 partial sums (same order in every CTA), x in registers,
+//              logits of this CTA's rows from the ring (as k_router_f)
+//   barrier 2  (every logit and x written)
+//   routing    recomputed in every CTA, then phase A, barrier 3 and phase B as in k_experts_f.
+// Every CTA adds one to the exit ticket after its last barrier; the last one clears the
+// barrier count for the next launch.
+// =============================================================================
+namespace {
+
+// Scratch floats shared by the o_proj, router and phase A partial sums (each phase's use
+// ends before the next begins).  Phase B's gated activations live in the ring region, after
+// phase B's stages.
+__host__ __device__ constexpr size_t layer_scratch_floats(int NT, int RM, int RMr, int PM) {
+  const size_t o = (size_t)RM * kCW * NT + (size_t)NT * RM;   // o_proj partials + h^2
+  const size_t r = (size_t)RMr * kCW * NT + 64;                // router partials + rstd
+  const size_t pa = (size_t)PM * 2 * kCW * NT;                 // phase A partials
+  const size_t m1 = o > r ? o : r;
+  return m1 > pa ? m1 : pa;
+}
+
+// Called by thread 0 after its CTA's last grid barrier.
+__device__ __forceinline__ void layer_exit(unsigned* counters) {
+  const unsigned G = gridDim.x;
+  if (atomicAdd(&counters[kCntLayerExit], 1u) == G - 1) {  // every CTA is past its last barrier
+    counters[kCntLayer] = 0;
+    counters[kCntLayerExit] = 0;
+    __threadfence();
+  }
+}
+
+}  // namespace
+
+template <int NT, int EPL>
+__global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int kEPS = experts_per_stage(EPL);
+  const int G = gridDim.x, c = blockIdx.x;
+  const int d = a.d, d_o = a.d_o, I = a.I, B = a.B, E = a.E;
+  const int SO = a.k1.stages, RS = a.k1.rows_per_stage, RM = a.k1.rows_max;
+  const int RSr = a.k2.rows_per_stage, RMr = a.k2.rows_max;
+  const int SA = a.k3.stages, PS = a.k3.rows_per_stage, PM = a.k3.rows_max;
+  const int SBn = a.k4.stages;
+  const uint32_t orow_bytes = (uint32_t)d_o * 2u, row_bytes = (uint32_t)d * 2u, drow_bytes = (uint32_t)I * 2u;
+  const size_t SO_B = std::max(al128((size_t)RS * orow_bytes), al128(row_bytes));  // a W_r row fits a stage
+  const size_t SA_B = al128((size_t)2 * PS * row_bytes), SB_B = al128((size_t)kEPS * RM * drow_bytes);
+  const size_t a_s_bytes = (size_t)std::min(E, B * a.k) * NT * I * 4;
+  const size_t region =
+      std::max(std::max((size_t)SO * SO_B, (size_t)SA * SA_B), (size_t)SBn * SB_B + a_s_bytes);
+  const size_t scratch_f = layer_scratch_floats(NT, RM, RMr, PM);
+  long long lo, hi;
+  split_range(d, G, c, lo, hi);
+  const int i0 = (int)lo, nrows = (int)(hi - lo);  // o_proj rows = phase B output rows
+  split_range(E, G, c, lo, hi);
+  const int e0 = (int)lo, nr = (int)(hi - lo);      // router rows
+
+  unsigned char* ring = smem;
+  float* part = reinterpret_cast<float*>(ring + region);
+  float* sq = part + RM * kCW * NT;   // o_proj: [NT][RM]
+  float* rstd_s = part + RMr * kCW * NT;  // router
+  // phase B: after phase B's stages (phase A's fills have all landed and been read by then)
+  float* a_s = reinterpret_cast<float*>(ring + (size_t)SBn * SB_B);
+  SmallRoute* rt = reinterpret_cast<SmallRoute*>(smem + al128(region + scratch_f * sizeof(float)));
+  RouteScratch* sc = reinterpret_cast<RouteScratch*>(rt + 1);
+  float* fb = reinterpret_cast<float*>(sc + 1);
+  uint64_t* fullO = reinterpret_cast<uint64_t*>(
+      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + 2 * 2 * kCandStride) - smem)));
+  uint64_t* emptyO = fullO + kMaxStages;
+  uint64_t* fullA = emptyO + kMaxStages;
+  uint64_t* emptyA = fullA + kMaxStages;
+  uint64_t* fullB = emptyA + kMaxStages;
+  uint64_t* emptyB = fullB + kMaxStages;
+  int* s_misc = reinterpret_cast<int*>(emptyB + kMaxStages);
+  volatile int* abort_flag = s_misc;
+  unsigned* bar_count = &a.ws.counters[kCntLayer];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  if (tid == 0) {
+    init_ring(fullO, emptyO, SO, kCW);
+    init_ring(fullA, emptyA, SA, kCW);
+    init_ring(fullB, emptyB, SBn, kCW);
+    s_misc[0] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_trigger();
+
+  const int qbase_o = (d_o / 8) * warp / kCW, qpw_o = (d_o / 8) * (warp + 1) / kCW - qbase_o;
+  const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
+  int itO = 0;  // O-ring fills (producer) / waits (consumers)
+  if (warp == kCW) {
+    if (lane == 0) {  // weights are static: W_o, then W_r, before the dependency resolves
+      const uint64_t pol = policy_evict_first();
+      bulk_prefetch_l2(a.gamma, row_bytes);  // every CTA reads all of gamma after barrier 1
+      for (int r = i0; r < i0 + nrows; r += RS, ++itO) {
+        const int n = min(RS, i0 + nrows - r);
+        if (!ring_acquire(emptyO, itO, SO, abort_flag, a.ws.err)) break;
+        const int s = itO % SO;
+        mbar_arrive_expect_tx(&fullO[s], n * orow_bytes);
+        bulk_g2s(ring + s * SO_B, a.w_o + (size_t)r * d_o, n * orow_bytes, &fullO[s], pol);
+      }
+      for (int j = 0; j < nr && !*abort_flag; j += RSr, ++itO) {
+        const int n = min(RSr, nr - j);
+        if (!ring_acquire(emptyO, itO, SO, abort_flag, a.ws.err)) break;
+        const int s = itO % SO;
+        mbar_arrive_expect_tx(&fullO[s], n * row_bytes);
+        bulk_g2s(ring + s * SO_B, a.w_r + (size_t)(e0 + j) * d, n * row_bytes, &fullO[s], pol);
+      }
+      if (a.pf_w_o) {  // next layer: what the same CTA reads first, into L2
+        if (nr > 0) bulk_prefetch_l2(a.pf_w_r + (size_t)e0 * d, nr * row_bytes);
+        if (c == 0) bulk_prefetch_l2(a.pf_gamma, row_bytes);
+        size_t left = (size_t)min(a.pf_w_o_rows, nrows) * orow_bytes;
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(a.pf_w_o + (size_t)i0 * d_o);
+        for (size_t off = 0; left > 0;) {
+          const uint32_t n = (uint32_t)min(left, (size_t)65536);
+          bulk_prefetch_l2(src + off, n);
+          off += n;
+          left -= n;
+        }
+      }
+      // The O ring's last fills land and are read (the router rows, after barrier 1) while
+      // the consumers work towards barrier 2; phase A may then reuse the region at once.
+      ring_drain(fullO, itO, SO, a.ws.err);
+      for (int i = itO - SO < 0 ? 0 : itO - SO; i < itO; ++i) mbar_drain(&emptyO[i % SO], (i / SO) & 1, a.ws.err);
+    }
+  } else {
+    // ---- o_proj (consumers) ----------------------------------------------------------
+    pdl_wait();  // attn_out and residual may come from the previous kernel
+    // this thread's residual element of the epilogue (rows x tokens <= 2 * 60 < kCT)
+    float res_v = 0.f;
+    if (tid < nrows * B) {
+      const int rr = tid / B, t = tid % B;
+      res_v = bf16f(__ldcg(reinterpret_cast<const unsigned short*>(a.resid + (size_t)t * d + i0 + rr)));
+    }
+    {
+      constexpr int kRI = 2;
+      float xa[NT][kCPLf][8];
 #pragma unroll
-  for (int i = 0; i < kRPW; ++i)
+      for (int t = 0; t < NT; ++t)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) acc[i][t] = 0.f;
-  int g = 0;
-  for (int u0 = 0; u0 < U && nrows > 0; u0 += kEPS, ++g) {
-    const int s = g % SBn, ne = min(kEPS, U - u0);
-    mbar_wait(&fullB[s], (g / SBn) & 1, abort_flag, a.ws.err);
-    const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SB_B);
-    if constexpr (EPL == 4 || EPL == 8) {
-      using WT = typename std::conditional<EPL == 4, uint2, uint4>::type;
-      float av[kEPS][NT][EPL];
-      WT wv[kEPS][kRPW];
+        for (int j = 0; j < kCPLf; ++j) {
+          uint4 u = make_uint4(0, 0, 0, 0);
+          if (t < B && cvalid(qpw_o, j, lane))
+            u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)(qbase_o + j * 32 + lane) * 8);
+          unpack8f(u, xa[t][j]);
+        }
+      for (int r = i0; r < i0 + nrows; r += RS, ++itO) {
+        const int n = min(RS, i0 + nrows - r), s = itO % SO;
+        mbar_wait(&fullO[s], (itO / SO) & 1, abort_flag, a.ws.err);
+        const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SO_B);
+        for (int j0 = 0; j0 < n; j0 += kRI) {
+          const uint16_t* rp[kRI];
 #pragma unroll
-      for (int e = 0; e < kEPS; ++e) {
+          for (int k = 0; k < kRI; ++k) rp[k] = st + (size_t)min(j0 + k, n - 1) * d_o;
+          float v[kRI * NT];
+          rows_dot<NT, kRI>(rp, n - j0, xa, qbase_o, qpw_o, lane, v);
+          const float tot = warp_reduce_multi<kRI * NT>(v, lane);
+          const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
+          if (multi_writer<kRI * NT>(lane) && j < n) part[((r - i0 + j) * kCW + warp) * NT + t] = tot;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&emptyO[s]);
+      }
+    }
+    csync();
+    if (tid < nrows * B) {
+      const int rr = tid / B, t = tid % B;
+      float sacc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kCW; ++w) sacc += part[(rr * kCW + w) * NT + t];
+      const float hv = res_v + sacc;
+      a.ws.h[(size_t)t * d + i0 + rr] = hv;
+      sq[t * RM + rr] = hv * hv;
+    }
+    csync();
+    if (warp < B) {  // per-CTA sum of h^2, fixed order
+      float ss = 0.f;
+      for (int rr = lane; rr < nrows; rr += 32) ss += sq[warp * RM + rr];
+      ss = warp_sum(ss);
+      if (lane == 0) a.ws.ss_part[(size_t)c * a.maxB + warp] = ss;
+    }
+    grid_barrier(bar_count, (unsigned)G, abort_flag, a.ws.err);
+
+    // ---- router (consumers) ----------------------------------------------------------
+    {
+      for (int t = warp; t < B; t += kCW) {  // fixed order: same bits in every CTA
+        float ss = 0.f;
+        for (int c0 = 0; c0 < G; c0 += 8 * 32) {
+          float pv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int cc = c0 + k * 32 + lane;
+            pv[k] = cc < G ? ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]) : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) ss += pv[k];
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) {
+          const float rv = 1.0f / sqrtf(ss / (float)d + a.eps);
+          rstd_s[t] = rv;
+          if (c == 0) a.ws.rstd[t] = rv;
+        }
+      }
+      float xr[NT][kCPLf][8];
+#pragma unroll
+      for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int j = 0; j < kCPLf; ++j) {
+          if (t < B && cvalid(qpw, j, lane)) {
+            const float* hp = a.ws.h + (size_t)t * d + (size_t)(qbase + j * 32 + lane) * 8;
+            const float4 h0 = ld_act4(hp), h1 = ld_act4(hp + 4);
+            xr[t][j][0] = h0.x; xr[t][j][1] = h0.y; xr[t][j][2] = h0.z; xr[t][j][3] = h0.w;
+            xr[t][j][4] = h1.x; xr[t][j][5] = h1.y; xr[t][j][6] = h1.z; xr[t][j][7] = h1.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+          }
+        }
+      csync();
+#pragma unroll
+      for (int j = 0; j < kCPLf; ++j) {
+        const int q = qbase + j * 32 + lane;
+        float gam[8];
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (cvalid(qpw, j, lane)) u = ld_weight_u4(a.gamma + (size_t)q * 8);
+        unpack8f(u, gam);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          const float* ap = a_s + ((size_t)(u0 + min(e, ne - 1)) * NT + t) * I + lane * EPL;
+          const float rv = (t < B) ? rstd_s[t] : 0.f;
 #pragma unroll
-          for (int x = 0; x < EPL; x += 4) {
-            const float4 f = (e < ne) ? *reinterpret_cast<const float4*>(ap + x) : make_float4(0.f, 0.f, 0.f, 0.f);
-            av[e][t][x] = f.x; av[e][t][x + 1] = f.y; av[e][t][x + 2] = f.z; av[e][t][x + 3] = f.w;
+          for (int e = 0; e < 8; ++e) xr[t][j][e] = xr[t][j][e] * rv * gam[e];
+          if (t < B && cvalid(qpw, j, lane) && q % G == c) {  // each chunk of x is written by one CTA
+            float* xp = a.ws.x + (size_t)t * d + (size_t)q * 8;
+            *reinterpret_cast<float4*>(xp) = make_float4(xr[t][j][0], xr[t][j][1], xr[t][j][2], xr[t][j][3]);
+            *reinterpret_cast<float4*>(xp + 4) = make_float4(xr[t][j][4], xr[t][j][5], xr[t][j][6], xr[t][j][7]);
           }
-        }
-#pragma unroll
-        for (int i = 0; i < kRPW; ++i) {
-          const int rl = warp + kCW * i;
-          WT w{};
-          if (e < ne && rl < nrows) w = *reinterpret_cast<const WT*>(st + ((size_t)e * nrows + rl) * I + lane * EPL);
-          wv[e][i] = w;
         }
       }
+      // every W_r fill first (they landed during the o_proj tail), then passes of 4 / NT
+      // rows across stage boundaries
+      const int itR = itO, nfr = (nr + RSr - 1) / RSr;
+      for (int f = 0; f < nfr; ++f)
+        mbar_wait(&fullO[(itR + f) % SO], ((itR + f) / SO) & 1, abort_flag, a.ws.err);
+      constexpr int kRI = 4 / NT;
+      for (int j0 = 0; j0 < nr; j0 += kRI) {
+        const uint16_t* rp[kRI];
 #pragma unroll
-      for (int e = 0; e < kEPS; ++e)
-#pragma unroll
-        for (int i = 0; i < kRPW; ++i) {
-          float wf[8];
-          if constexpr (EPL == 4) {
-            wf[0] = bf16lo(wv[e][i].x); wf[1] = bf16hi(wv[e][i].x);
-            wf[2] = bf16lo(wv[e][i].y); wf[3] = bf16hi(wv[e][i].y);
-          } else {
-            unpack8f(reinterpret_cast<const uint4&>(wv[e][i]), wf);
-          }
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            float sdot = 0.f;
-#pragma unroll
-            for (int x = 0; x < EPL; ++x) sdot = fmaf(wf[x], av[e][t][x], sdot);
-            acc[i][t] += sdot;
-          }
+        for (int k = 0; k < kRI; ++k) {
+          const int j = min(j0 + k, nr - 1), f = j / RSr;
+          rp[k] = reinterpret_cast<const uint16_t*>(ring + ((itR + f) % SO) * SO_B) + (size_t)(j - f * RSr) * d;
         }
-    } else {  // any other I: one expert per stage, epl <= 16 elements per lane
-      const float* ap = a_s + (size_t)u0 * NT * I + lane * epl;
+        float v[kRI * NT];
+        rows_dot<NT, kRI>(rp, nr - j0, xr, qbase, qpw, lane, v);
+        const float tot = warp_reduce_multi<kRI * NT>(v, lane);
+        const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
+        if (multi_writer<kRI * NT>(lane) && j < nr) part[(j * kCW + warp) * NT + t] = tot;
+      }
+      __syncwarp();
+      if (lane == 0)
+        for (int f = 0; f < nfr; ++f) mbar_arrive(&emptyO[(itR + f) % SO]);
+      itO += nfr;
+      csync();
+      for (int z = tid; z < nr * B; z += kCT) {
+        const int j = z / B, t = z % B;
+        float sacc = 0.f;
 #pragma unroll
-      for (int i = 0; i < kRPW; ++i) {
-        const int rl = warp + kCW * i;
-        if (rl < nrows) {
-          const uint16_t* wr = st + (size_t)rl * I + lane * epl;
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            float sdot = 0.f;
-#pragma unroll
-            for (int x = 0; x < 16; ++x)
-              if (x < epl) sdot = fmaf(bf16f(wr[x]), ap[(size_t)t * I + x], sdot);
-            acc[i][t] += sdot;
-          }
-        }
+        for (int w = 0; w < kCW; ++w) sacc += part[(j * kCW + w) * NT + t];
+        a.ws.logits[(size_t)t * E + e0 + j] = sacc;
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&emptyB[s]);
+    grid_barrier(bar_count, 2u * (unsigned)G, abort_flag, a.ws.err);
   }
+  __syncthreads();  // the producer warp joins: logits are complete
+
+  route_small_cta(a, rt, sc, fb, c == 0);
+  float xr[NT][kCPLf][8];
+  if (warp < kCW) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int j = 0; j < kCPLf; ++j) {
+        if (t < B && cvalid(qpw, j, lane)) {
+          const float* xp = a.ws.x + (size_t)t * d + (size_t)(qbase + j * 32 + lane) * 8;
+          const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
+          xr[t][j][0] = x0.x; xr[t][j][1] = x0.y; xr[t][j][2] = x0.z; xr[t][j][3] = x0.w;
+          xr[t][j][4] = x1.x; xr[t][j][5] = x1.y; xr[t][j][6] = x1.z; xr[t][j][7] = x1.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+        }
+      }
+  }
+
+  const int U = rt->U;
+  long long q0l, q1l;
+  split_range((long long)U * I, G, c, q0l, q1l);
+  const int q0 = (int)q0l, q1 = (int)q1l;
+
+  if (warp == kCW) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      // This CTA's W_down blocks go to L2 while phase A streams, so phase B reads them from
+      // L2: one expert's block per refill once the ring is primed (the prefetches queue in
+      // the same copy engine as the stages, so they are spread out rather than issued at once).
+      int npf = 0;
+      auto prefetch_down = [&](int upto) {
+        for (; npf < upto && npf < U && nrows > 0; ++npf)
+          bulk_prefetch_l2(a.w_down + ((size_t)rt->un_e[npf] * d + i0) * I, nrows * drow_bytes);
+      };
+      int it = 0;
+      int u = q0 / I, p = q0 - u * I;
+      for (int q = q0; q < q1; ++it) {
+        if (it >= SA) prefetch_down(it - SA + 1);
+        const int np = min(min(PS, I - p), q1 - q);
+        if (!ring_acquire(emptyA, it, SA, abort_flag, a.ws.err)) break;
+        const int s = it % SA;
+        const uint16_t* base = a.w_gu + ((size_t)rt->un_e[u] * 2 * I + p) * d;
+        mbar_arrive_expect_tx(&fullA[s], 2u * np * row_bytes);
+        bulk_g2s(ring + s * SA_B, base, np * row_bytes, &fullA[s], pol);
+        bulk_g2s(ring + s * SA_B + (size_t)PS * row_bytes, base + (size_t)I * d, np * row_bytes, &fullA[s], pol);
+        q += np;
+        p += np;
+        if (p == I) { p = 0; ++u; }
+      }
+      prefetch_down(U);
+      ring_drain(fullA, it, SA, a.ws.err);
+      for (int i = it - SA < 0 ? 0 : it - SA; i < it; ++i) mbar_drain(&emptyA[i % SA], (i / SA) & 1, a.ws.err);
+      if (nrows > 0) {
+        const uint32_t blk = (uint32_t)nrows * drow_bytes;
+        int jt = 0;
+        for (int u0 = 0; u0 < U; u0 += kEPS, ++jt) {
+          const int ne = min(kEPS, U - u0);
+          if (!ring_acquire(emptyB, jt, SBn, abort_flag, a.ws.err)) break;
+          const int s = jt % SBn;
+          mbar_arrive_expect_tx(&fullB[s], ne * blk);
+          for (int e = 0; e < ne; ++e)
+            bulk_g2s(ring + s * SB_B + (size_t)e * blk, a.w_down + ((size_t)rt->un_e[u0 + e] * d + i0) * I, blk,
+                     &fullB[s], pol);
+        }
+        ring_drain(fullB, jt, SBn, a.ws.err);
+      }
+    }
+    return;
+  }
+
+  // ---- phase A (consumers) ------------------------------------------------------------
   {
-    float v[kRPW * NT];
+    constexpr int kRI = 4 / NT;
+    int it = 0;
+    int p = q0 - (q0 / I) * I;
+    for (int q = q0; q < q1; ++it) {
+      const int np = min(min(PS, I - p), q1 - q), s = it % SA;
+      mbar_wait(&fullA[s], (it / SA) & 1, abort_flag, a.ws.err);
+      const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SA_B);
+      const int nrow = 2 * np;
+      for (int r0 = 0; r0 < nrow; r0 += kRI) {
+        const uint16_t* rp[kRI];
 #pragma unroll
-    for (int i = 0; i < kRPW; ++i)
+        for (int k = 0; k < kRI; ++k) {
+          const int i = min(r0 + k, nrow - 1), pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
+          rp[k] = st + (size_t)(gu * PS + pi) * d;
+        }
+        float v[kRI * NT];
+        rows_dot<NT, kRI>(rp, nrow - r0, xr, qbase, qpw, lane, v);
+        const float tot = warp_reduce_multi<kRI * NT>(v, lane);
+        const int vi = multi_index<kRI * NT>(lane), i = r0 + vi / NT, t = vi % NT;
+        if (multi_writer<kRI * NT>(lane) && i < nrow) {
+          const int pi = (i < np) ? i : i - np, gu = (i < np) ? 0 : 1;
+          part[(((q - q0 + pi) * 2 + gu) * kCW + warp) * NT + t] = tot;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&emptyA[s]);
+      q += np;
+      p += np;
+      if (p == I) p = 0;
+    }
+    csync();
+    for (int z = tid; z < (q1 - q0) * B; z += kCT) {
+      const int pl = z / B, t = z % B;
+      float gs = 0.f, us = 0.f;
 #pragma unroll
-      for (int t = 0; t < NT; ++t) v[i * NT + t] = acc[i][t];
-    const float tot = warp_reduce_multi<kRPW * NT>(v, lane);
-    const int vi = multi_index<kRPW * NT>(lane), i = vi / NT, t = vi % NT, rl = warp + kCW * i;
-    if (multi_writer<kRPW * NT>(lane) && rl < nrows && t < B) {
-      const size_t o = (size_t)t * d + i0 + rl;
-      const __nv_bfloat16 bv = __float2bfloat16_rn(ld_act(&a.ws.h[o]) + tot);
-      a.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
+      for (int w = 0; w < kCW; ++w) {
+        gs += part[((pl * 2 + 0) * kCW + w) * NT + t];
+        us += part[((pl * 2 + 1) * kCW + w) * NT + t];
+      }
+      const int qq = q0 + pl, u = qq / I, pp = qq - u * I;
+      for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+        if (rt->ent_tok[en] == t) a.ws.a[(size_t)en * I + pp] = gs / (1.0f + expf(-gs)) * us;
     }
   }
+
+  grid_barrier(bar_count, 3u * (unsigned)G, abort_flag, a.ws.err);
+  if (tid == 0) layer_exit(a.ws.counters);
+
+  // ---- phase B (consumers) ------------------------------------------------------------
+  for (int z = tid; z < U * NT * (I / 4); z += kCT) {
+    const int cq = z % (I / 4), ut = z / (I / 4), t = ut % NT, u = ut / NT;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+      if (rt->ent_tok[en] == t) {
+        const float g = rt->ent_gate[en];
+        const float4 x4 = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
+        v = make_float4(g * x4.x, g * x4.y, g * x4.z, g * x4.w);
+      }
+    *reinterpret_cast<float4*>(a_s + ((size_t)u * NT + t) * I + cq * 4) = v;
+  }
+  csync();
+  combine_down<NT, EPL>(a, ring, SB_B, SBn, fullB, emptyB, abort_flag, a_s, U, i0, nrows, warp, lane);
 }
 
 // =============================================================================
@@ -732,6 +1163,56 @@ bool plan_small(LayerArgs& a, int G, size_t optin) {
   return true;
 }
 
+bool plan_fused(LayerArgs& a, int G, size_t optin) {
+  const size_t budget = optin - 1024 - 256;
+  const int NT = 2;
+  KTune& o = a.k1;   // o_proj ring (W_r rows follow in the same ring)
+  KTune& r = a.k2;   // router rows
+  KTune& pa = a.k3;  // phase A
+  KTune& pb = a.k4;  // phase B
+  const size_t orow = (size_t)a.d_o * 2, row = (size_t)a.d * 2;
+  o.rows_max = (a.d + G - 1) / G;
+  if (o.rows_max > 4 * kCW) return false;
+  r.rows_max = (a.E + G - 1) / G;
+  const long long umax = std::min(a.E, std::max(a.B, 1) * a.k);
+  pa.rows_max = (int)((umax * a.I + G - 1) / G);
+  pb.rows_max = o.rows_max;
+  const size_t scratch_f = layer_scratch_floats(NT, o.rows_max, r.rows_max, pa.rows_max);
+  const size_t a_s_bytes = (size_t)umax * NT * a.I * 4;
+  const size_t extra = up128(scratch_f * 4) + kRouteBytes + 6 * kMaxStages * 8 + 64;
+  if (extra >= budget) return false;
+  const size_t cap = budget - extra;
+  o.rows_per_stage = (int)std::max<size_t>(1, std::min<size_t>(32768 / orow, (size_t)o.rows_max));
+  const size_t SO = std::max(up128((size_t)o.rows_per_stage * orow), up128(row));
+  o.stages = (int)std::min<size_t>(kMaxStages, cap / SO);
+  r.rows_per_stage = (int)(SO / row);
+  // the router rows' fills are all resident at once (the consumers wait for every one)
+  if ((r.rows_max + r.rows_per_stage - 1) / r.rows_per_stage > o.stages) return false;
+  size_t SA = 0;
+  pa.stages = 0;
+  for (int ps = 2; ps >= 1 && pa.stages < 2; --ps) {
+    pa.rows_per_stage = ps;
+    SA = up128((size_t)2 * ps * row);
+    pa.stages = (int)std::min<size_t>(kMaxStages, cap / SA);
+  }
+  const int eps = experts_per_stage(a.I / 32);
+  pb.rows_per_stage = eps;
+  const size_t SBd = up128((size_t)eps * pb.rows_max * a.I * 2);
+  pb.stages = cap > a_s_bytes ? (int)std::min<size_t>(kMaxStages, (cap - a_s_bytes) / SBd) : 0;
+  if (o.stages < 2 || pa.stages < 2 || pb.stages < 2) return false;
+  const size_t region = std::max(std::max((size_t)o.stages * SO, (size_t)pa.stages * SA),
+                                 (size_t)pb.stages * SBd + a_s_bytes);
+  o.smem = region + extra;
+  r.smem = pa.smem = pb.smem = o.smem;
+  return o.smem <= budget;
+}
+
+bool layer_fused_ok(const LayerArgs& a0, size_t optin) {
+  LayerArgs a = a0;
+  return a.B <= 2 && a.k <= 32 && a.d <= 8192 && a.d_o <= 8192 && a.E <= 2 * kRouteThreads &&
+         plan_fused(a, 148, optin);
+}
+
 bool small_path_ok(const LayerArgs& a0, size_t optin) {
   LayerArgs a = a0;
   return a.B <= 2 && a.k <= 32 && a.d <= 8192 && a.d_o <= 8192 && plan_small(a, 148, optin);
@@ -765,6 +1246,12 @@ cudaError_t set_small_attributes(size_t optin) {
   SETS((k_experts_f<2, 8>));
   SETS((k_experts_f<1, 0>));
   SETS((k_experts_f<2, 0>));
+  SETS((k_layer_f<1, 4>));
+  SETS((k_layer_f<2, 4>));
+  SETS((k_layer_f<1, 8>));
+  SETS((k_layer_f<2, 8>));
+  SETS((k_layer_f<1, 0>));
+  SETS((k_layer_f<2, 0>));
 #undef SETS
   return e;
 }
@@ -800,6 +1287,18 @@ cudaError_t launch_experts_s(const LayerArgs& a0, int grid, cudaStream_t s, bool
   if (epl == 8)
     return a.B == 1 ? launch_f(k_experts_f<1, 8>, grid, sm, s, pdl, a, true) : launch_f(k_experts_f<2, 8>, grid, sm, s, pdl, a, true);
   return a.B == 1 ? launch_f(k_experts_f<1, 0>, grid, sm, s, pdl, a, true) : launch_f(k_experts_f<2, 0>, grid, sm, s, pdl, a, true);
+}
+
+cudaError_t launch_layer_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
+  LayerArgs a = a0;
+  if (!plan_fused(a, grid, optin)) return cudaErrorInvalidConfiguration;
+  const int epl = a.I / 32;
+  const size_t sm = a.k1.smem;
+  if (epl == 4)
+    return a.B == 1 ? launch_f(k_layer_f<1, 4>, grid, sm, s, pdl, a, true) : launch_f(k_layer_f<2, 4>, grid, sm, s, pdl, a, true);
+  if (epl == 8)
+    return a.B == 1 ? launch_f(k_layer_f<1, 8>, grid, sm, s, pdl, a, true) : launch_f(k_layer_f<2, 8>, grid, sm, s, pdl, a, true);
+  return a.B == 1 ? launch_f(k_layer_f<1, 0>, grid, sm, s, pdl, a, true) : launch_f(k_layer_f<2, 0>, grid, sm, s, pdl, a, true);
 }
 
 }  // namespace moe

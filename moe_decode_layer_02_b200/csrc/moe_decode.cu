@@ -2,14 +2,14 @@
 // capture of the per-layer kernel chain, and the host-buffer variant of the step.
 //
 // A step of n_layers layers is captured once per (batch, buffer addresses) into one
-// CUDA graph: per layer K1 o_proj+residual+RMS stats -> K2 router (+ routing tables above
-// batch 2) -> the expert kernel(s): one fused gate/up + down kernel with per-CTA routing at
-// batch <= 2, separate gate/up and down kernels above, chained with
-// programmatic dependent launch so each kernel's CTAs start (and fetch their static
-// weights) while the previous kernel drains.  With prefetch on, layer l's router kernel
-// also prefetches into L2 what layer l+1 reads first (its router rows, RMSNorm scale and
-// the leading rows of its W_o), in the window where the router, top-k and the first
-// expert bytes leave HBM idle.
+// CUDA graph.  At batch 1 a layer is one cooperative kernel (o_proj + residual + RMS
+// statistics, router, per-CTA routing, gate/up, down + combine, with grid barriers
+// between the phases); at batch 2 it is o_proj -> router -> the small-M expert kernel
+// (per-CTA routing, gate/up, down + combine); above batch 2 it is o_proj -> router +
+// routing tables -> gate/up -> down + combine.  Kernels are chained with programmatic dependent launch so
+// each one's producer fetches its static weights while the previous kernel drains.  With
+// prefetch on, layer l also prefetches into L2 what layer l+1 reads first (its router
+// rows, RMSNorm scale and the leading rows of its W_o).
 //
 // Sources: "vLLM speeds up Kimi K3 up to 1.9x on NVIDIA GB300 with agent-assisted
 // kernels", section "How the specialised decode path works" (kernel choice by batch
@@ -112,12 +112,17 @@ bool use_large(const moe_decode_handle* h, int B) {
 struct Variant {
   bool oproj_small;   // whole-row o_proj (batch <= 2)
   bool experts_small; // small-M gate/up and down with per-CTA routing (batch <= 2)
+  bool fused;         // the three batch <= 2 kernels as one launch
 };
 
 Variant variant_of(const moe_decode_handle* h, const LayerArgs& a) {
   Variant v;
   v.experts_small = !use_large(h, a.B) && small_path_ok(a, h->smem_optin);
   v.oproj_small = v.experts_small && oproj_small_ok(a, h->smem_optin);
+  // One fused launch per layer at batch 1 (measured: on par with the three kernels for one
+  // layer, ahead in stacks); at batch 2 the three kernels are ahead (one token twice: by
+  // ~1.5 us), so they stay.
+  v.fused = v.oproj_small && a.B == 1 && h->cfg.force_variant != 1 && layer_fused_ok(a, h->smem_optin);
   return v;
 }
 
@@ -161,6 +166,11 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     LayerArgs a = layer_args(h, l, B, attn, resid, out, idx, gate);
     const Variant v = variant_of(h, a);
+    if (v.fused) {
+      e = launch_layer_s(a, G, h->cap, l > 0, h->smem_optin);
+      kernels += 1;
+      continue;
+    }
     e = v.oproj_small                         ? launch_oproj_s(a, G, h->cap, l > 0, h->smem_optin)
         : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, h->cap, l > 0)
                                             : launch_oproj(a, G, h->cap, l > 0);
@@ -420,6 +430,8 @@ int moe_decode_sync_status(moe_decode_handle* h, void* stream) {
     return MOE_ERR_CUDA;
   }
   if (word) {
+    // a bounded wait that ran out may leave a grid-barrier count behind
+    cudaMemset(h->ws.counters, 0, sizeof(unsigned) * kNumCounters);
     cudaMemset(h->ws.err, 0, sizeof word);
     cudaDeviceSynchronize();
     return (word & kErrTimeout) ? MOE_ERR_DEVICE_TIMEOUT : MOE_ERR_DEVICE_BOUNDS;
@@ -453,7 +465,8 @@ int moe_decode_kernels_per_step(moe_decode_handle* h, int batch) {
   LayerArgs a = h->plan_base;
   a.B = batch;
   plan_layer(a, h->num_sms, h->smem_optin);
-  const int per_layer = variant_of(h, a).experts_small ? 3 : 4;
+  const Variant v = variant_of(h, a);
+  const int per_layer = v.fused ? 1 : v.experts_small ? 3 : 4;
   return per_layer * L;
 }
 
@@ -485,6 +498,10 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
   for (int l = 0; l < c.n_layers; ++l) {
     LayerArgs a = layer_args(h, l, batch, attn_out, residual_in, out, topk_idx, topk_gate);
     const Variant v = variant_of(h, a);
+    if (v.fused) {
+      timed(6, s, [&](cudaStream_t st) { return launch_layer_s(a, G, st, false, h->smem_optin); });
+      continue;
+    }
     timed(1, s, [&](cudaStream_t st) {
       return v.oproj_small                         ? launch_oproj_s(a, G, st, false, h->smem_optin)
              : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, st, false)

@@ -7,10 +7,11 @@
 //     (it may not fit, and it fragments memory the pool expects to own);
 //   - code that runs under a hard per-process memory cap, where one more allocation can be
 //     the one that fails in the middle of serving.
-// For them this entry point runs the same three kernels as the batch <= 2 path of
-// moe_decode_step (o_proj + residual + RMS statistics, router + top-k, the fused expert
-// kernel), launched directly on the caller's stream, with every intermediate in one
-// file-scope device array of MOE_STATIC_SCRATCH_BYTES.  Nothing is allocated per call: no
+// For them this entry point runs the same kernels as the batch <= 2 path of moe_decode_step
+// (at batch 1 the fused layer kernel: o_proj + residual + RMS statistics, router + top-k,
+// experts; at batch 2 the o_proj, router and small-M expert kernels), launched directly on
+// the caller's stream, with every intermediate in one file-scope device array of
+// MOE_STATIC_SCRATCH_BYTES.  Nothing is allocated per call: no
 // cudaMalloc/cudaFree and no library routine that allocates.  The array is part of the
 // loaded module, so it exists once per device the library runs on.
 //
@@ -19,9 +20,9 @@
 // later calls on that device reuse both.  That first call should come before any stream
 // capture begins.
 //
-// Zero start.  The expert kernel's grid barrier needs its arrival count at zero and the
-// error word must start at zero; every call clears both (one cudaMemsetAsync on the
-// caller's stream) before its kernels run.  Nothing else in the array needs a known value.
+// Zero start.  The grid barriers need their arrival counts at zero and the error word
+// must start at zero; every call clears them (one cudaMemsetAsync on the caller's stream)
+// before its kernels run.  Nothing else in the array needs a known value.
 //
 // Sharing.  Every call on a device uses the same array.  Calls whose executions overlap
 // (issued on different streams, or from different threads without ordering between them)
@@ -196,9 +197,13 @@ int moe_decode_step_static(const moe_decode_config* cfg, const moe_decode_layer_
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(a.ws.counters, 0, sizeof(unsigned) * (kNumCounters + 1), s);
-  if (e == cudaSuccess) e = launch_oproj_s(a, G, s, false, ds.smem_optin);
-  if (e == cudaSuccess) e = launch_router_s(a, G, s, true, ds.smem_optin);
-  if (e == cudaSuccess) e = launch_experts_s(a, G, s, true, ds.smem_optin);
+  if (batch == 1 && layer_fused_ok(a, ds.smem_optin)) {  // the kernels moe_decode_step picks
+    if (e == cudaSuccess) e = launch_layer_s(a, G, s, false, ds.smem_optin);
+  } else {
+    if (e == cudaSuccess) e = launch_oproj_s(a, G, s, false, ds.smem_optin);
+    if (e == cudaSuccess) e = launch_router_s(a, G, s, true, ds.smem_optin);
+    if (e == cudaSuccess) e = launch_experts_s(a, G, s, true, ds.smem_optin);
+  }
   if (e == cudaSuccess && err_word)
     e = cudaMemcpyAsync(err_word, a.ws.err, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s);
   if (e != cudaSuccess) {

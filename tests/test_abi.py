@@ -98,11 +98,19 @@ def test_step_argument_checks():
             md.moe_decode_get_intermediate(h, 9, out, 16)
         md.moe_decode_step(h, 2, attn, res, out)
         assert md.moe_decode_sync_status(h) == 0
-        assert md.moe_decode_kernels_per_step(h, 2) == 3  # small path: o_proj, router, experts
-        assert md.moe_decode_kernels_per_step(h, 4) == 4  # split-K path: o_proj, router, gate/up, down
+        assert md.moe_decode_kernels_per_step(h, 1) == 1  # batch 1: one fused layer kernel
+        assert md.moe_decode_kernels_per_step(h, 2) == 3  # o_proj, router, small-M experts
+        assert md.moe_decode_kernels_per_step(h, 4) == 4  # o_proj, router, gate/up, down
     finally:
         assert md.moe_decode_destroy(h) == 0
     assert md.moe_decode_destroy(h) == md.MOE_ERR_INVALID_ARG  # destroyed twice: rejected
+    for variant, per_b1 in ((1, 3), (2, 4)):  # unfused small-batch kernels; large-batch kernels
+        h = md.moe_decode_create(md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, 4,
+                                           force_variant=variant), w)
+        try:
+            assert md.moe_decode_kernels_per_step(h, 1) == per_b1
+        finally:
+            assert md.moe_decode_destroy(h) == 0
 
 
 @pytest.mark.gpu
