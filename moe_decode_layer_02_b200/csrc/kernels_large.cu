@@ -161,10 +161,15 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
     const int off = tb.uoff[u];
     const int m = min(tb.uoff[u + 1] - off, B);
     float* pb = part + (size_t)(ch & 1) * part_f;
+    const int ng = (m + NT - 1) / NT;  // token groups of this expert
     for (int gu = 0; gu < 2; ++gu, ++it) {
       const int s = it % SA;
       bool waited = false;
-      for (int g0 = 0; g0 < m; g0 += NT) {
+      // Groups in serpentine order (reversed on every other stage), so each stage starts
+      // with the group whose x the previous stage left in registers: ng - 1 reloads per
+      // stage instead of ng.
+      for (int gi = 0; gi < ng; ++gi) {
+        const int g0 = ((it & 1) ? ng - 1 - gi : gi) * NT;
         if (u != cached_u || g0 != cached_g) {  // x of this group's tokens, in registers
 #pragma unroll
           for (int t = 0; t < NT; ++t) {

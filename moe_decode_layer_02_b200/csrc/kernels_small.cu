@@ -513,7 +513,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   pdl_wait();  // logits and x come from the router kernel
   pdl_trigger();
 
-  route_small_cta(a, rt, sc, fb, c == 0);  // barriers inside also publish the ring init
+  // barriers inside also publish the ring init
+  route_small_cta(a.ws.logits, B, a.E, a.k, a.user_idx, a.user_gate, a.ws.err, rt, sc, fb, c == 0);
   // x of every token, in registers (consumers).  Loaded after routing: the loads hit L2 and
   // land before the first weight stage, and holding x across the routing code would spill.
   const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
@@ -939,7 +940,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   }
   __syncthreads();  // the producer warp joins: logits are complete
 
-  route_small_cta(a, rt, sc, fb, c == 0);
+  route_small_cta(a.ws.logits, B, E, a.k, a.user_idx, a.user_gate, a.ws.err, rt, sc, fb, c == 0);
   float xr[NT][kCPLf][8];
   if (warp < kCW) {
 #pragma unroll

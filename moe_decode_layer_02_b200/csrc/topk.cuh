@@ -279,9 +279,10 @@ namespace {
 //     repeated arg-max instead), computes the gates and marks the selection in a bitmap;
 //  5. warp 0 scans the bitmaps (word = lane) and places every entry: its union index and
 //     its position in the (expert, token)-sorted entry list are a scan value plus a popcount.
-__device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch* sc, float* fallback_cand,
-                                bool write_user) {
-  const int B = a.B, E = a.E, K = a.k;
+// Inlined: a separate (non-inlined) function measured twice as slow in the fused kernel.
+__device__ __forceinline__ void route_small_cta(const float* logits, int B, int E, int K, int* user_idx,
+                                             float* user_gate, uint32_t* err, SmallRoute* rt, RouteScratch* sc,
+                                             float* fallback_cand, bool write_user) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int kPer = 2;  // logits per thread per token
   float v[2][kPer];
@@ -292,7 +293,7 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
       const int e = tid + i * kRouteThreads;
       float x = -INFINITY;
       if (t < B && e < E) {
-        x = ld_act(a.ws.logits + (size_t)t * E + e);
+        x = ld_act(logits + (size_t)t * E + e);
         if (x != x) x = -INFINITY;
       }
       v[t][i] = x;
@@ -385,8 +386,7 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
     int my_i = 0;
     if (C > kCandMax) {
       float* cvv = fallback_cand + t * 2 * kCandStride;
-      warp_topk(a.ws.logits + (size_t)t * E, E, K, cvv, reinterpret_cast<int*>(cvv + kCandStride), lane, my_v,
-                my_i);
+      warp_topk(logits + (size_t)t * E, E, K, cvv, reinterpret_cast<int*>(cvv + kCandStride), lane, my_v, my_i);
     } else if (lane < K) {
       my_v = sc->sel_v[t][lane];
       my_i = sc->sel_i[t][lane];
@@ -394,13 +394,13 @@ __device__ void route_small_cta(const LayerArgs& a, SmallRoute* rt, RouteScratch
     const float gte = warp_gate(my_v, lane, K);
     if (lane < K) {
       const int e = (my_i >= 0 && my_i < E) ? my_i : 0;
-      if (e != my_i) atomicOr(a.ws.err, kErrBounds);
+      if (e != my_i) atomicOr(err, kErrBounds);
       rt->idx[t][lane] = e;
       rt->gate[t][lane] = gte;
       atomicOr(&sc->bm[t][e >> 5], 1u << (e & 31));
       if (write_user) {
-        if (a.user_idx) a.user_idx[t * K + lane] = e;
-        if (a.user_gate) a.user_gate[t * K + lane] = gte;
+        if (user_idx) user_idx[t * K + lane] = e;
+        if (user_gate) user_gate[t * K + lane] = gte;
       }
     }
   }
