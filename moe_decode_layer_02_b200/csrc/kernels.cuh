@@ -70,6 +70,10 @@ cudaError_t set_small_attributes(size_t smem_optin);
 cudaError_t launch_oproj_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t launch_router_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t launch_experts_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
+// The router above batch 2 with h staged by TMA (plus the routing tables).
+bool plan_router_big(LayerArgs& a, int grid, size_t smem_optin);
+bool router_big_ok(const LayerArgs& a, size_t smem_optin);
+cudaError_t launch_router_big(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 // The three small-batch kernels fused into one cooperative launch per layer (batch <= 2).
 bool plan_fused(LayerArgs& a, int grid, size_t smem_optin);
 bool layer_fused_ok(const LayerArgs& a, size_t smem_optin);

@@ -312,6 +312,177 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
 }
 
 // =============================================================================
+// Router for batch >= 3: the same arithmetic as k_router_f, with h staged by TMA.
+//   The CTA's W_r slice is one bulk copy issued before the dependency wait (as in
+//   k_router_f).  After it, the producer streams h two tokens at a time (one bulk copy of
+//   2 x d fp32) into a ring, so the consumers never wait on an L2 round trip per token pair:
+//   they turn a stage into x = h * rstd * gamma in registers (releasing the stage at once),
+//   write their share of x, and dot it with the staged router rows.  The partial sums of
+//   consecutive pairs alternate between two buffers.  The last CTA then builds the routing
+//   tables, with the ring as its scratch.
+// =============================================================================
+__global__ void __launch_bounds__(kThreadsS, 1) k_router_big(const LayerArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  constexpr int NT = 2;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int d = a.d, E = a.E, B = a.B;
+  const int RM = a.k2.rows_max, SH = a.k2.stages;
+  long long lo, hi;
+  split_range(E, G, c, lo, hi);
+  const int e0 = (int)lo, nrows = (int)(hi - lo);
+  const uint32_t row_bytes = (uint32_t)d * 2u, hrow_bytes = (uint32_t)d * 4u;
+  const size_t SHB = al128((size_t)NT * hrow_bytes);  // one stage: two tokens of h
+  const size_t region = std::max((size_t)SH * SHB, (size_t)kTopkScratch);
+
+  uint16_t* wsl = reinterpret_cast<uint16_t*>(smem);                                  // [RM][d]
+  unsigned char* ring = smem + al128((size_t)RM * row_bytes);                          // h stages
+  float* part = reinterpret_cast<float*>(ring + region);                               // [2][RM][kCW][NT]
+  float* rstd_s = part + 2 * RM * kCW * NT;                                            // [64]
+  uint64_t* fullW = reinterpret_cast<uint64_t*>(
+      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(rstd_s + 64) - smem)));
+  uint64_t* fullH = fullW + 1;
+  uint64_t* emptyH = fullH + kMaxStages;
+  int* s_misc = reinterpret_cast<int*>(emptyH + kMaxStages);
+  volatile int* abort_flag = s_misc;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  if (tid == 0) {
+    init_ring(fullW, nullptr, 1);
+    init_ring(fullH, emptyH, SH, kCW);
+    s_misc[0] = 0;
+    s_misc[1] = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_trigger();
+
+  const int npairs = (B + NT - 1) / NT;
+  if (warp == kCW) {
+    if (lane == 0) {
+      if (nrows > 0) {
+        mbar_arrive_expect_tx(&fullW[0], nrows * row_bytes);
+        bulk_g2s(wsl, a.w_r + (size_t)e0 * d, nrows * row_bytes, &fullW[0], policy_evict_first());
+      }
+      if (a.pf_w_o) {  // next layer's first reads into L2, as in k_router_f
+        if (nrows > 0) bulk_prefetch_l2(a.pf_w_r + (size_t)e0 * d, nrows * row_bytes);
+        if (c == 0) bulk_prefetch_l2(a.pf_gamma, row_bytes);
+        long long o0, o1;
+        split_range(d, G, c, o0, o1);
+        const size_t orow = (size_t)a.d_o * 2;
+        size_t left = (size_t)min((long long)a.pf_w_o_rows, o1 - o0) * orow;
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(a.pf_w_o + (size_t)o0 * a.d_o);
+        for (size_t off = 0; left > 0;) {
+          const uint32_t n = (uint32_t)min(left, (size_t)65536);
+          bulk_prefetch_l2(src + off, n);
+          off += n;
+          left -= n;
+        }
+      }
+      pdl_wait();  // h comes from the o_proj kernel
+      const uint64_t pol = policy_evict_first();
+      int g = 0;
+      for (; g < npairs; ++g) {
+        const int nt = min(NT, B - g * NT);
+        if (!ring_acquire(emptyH, g, SH, abort_flag, a.ws.err)) break;
+        const int s = g % SH;
+        mbar_arrive_expect_tx(&fullH[s], nt * hrow_bytes);
+        bulk_g2s(ring + s * SHB, a.ws.h + (size_t)g * NT * d, nt * hrow_bytes, &fullH[s], pol);
+      }
+      ring_drain(fullH, g, SH, a.ws.err);
+      if (nrows > 0) mbar_drain(&fullW[0], 0, a.ws.err);
+    }
+  } else {
+    const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
+    float gam[kCPLf][8];
+#pragma unroll
+    for (int j = 0; j < kCPLf; ++j) {
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (cvalid(qpw, j, lane)) u = ld_weight_u4(a.gamma + (size_t)(qbase + j * 32 + lane) * 8);
+      unpack8f(u, gam[j]);
+    }
+    pdl_wait();  // the sums of h^2 come from the o_proj kernel
+    for (int t = warp; t < B; t += kCW) {  // fixed order: same bits in every CTA
+      float ss = 0.f;
+      for (int c0 = 0; c0 < G; c0 += 8 * 32) {
+        float pv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int cc = c0 + k * 32 + lane;
+          pv[k] = cc < G ? ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) ss += pv[k];
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) {
+        const float r = 1.0f / sqrtf(ss / (float)d + a.eps);
+        rstd_s[t] = r;
+        if (c == 0) a.ws.rstd[t] = r;
+      }
+    }
+    csync();
+    if (nrows > 0) mbar_wait(&fullW[0], 0, abort_flag, a.ws.err);
+    for (int g = 0; g < npairs; ++g) {
+      const int t0 = g * NT, nt = min(NT, B - t0), s = g % SH;
+      float* pb = part + (size_t)(g & 1) * RM * kCW * NT;
+      mbar_wait(&fullH[s], (g / SH) & 1, abort_flag, a.ws.err);
+      float xr[NT][kCPLf][8];
+      const float* hs = reinterpret_cast<const float*>(ring + s * SHB);
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const float r = (t < nt) ? rstd_s[t0 + t] : 0.f;
+#pragma unroll
+        for (int j = 0; j < kCPLf; ++j) {
+          const int q = qbase + j * 32 + lane;
+          if (t < nt && cvalid(qpw, j, lane)) {
+            const float4 h0 = *reinterpret_cast<const float4*>(hs + (size_t)t * d + (size_t)q * 8);
+            const float4 h1 = *reinterpret_cast<const float4*>(hs + (size_t)t * d + (size_t)q * 8 + 4);
+            xr[t][j][0] = h0.x; xr[t][j][1] = h0.y; xr[t][j][2] = h0.z; xr[t][j][3] = h0.w;
+            xr[t][j][4] = h1.x; xr[t][j][5] = h1.y; xr[t][j][6] = h1.z; xr[t][j][7] = h1.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xr[t][j][e] = xr[t][j][e] * r * gam[j][e];
+          if (t < nt && cvalid(qpw, j, lane) && q % G == c) {  // each chunk of x is written by one CTA
+            float* xp = a.ws.x + (size_t)(t0 + t) * d + (size_t)q * 8;
+            *reinterpret_cast<float4*>(xp) = make_float4(xr[t][j][0], xr[t][j][1], xr[t][j][2], xr[t][j][3]);
+            *reinterpret_cast<float4*>(xp + 4) = make_float4(xr[t][j][4], xr[t][j][5], xr[t][j][6], xr[t][j][7]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&emptyH[s]);  // h of this pair is in registers now
+      constexpr int kRI = 4 / NT;
+      for (int j0 = 0; j0 < nrows; j0 += kRI) {
+        const uint16_t* rp[kRI];
+#pragma unroll
+        for (int k = 0; k < kRI; ++k) rp[k] = wsl + (size_t)min(j0 + k, nrows - 1) * d;
+        float v[kRI * NT];
+        rows_dot<NT, kRI>(rp, nrows - j0, xr, qbase, qpw, lane, v);
+        const float tot = warp_reduce_multi<kRI * NT>(v, lane);
+        const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
+        if (multi_writer<kRI * NT>(lane) && j < nrows) pb[(j * kCW + warp) * NT + t] = tot;
+      }
+      csync();  // this pair's partials are complete (the next pair writes the other buffer)
+      for (int z = tid; z < nrows * nt; z += kCT) {
+        const int j = z / nt, t = z % nt;
+        float sacc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCW; ++w) sacc += pb[(j * kCW + w) * NT + t];
+        a.ws.logits[(size_t)(t0 + t) * E + e0 + j] = sacc;
+      }
+    }
+  }
+  // the last CTA builds the routing tables; the ring (every fill landed and read) is its scratch
+  if (last_cta_s(&a.ws.counters[kCntRouter], &s_misc[1])) {
+    topk_route(a, ring);
+    if (tid == 0) a.ws.counters[kCntRouter] = 0;
+  }
+}
+
+// =============================================================================
 // Grid barrier for the expert kernel (cooperative launch: every CTA is resident).
 // Each CTA adds one to a counter with release semantics and waits (acquire loads) until it
 // reaches the grid size.  The wait is bounded in time; on expiry the CTA records
@@ -1208,6 +1379,30 @@ bool plan_fused(LayerArgs& a, int G, size_t optin) {
   return o.smem <= budget;
 }
 
+// The TMA-staged router above batch 2: W_r slice, h ring (>= 2 stages of two tokens; also
+// the routing-table builder's scratch), two partial buffers, rstd, barriers.
+bool plan_router_big(LayerArgs& a, int G, size_t optin) {
+  const size_t budget = optin - 1024 - 256;
+  KTune& t = a.k2;
+  t.rows_max = (a.E + G - 1) / G;
+  const size_t w = up128((size_t)t.rows_max * a.d * 2), SHB = up128((size_t)2 * a.d * 4);
+  const size_t tail = up128(((size_t)2 * t.rows_max * kCW * 2 + 64) * 4) + (1 + 2 * kMaxStages) * 8 + 64;
+  t.stages = 0;
+  for (int sh = kMaxStages; sh >= 2; --sh)
+    if (w + std::max((size_t)sh * SHB, (size_t)kTopkScratch) + tail <= budget) {
+      t.stages = sh;
+      break;
+    }
+  if (t.stages < 2) return false;
+  t.smem = w + std::max((size_t)t.stages * SHB, (size_t)kTopkScratch) + tail;
+  return true;
+}
+
+bool router_big_ok(const LayerArgs& a0, size_t optin) {
+  LayerArgs a = a0;
+  return a.B >= 3 && a.B <= 64 && a.d <= 8192 && plan_router_big(a, 148, optin);
+}
+
 bool layer_fused_ok(const LayerArgs& a0, size_t optin) {
   LayerArgs a = a0;
   return a.B <= 2 && a.k <= 32 && a.d <= 8192 && a.d_o <= 8192 && a.E <= 2 * kRouteThreads &&
@@ -1247,6 +1442,7 @@ cudaError_t set_small_attributes(size_t optin) {
   SETS((k_experts_f<2, 8>));
   SETS((k_experts_f<1, 0>));
   SETS((k_experts_f<2, 0>));
+  SETS(k_router_big);
   SETS((k_layer_f<1, 4>));
   SETS((k_layer_f<2, 4>));
   SETS((k_layer_f<1, 8>));
@@ -1300,6 +1496,12 @@ cudaError_t launch_layer_s(const LayerArgs& a0, int grid, cudaStream_t s, bool p
   if (epl == 8)
     return a.B == 1 ? launch_f(k_layer_f<1, 8>, grid, sm, s, pdl, a, true) : launch_f(k_layer_f<2, 8>, grid, sm, s, pdl, a, true);
   return a.B == 1 ? launch_f(k_layer_f<1, 0>, grid, sm, s, pdl, a, true) : launch_f(k_layer_f<2, 0>, grid, sm, s, pdl, a, true);
+}
+
+cudaError_t launch_router_big(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
+  LayerArgs a = a0;
+  if (!plan_router_big(a, grid, optin)) return cudaErrorInvalidConfiguration;
+  return launch_f(k_router_big, grid, a.k2.smem, s, pdl, a);
 }
 
 }  // namespace moe

@@ -174,7 +174,9 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
     e = v.oproj_small                         ? launch_oproj_s(a, G, h->cap, l > 0, h->smem_optin)
         : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, h->cap, l > 0)
                                             : launch_oproj(a, G, h->cap, l > 0);
-    if (e == cudaSuccess) e = launch_router_s(a, G, h->cap, true, h->smem_optin);
+    if (e == cudaSuccess)
+      e = (!v.experts_small && router_big_ok(a, h->smem_optin)) ? launch_router_big(a, G, h->cap, true, h->smem_optin)
+                                                                : launch_router_s(a, G, h->cap, true, h->smem_optin);
     kernels += 2;
     if (v.experts_small) {
       if (e == cudaSuccess) e = launch_experts_s(a, G, h->cap, true, h->smem_optin);
@@ -507,7 +509,10 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
              : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, st, false)
                                                  : launch_oproj(a, G, st, false);
     });
-    timed(2, s, [&](cudaStream_t st) { return launch_router_s(a, G, st, false, h->smem_optin); });
+    timed(2, s, [&](cudaStream_t st) {
+      return (!v.experts_small && router_big_ok(a, h->smem_optin)) ? launch_router_big(a, G, st, false, h->smem_optin)
+                                                                   : launch_router_s(a, G, st, false, h->smem_optin);
+    });
     if (v.experts_small) {
       timed(3, s, [&](cudaStream_t st) { return launch_experts_s(a, G, st, false, h->smem_optin); });
     } else {
