@@ -169,14 +169,31 @@ def weight_bytes(dims, n_union_per_layer):
     return sum(d * do * 2 + d * 2 + E * d * 2 + u * (2 * I * d * 2 + d * I * 2) for u in n_union_per_layer)
 
 
-def kernels_sha():
-    """Hash of the kernel sources: ncu traffic figures are valid only for the code they were taken on."""
+def code_only(text):
+    """C++ source without comments or blank lines (string literals left as they are)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = []
+    for line in text.splitlines():
+        i = line.find("//")
+        if i >= 0 and line.count('"', 0, i) % 2 == 0:
+            line = line[:i]
+        line = line.rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
+def kernels_sha(kernel_dir=None):
+    """Hash of the kernel code (comments ignored): ncu traffic figures are valid only for the
+    code they were taken on."""
     import hashlib
+    kdir = kernel_dir or KERNEL_DIR
     hs = hashlib.sha256()
-    for f in sorted(os.listdir(KERNEL_DIR)):
+    for f in sorted(os.listdir(kdir)):
         if f.endswith((".cu", ".cuh")):
             hs.update(f.encode())
-            hs.update(open(os.path.join(KERNEL_DIR, f), "rb").read())
+            hs.update(code_only(open(os.path.join(kdir, f), encoding="utf-8").read()).encode())
     return hs.hexdigest()[:16]
 
 

@@ -1,7 +1,8 @@
 // sm_100a kernels of one MoE decode-layer step.
 //
-// The large-batch o_proj (the small-batch kernels and the router are in kernels_small.cu,
-// the large-batch expert kernels in kernels_large.cu):
+// The fallback large-batch o_proj, used above batch 2 where the TMA tensor maps of
+// k_oproj_tc (kernels_tc.cu) cannot be encoded (the small-batch kernels and the router are
+// in kernels_small.cu, the large-batch expert kernels in kernels_large.cu):
 //   K1 k_oproj           h = residual + W_o . attn_out on the tensor cores (weights as the
 //                        MMA's N operand, staged through a shared-memory ring by TMA bulk
 //                        copies), tokens in groups of up to 8, per-CTA sums of h^2.

@@ -11,13 +11,17 @@
 //     as fp32 (exact; x is not rounded for the router), reads 16-byte weight chunks from
 //     shared memory (lanes contiguous, conflict-free) and accumulates in fp32;
 //   * row partials go to shared memory and are reduced once, in a fixed order, at the end.
-// No grid-wide synchronisation: RMSNorm statistics are per-CTA partial sums that the router
-// reduces itself, and the top-k selection and routing are recomputed in every expert CTA.
+// RMSNorm statistics are per-CTA partial sums that every router CTA reduces itself in the
+// same order, and the top-k selection and routing are recomputed in every expert CTA.
 //
-//   k_oproj_f    h = residual + W_o . attn_out, per-CTA sums of h^2            (batch <= 2)
-//   k_router_f   rstd, x = h * rstd * gamma, logits = W_r . x   (any batch; at batch >= 3
-//                the last CTA also builds the global routing tables)
-//   k_experts_f  the expert kernel (batch <= 2): routing once per CTA; gate/up + SiLU*mul
+//   k_layer_f    batch 1: the whole layer step as one cooperative launch (the three kernels
+//                below as phases, with grid barriers where the kernel boundaries were)
+//   k_oproj_f    h = residual + W_o . attn_out, per-CTA sums of h^2                (batch 2)
+//   k_router_f   rstd, x = h * rstd * gamma, logits = W_r . x   (batch 2; above batch 2
+//                where k_router_big does not fit, its last CTA also building the global
+//                routing tables)
+//   k_router_big the router above batch 2, h staged by TMA, plus the routing tables
+//   k_experts_f  the expert kernel (batch 2): routing once per CTA; gate/up + SiLU*mul
 //                for each (selected expert, row pair), each pair streamed once; a grid
 //                barrier; then out = bf16(h + sum_j gate_j * W_down[e_j] . a_j), with W_down
 //                streaming into the freed ring while the barrier is open
