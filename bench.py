@@ -52,6 +52,8 @@ WORKLOADS = {
     "tp16e64_b2": ("TP16E64", 2, 1, "indep"),
     "tp8e64_b64": ("TP8E64", 64, 1, "indep"),
     "tp8e224k4_b16": ("TP8E224K4", 16, 1, "indep"),
+    # profiling case for the next-layer prefetch: two such layers (~1.2 GB on the device)
+    "stack2e64_b1": ("TP16E64", 1, 2, "indep"),
 }
 
 KERNEL_DIR = os.path.join(ROOT, "moe_decode_layer_02_b200", "csrc")
