@@ -186,6 +186,21 @@ def code_only(text):
     return "\n".join(out)
 
 
+def max_over_ranks(x, world, device):
+    """The largest per-rank value over all ranks (a multi-GPU job's time is its slowest rank's)."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_us_per_layer_step(t_max_ms, world, steps, layers):
+    """Whole-job figure: N replicas each run `steps` steps of `layers` layers in t_max_ms."""
+    return t_max_ms * 1000.0 / (world * steps * layers)
+
+
 def kernels_sha(kernel_dir=None):
     """Hash of the kernel code (comments ignored): ncu traffic figures are valid only for the
     code they were taken on."""
@@ -302,10 +317,7 @@ def run_ours(args, rank, world):
     rc = max(abs(md.moe_decode_sync_status(x, s)) for x in hs)
     if rc:
         raise RuntimeError(md.strerror(-rc))
-    tot = torch.tensor([sum(step_ms)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
-    t_max_ms = float(tot.item())
+    t_max_ms = max_over_ranks(sum(step_ms), world, "cuda")
 
     # ---- secondary: the same weights back to back (warm L2), and a 256 MiB L2 flush before each
     # step instead of the rotation (the flush leaves dirty lines whose write-back lands inside
@@ -452,7 +464,7 @@ def main():
     hbm, bf16, src = peaks()
     dims = r["dims"]
     K = args.steps
-    us_per_layer = r["t_max_ms"] * 1000 / (world * K * L)
+    us_per_layer = job_us_per_layer_step(r["t_max_ms"], world, K, L)
     wbytes = weight_bytes(dims, r["n_union"]) / r["R"]  # n_union holds R copies x L layers
     per_step_ms = r["t_max_ms"] / K
     gbs = wbytes / (per_step_ms * 1e-3) / 1e9
