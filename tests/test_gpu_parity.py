@@ -108,6 +108,25 @@ def test_ragged_shapes(B):
         st.close()
 
 
+# --- the largest shapes the library accepts, one dimension at a time -----------------------
+#   d = d_o = 8192 with k = 32 and I = 512 (64 experts keep the weights at ~1.2 GB), and
+#   E = 1024 with k = 32 on d = 1024 (large enough a logit spread for gapped draws).  Batch 1 (the fused kernel, or the large-batch kernels
+#   where its shared memory does not fit), 2 and 64.
+@pytest.mark.slow
+@pytest.mark.parametrize("B", [1, 2, 64])
+@pytest.mark.parametrize("dims", [synth.Dims(8192, 8192, 64, 32, 512), synth.Dims(1024, 256, 1024, 32, 32)],
+                         ids=["d8192_k32_I512", "E1024_k32"])
+def test_maximum_sizes(dims, B):
+    seed = synth.config_seed(13) + B + dims.E
+    st = H.GpuStack(seed, dims, max_batch=64)
+    try:
+        sampled = [0] if B == 1 else [0, B - 1]
+        case = build_case(seed, dims, B, checked=sampled, moe_tokens=sampled)
+        check_case(st, case, sampled=sampled)
+    finally:
+        st.close()
+
+
 @pytest.mark.parametrize("B", [1, 3])
 def test_degenerate_k_equals_e_and_k1(B):
     for dims in (synth.Dims(128, 64, 4, 4, 32), synth.Dims(128, 128, 8, 1, 64)):
