@@ -56,8 +56,11 @@ struct moe_decode_handle {
   Workspace ws{};
   void* ws_base = nullptr;
   uint16_t* resid_pp[2] = {nullptr, nullptr};
-  // staging for moe_decode_step_host
-  void *h_attn = nullptr, *h_resid = nullptr, *h_out = nullptr, *h_idx = nullptr, *h_gate = nullptr;
+  // staging for moe_decode_step_host: device buffers for a step's inputs and outputs, each
+  // group contiguous, and pinned host mirrors of them, so a step moves one copy each way
+  void *h_in = nullptr, *h_outs = nullptr;      // device: inputs, outputs
+  void *pin_in = nullptr, *pin_out = nullptr;   // pinned host mirrors
+  size_t in_bytes = 0, out_bytes = 0;           // capacities (max_batch)
   LayerArgs plan_base{};
   cudaStream_t cap = nullptr;
   std::vector<GraphEntry> graphs;
@@ -376,46 +379,56 @@ int moe_decode_step_host(moe_decode_handle* h, int batch, const void* attn_out_h
   if (!attn_out_host || !residual_in_host || !out_host) return MOE_ERR_INVALID_ARG;
   const moe_decode_config& c = h->cfg;
   const size_t maxB = c.max_batch;
-  if (!h->h_attn) {
-    size_t sz = up256(2ull * c.n_layers * maxB * c.d_o) + 2 * up256(2ull * maxB * c.d) +
-                2 * up256(4ull * c.n_layers * maxB * c.top_k);
-    void* p = nullptr;
-    if (cudaMalloc(&p, sz) != cudaSuccess) {
-      cudaGetLastError();
-      return MOE_ERR_OOM;
-    }
-    char* b = static_cast<char*>(p);
-    h->h_attn = b;
-    b += up256(2ull * c.n_layers * maxB * c.d_o);
-    h->h_resid = b;
-    b += up256(2ull * maxB * c.d);
-    h->h_out = b;
-    b += up256(2ull * maxB * c.d);
-    h->h_idx = b;
-    b += up256(4ull * c.n_layers * maxB * c.top_k);
-    h->h_gate = b;
-  }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Layout for `batch` tokens: inputs [attn_out | residual_in], outputs [out | idx | gate],
+  // each part starting on a 256-byte boundary.
   const size_t n_attn = 2ull * c.n_layers * batch * c.d_o, n_res = 2ull * batch * c.d,
                n_tk = 4ull * c.n_layers * batch * c.top_k;
-  cudaError_t e = cudaMemcpyAsync(h->h_attn, attn_out_host, n_attn, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(h->h_resid, residual_in_host, n_res, cudaMemcpyHostToDevice, s);
+  const size_t o_res = up256(n_attn), in_used = o_res + n_res;
+  const size_t o_idx = up256(n_res), o_gate = o_idx + up256(n_tk);
+  const size_t out_used = (topk_gate_host ? o_gate + n_tk : topk_idx_host ? o_idx + n_tk : n_res);
+  if (!h->h_in) {
+    h->in_bytes = up256(2ull * c.n_layers * maxB * c.d_o) + up256(2ull * maxB * c.d);
+    h->out_bytes = up256(2ull * maxB * c.d) + 2 * up256(4ull * c.n_layers * maxB * c.top_k);
+    void *di = nullptr, *dout = nullptr, *pi = nullptr, *po = nullptr;
+    if (cudaMalloc(&di, h->in_bytes) != cudaSuccess || cudaMalloc(&dout, h->out_bytes) != cudaSuccess ||
+        cudaHostAlloc(&pi, h->in_bytes, cudaHostAllocDefault) != cudaSuccess ||
+        cudaHostAlloc(&po, h->out_bytes, cudaHostAllocDefault) != cudaSuccess) {
+      cudaGetLastError();
+      if (di) cudaFree(di);
+      if (dout) cudaFree(dout);
+      if (pi) cudaFreeHost(pi);
+      if (po) cudaFreeHost(po);
+      return MOE_ERR_OOM;
+    }
+    h->h_in = di;
+    h->h_outs = dout;
+    h->pin_in = pi;
+    h->pin_out = po;
+  }
+  char* din = static_cast<char*>(h->h_in);
+  char* dout = static_cast<char*>(h->h_outs);
+  char* pin = static_cast<char*>(h->pin_in);
+  char* pout = static_cast<char*>(h->pin_out);
+  std::memcpy(pin, attn_out_host, n_attn);
+  std::memcpy(pin + o_res, residual_in_host, n_res);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(din, pin, in_used, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
-  int rc = moe_decode_step(h, batch, h->h_attn, h->h_resid, h->h_out, topk_idx_host ? (int32_t*)h->h_idx : nullptr,
-                           topk_gate_host ? (float*)h->h_gate : nullptr, stream);
+  int rc = moe_decode_step(h, batch, din, din + o_res, dout, topk_idx_host ? (int32_t*)(dout + o_idx) : nullptr,
+                           topk_gate_host ? (float*)(dout + o_gate) : nullptr, stream);
   if (rc) return rc;
-  e = cudaMemcpyAsync(out_host, h->h_out, n_res, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess && topk_idx_host) e = cudaMemcpyAsync(topk_idx_host, h->h_idx, n_tk, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess && topk_gate_host)
-    e = cudaMemcpyAsync(topk_gate_host, h->h_gate, n_tk, cudaMemcpyDeviceToHost, s);
+  e = cudaMemcpyAsync(pout, dout, out_used, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
+  std::memcpy(out_host, pout, n_res);
+  if (topk_idx_host) std::memcpy(topk_idx_host, pout + o_idx, n_tk);
+  if (topk_gate_host) std::memcpy(topk_gate_host, pout + o_gate, n_tk);
   return MOE_OK;
 }
 
@@ -540,7 +553,10 @@ int moe_decode_destroy(moe_decode_handle* h) {
   }
   cudaDeviceSynchronize();
   release(h);
-  if (h->h_attn) cudaFree(h->h_attn);
+  if (h->h_in) cudaFree(h->h_in);
+  if (h->h_outs) cudaFree(h->h_outs);
+  if (h->pin_in) cudaFreeHost(h->pin_in);
+  if (h->pin_out) cudaFreeHost(h->pin_out);
   h->poisoned = true;
   delete h;
   return MOE_OK;

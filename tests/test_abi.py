@@ -133,5 +133,12 @@ def test_host_buffer_step_matches_device_step():
         st.md.moe_decode_step_host(st.h, 3, np.ascontiguousarray(case["attn"]), np.ascontiguousarray(case["resid"]),
                                    out_h, idx_h, gate_h)
         assert np.array_equal(out_h, out_d) and np.array_equal(idx_h, idx_d) and np.array_equal(gate_h, gate_d)
+        # another batch, outputs only (no top-k buffers), into unpinned numpy memory
+        case1 = build_case(seed + 1, synth.TINY, 1, checked=[0])
+        out1_d, _, _ = st.step(case1["attn"], case1["resid"])
+        out1_h = np.zeros((1, synth.TINY.d), np.uint16)
+        st.md.moe_decode_step_host(st.h, 1, np.ascontiguousarray(case1["attn"]),
+                                   np.ascontiguousarray(case1["resid"]), out1_h)
+        assert np.array_equal(out1_h, out1_d)
     finally:
         st.close()
