@@ -145,6 +145,20 @@ MOE_API int moe_decode_step_host(moe_decode_handle* h, int batch, const void* at
  * MOE_ERR_CUDA on a CUDA error, else MOE_OK. */
 MOE_API int moe_decode_sync_status(moe_decode_handle* h, void* stream);
 
+/* Makes the device error reporting run, without a fault, so that callers and tests can
+ * check their handling of it.  Launches on `stream` one small kernel that uses the same
+ * bounded-wait and index-check code as the step's kernels:
+ *   what = 1  an mbarrier wait that nothing completes and a grid barrier that one arrival
+ *             short can never open, each giving up after limit_ns nanoseconds; the next
+ *             moe_decode_sync_status returns MOE_ERR_DEVICE_TIMEOUT;
+ *   what = 2  an expert index one past the end, clamped and skipped; the next
+ *             moe_decode_sync_status returns MOE_ERR_DEVICE_BOUNDS.
+ * 0 < limit_ns <= 10,000,000 (10 ms); anything else is MOE_ERR_INVALID_ARG.  The record
+ * stays in the handle's error word until moe_decode_sync_status reads and clears it; steps
+ * in between run normally.  Returns MOE_OK once launched, MOE_ERR_CUDA if the launch fails. */
+MOE_API int moe_decode_check_error_path(moe_decode_handle* h, int what, unsigned long long limit_ns,
+                                        void* stream);
+
 /* Intermediates of the most recent step's LAST layer, for tests:
  *   which = 0  h      [batch][d]          fp32
  *           1  rstd   [batch]             fp32
@@ -181,8 +195,10 @@ MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void*
  * It runs the same kernels as moe_decode_step's batch <= 2 path, launched directly on
  * `stream` (no graph, no handle), with every intermediate in one static device array of
  * MOE_STATIC_SCRATCH_BYTES that is part of the loaded library (one per device).
- *   cfg          layer shapes as for moe_decode_create (host); n_layers must be 1 and
- *                force_variant 0 or 1; enable_prefetch is ignored
+ *   cfg          layer shapes as for moe_decode_create (host, checked against the same
+ *                supported set); n_layers must be 1 and force_variant 0 or 1 (1: the three
+ *                small-batch kernels at batch 1 too, as in moe_decode_step); enable_prefetch
+ *                is ignored
  *   w            the layer's weights (host struct of device pointers, as for create)
  *   batch        1 or 2, and <= cfg->max_batch
  *   attn_out     [batch][d_o] bf16, residual_in [batch][d] bf16, out [batch][d] bf16 (device)

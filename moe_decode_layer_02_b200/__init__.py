@@ -27,7 +27,8 @@ MOE_STATIC_SCRATCH_BYTES = 256 * 1024
 
 EXPORTED = ("moe_decode_create", "moe_decode_step", "moe_decode_step_host", "moe_decode_sync_status",
             "moe_decode_get_intermediate", "moe_decode_kernels_per_step", "moe_decode_profile_step",
-            "moe_decode_step_static", "moe_decode_destroy", "moe_decode_strerror")
+            "moe_decode_step_static", "moe_decode_check_error_path", "moe_decode_destroy",
+            "moe_decode_strerror")
 
 KERNEL_NAMES = {1: "oproj_residual_rmsnorm", 2: "router_topk", 3: "experts_small_m", 4: "gateup_rows",
                 5: "down_rows", 6: "layer_fused_small_m"}
@@ -74,6 +75,7 @@ def load(path: str = LIB_PATH):
     lib.moe_decode_profile_step.argtypes = [P, I, P, P, P, P, P, P, P, P, I]
     lib.moe_decode_step_static.argtypes = [ctypes.POINTER(moe_decode_config),
                                            ctypes.POINTER(moe_decode_layer_weights), I, P, P, P, P, P, P, P]
+    lib.moe_decode_check_error_path.argtypes = [P, I, ctypes.c_ulonglong, P]
     lib.moe_decode_destroy.argtypes = [P]
     lib.moe_decode_strerror.argtypes = [I]
     lib.moe_decode_strerror.restype = ctypes.c_char_p
@@ -178,6 +180,11 @@ def moe_decode_step_static(cfg: moe_decode_config, weights, batch: int, attn_out
     _check(load().moe_decode_step_static(ctypes.byref(cfg), ctypes.byref(w), batch, _addr(attn_out),
                                          _addr(residual_in), _addr(out), _addr(topk_idx), _addr(topk_gate),
                                          _addr(err_word), _stream(stream)), "moe_decode_step_static")
+
+
+def moe_decode_check_error_path(h: int, what: int, limit_ns: int = 1_000_000, stream=None) -> None:
+    """Launches the error-path probe (1: bounded waits run out; 2: an out-of-range index)."""
+    _check(load().moe_decode_check_error_path(h, what, limit_ns, _stream(stream)), "moe_decode_check_error_path")
 
 
 def moe_decode_destroy(h: int) -> int:

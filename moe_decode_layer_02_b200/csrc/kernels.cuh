@@ -3,11 +3,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/moe_decode.h"
+
 namespace moe {
+
+// The supported set of the C ABI (moe_decode.cu): MOE_OK or the MOE_ERR_* code create returns.
+int check_config(const moe_decode_config* c);
 
 // Device counters: fused layer kernel's exit ticket, router ticket, expert-kernel grid
 // barrier count, fused layer kernel's grid barrier count.  All are zero between launches.
-enum Counter { kCntLayerExit = 0, kCntRouter = 1, kCntGateUp = 2, kCntLayer = 3, kNumCounters = 4 };
+// kCntProbe: the error-path probe's grid-barrier count.
+enum Counter { kCntLayerExit = 0, kCntRouter = 1, kCntGateUp = 2, kCntLayer = 3, kCntProbe = 4, kNumCounters = 5 };
 
 // Library-owned device workspace (one per handle).
 struct Workspace {
@@ -79,6 +85,9 @@ bool plan_fused(LayerArgs& a, int grid, size_t smem_optin);
 bool layer_fused_ok(const LayerArgs& a, size_t smem_optin);
 cudaError_t launch_layer_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t set_kernel_attributes(size_t smem_optin);
+// The error-path probe (what 1: bounded waits run out; 2: an out-of-range index is clamped).
+cudaError_t launch_error_probe(unsigned* count, unsigned* err, int what, unsigned long long limit_ns, int E,
+                               int* sink, cudaStream_t s);
 
 // o_proj above batch 2 on the tensor cores with 2-D TMA tiles (kernels_tc.cu).
 bool oproj_tc_ok(const LayerArgs& a, int grid, size_t smem_optin);

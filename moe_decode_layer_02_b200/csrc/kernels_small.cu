@@ -510,7 +510,8 @@ __device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
 // the release (no second round trip).  Who clears it: for the expert kernel, the router
 // kernel before its dependents pass their dependency wait; for the fused layer kernel, its
 // own last CTA to finish (layer_exit).
-__device__ void grid_barrier(unsigned* count, unsigned target, volatile int* abort_flag, uint32_t* err) {
+__device__ void grid_barrier(unsigned* count, unsigned target, volatile int* abort_flag, uint32_t* err,
+                             unsigned long long limit_ns = kWaitLimitNs) {
   // The CTA's writes happen before thread 0's release add: bar.sync orders them before it
   // and the release is cumulative, so no separate fence is needed.
   csync();
@@ -519,7 +520,7 @@ __device__ void grid_barrier(unsigned* count, unsigned target, volatile int* abo
     if (ld_acquire_u32(count) < target) {
       const unsigned long long t0 = globaltimer();
       while (ld_acquire_u32(count) < target) {
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
           *abort_flag = 1;
           atomicOr(err, kErrTimeout);
           break;
@@ -1250,6 +1251,50 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   }
   csync();
   combine_down<NT, EPL>(a, ring, SB_B, SBn, fullB, emptyB, abort_flag, a_s, U, i0, nrows, warp, lane);
+}
+
+// =============================================================================
+// Error-path probe (moe_decode_check_error_path): makes the device error reporting of the
+// kernels above run without a fault.
+//   what 1: thread 0 waits on an mbarrier that nothing arrives on (mbar_wait), then every
+//           CTA waits at a grid barrier whose target is one arrival more than the grid
+//           (grid_barrier); both waits run out after limit_ns and record kErrTimeout.  Each
+//           CTA then takes its own arrival back, so the counter ends at zero.
+//   what 2: an expert index one past the end is met and clamped, recording kErrBounds, the
+//           way the routing and the expert kernels treat an out-of-range table entry.
+// Nothing is copied asynchronously, so no copy can still be in flight when a CTA exits.
+// =============================================================================
+__global__ void __launch_bounds__(kThreadsS, 1) k_error_probe(unsigned* count, uint32_t* err, int what,
+                                                              unsigned long long limit_ns, int E, int* sink) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_s;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (what == 1) {
+    if (threadIdx.x == 0) {
+      mbar_wait(&bar, 0, &abort_s, err, limit_ns);
+      abort_s = 0;  // the grid barrier below must still run out on its own
+    }
+    __syncthreads();
+    if (warp < kCW) grid_barrier(count, gridDim.x + 1u, &abort_s, err, limit_ns);
+    if (threadIdx.x == 0) atomicSub(count, 1u);
+  } else if (what == 2 && threadIdx.x == 0 && blockIdx.x == 0) {
+    const int want = E;  // one past the last expert
+    const int e = (want >= 0 && want < E) ? want : 0;
+    if (e != want) atomicOr(err, kErrBounds);
+    *sink = e;
+  }
+}
+
+cudaError_t launch_error_probe(unsigned* count, unsigned* err, int what, unsigned long long limit_ns, int E,
+                               int* sink, cudaStream_t s) {
+  k_error_probe<<<2, kThreadsS, 0, s>>>(count, err, what, limit_ns, E, sink);
+  return cudaGetLastError();
 }
 
 // =============================================================================

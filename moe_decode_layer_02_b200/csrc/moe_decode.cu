@@ -81,19 +81,6 @@ bool is_live(const moe_decode_handle* h) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_cfg(const moe_decode_config* c) {
-  if (c->d < 64 || c->d > 8192 || c->d % 64) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c->d_o < 64 || c->d_o > 8192 || c->d_o % 64) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c->top_k < 1 || c->top_k > 32) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c->n_experts < c->top_k || c->n_experts > 1024) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c->inter < 32 || c->inter > 512 || c->inter % 32) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c->max_batch < 1 || c->max_batch > 64) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c->n_layers < 1 || c->n_layers > 64) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (!(c->rms_eps > 0.f)) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c->force_variant < 0 || c->force_variant > 2) return MOE_ERR_INVALID_ARG;
-  return MOE_OK;
-}
-
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 void release(moe_decode_handle* h) {
@@ -229,6 +216,21 @@ int get_graph(moe_decode_handle* h, int B, const void* attn, const void* resid, 
 
 }  // namespace
 
+// Validation shared by moe_decode_create and moe_decode_step_static: the supported set of
+// include/moe_decode.h (shapes, batch and layer limits, eps, force_variant).
+int moe::check_config(const moe_decode_config* c) {
+  if (c->d < 64 || c->d > 8192 || c->d % 64) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->d_o < 64 || c->d_o > 8192 || c->d_o % 64) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->top_k < 1 || c->top_k > 32) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->n_experts < c->top_k || c->n_experts > 1024) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->inter < 32 || c->inter > 512 || c->inter % 32) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->max_batch < 1 || c->max_batch > 64) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->n_layers < 1 || c->n_layers > 64) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (!(c->rms_eps > 0.f)) return MOE_ERR_UNSUPPORTED_CONFIG;
+  if (c->force_variant < 0 || c->force_variant > 2) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
 extern "C" {
 
 int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weights* weights, void* stream,
@@ -236,7 +238,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   if (!out) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg || !weights) return MOE_ERR_INVALID_ARG;
-  int rc = check_cfg(cfg);
+  int rc = check_config(cfg);
   if (rc) return rc;
   for (int l = 0; l < cfg->n_layers; ++l) {
     const moe_decode_layer_weights& w = weights[l];
@@ -450,6 +452,20 @@ int moe_decode_sync_status(moe_decode_handle* h, void* stream) {
     cudaMemset(h->ws.err, 0, sizeof word);
     cudaDeviceSynchronize();
     return (word & kErrTimeout) ? MOE_ERR_DEVICE_TIMEOUT : MOE_ERR_DEVICE_BOUNDS;
+  }
+  return MOE_OK;
+}
+
+int moe_decode_check_error_path(moe_decode_handle* h, int what, unsigned long long limit_ns, void* stream) {
+  if (!h || !is_live(h) || h->poisoned) return MOE_ERR_INVALID_ARG;
+  if ((what != 1 && what != 2) || limit_ns == 0 || limit_ns > 10000000ull) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MOE_ERR_INVALID_ARG;
+  // the probe's sink is n_union, which every step rewrites before anything reads it
+  if (launch_error_probe(&h->ws.counters[kCntProbe], h->ws.err, what, limit_ns, h->cfg.n_experts, h->ws.n_union,
+                         static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }

@@ -143,12 +143,8 @@ int moe_decode_step_static(const moe_decode_config* cfg, const moe_decode_layer_
                            float* topk_gate, uint32_t* err_word, void* stream) {
   if (!cfg || !w || !attn_out || !residual_in || !out) return MOE_ERR_INVALID_ARG;
   const moe_decode_config& c = *cfg;
-  if (c.d < 64 || c.d > 8192 || c.d % 64) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c.d_o < 64 || c.d_o > 8192 || c.d_o % 64) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c.top_k < 1 || c.top_k > 32) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c.n_experts < c.top_k || c.n_experts > 1024) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c.inter < 32 || c.inter > 512 || c.inter % 32) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (!(c.rms_eps > 0.f)) return MOE_ERR_UNSUPPORTED_CONFIG;
+  const int rc_cfg = check_config(cfg);  // the supported set of moe_decode_create
+  if (rc_cfg) return rc_cfg;
   if (c.n_layers != 1 || c.force_variant == 2) return MOE_ERR_UNSUPPORTED_CONFIG;  // one layer, small path
   if (batch < 1 || batch > 2 || batch > c.max_batch) return MOE_ERR_INVALID_ARG;
   if (!w->w_o || !w->gamma || !w->w_router || !w->w_gate_up || !w->w_down) return MOE_ERR_INVALID_ARG;
@@ -197,7 +193,9 @@ int moe_decode_step_static(const moe_decode_config* cfg, const moe_decode_layer_
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(a.ws.counters, 0, sizeof(unsigned) * (kNumCounters + 1), s);
-  if (batch == 1 && layer_fused_ok(a, ds.smem_optin)) {  // the kernels moe_decode_step picks
+  // the kernels moe_decode_step picks: the fused layer kernel at batch 1 unless force_variant 1
+  // asks for the three small-batch kernels
+  if (batch == 1 && c.force_variant != 1 && layer_fused_ok(a, ds.smem_optin)) {
     if (e == cudaSuccess) e = launch_layer_s(a, G, s, false, ds.smem_optin);
   } else {
     if (e == cudaSuccess) e = launch_oproj_s(a, G, s, false, ds.smem_optin);

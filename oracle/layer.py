@@ -2,7 +2,8 @@
 
 TEST INFRASTRUCTURE ONLY (tests, smoke check, the benchmark's CPU-baseline
 leg).  Weights are regenerated on the host from the seeded generator; an
-expert's weights are materialised only when a checked token selects it.
+expert's weights are materialised only when a checked token selects it, and for a
+whole batch they are taken one expert at a time (``LayerRef.moe_many``).
 
 Gap rule.  The selected expert indices must match the CUDA path exactly, so
 inputs are drawn such that, for every checked token and layer, every adjacent
@@ -25,6 +26,16 @@ def top_gap(logits_row: np.ndarray, k: int) -> float:
     """Smallest adjacent gap among the k+1 largest values of one row."""
     s = np.sort(np.asarray(logits_row, np.float64))[::-1][: k + 1]
     return float(np.min(s[:-1] - s[1:])) if s.size > 1 else np.inf
+
+
+def top_gap_distinct(logits_row: np.ndarray, k: int) -> float:
+    """Smallest gap between adjacent DISTINCT values among the k+1 largest of one row, and
+    0 when the k-th and (k+1)-th largest are equal (the selected set is then not unique)."""
+    s = np.sort(np.asarray(logits_row, np.float64))[::-1][: k + 1]
+    if s.size > k and s[k - 1] == s[k]:
+        return 0.0
+    u = np.unique(s)
+    return float(np.min(np.diff(u))) if u.size > 1 else np.inf
 
 
 def boundary_gap(logits_row: np.ndarray, k: int) -> float:
@@ -59,6 +70,34 @@ class LayerRef:
         gus, dns = zip(*[self.expert(e) for e in sel])
         return self.o.moe_token(list(gus), list(dns), f["x"][b], f["h"][b], f["gate"][b], self.dims.I)
 
+    def moe_many(self, fronts: dict) -> dict:
+        """Steps 5-6 for many tokens, expert by expert.
+
+        ``fronts`` maps a token to its one-token front result.  Each selected expert's
+        weights are generated once, applied to every token that selected it and dropped,
+        so host memory stays bounded at any batch.  The arithmetic is the oracle's own
+        per-token path (oracle_expert for each selected slot, then oracle_combine over the
+        slots in ascending order), only the loop that materialises the weights differs.
+        Returns token -> (out_ref, out_bf16, a [k][I])."""
+        D = self.dims
+        users: dict[int, list] = {}
+        for b, f in fronts.items():
+            for j, e in enumerate(f["idx"][0]):
+                users.setdefault(int(e), []).append((b, j))
+        ys = {b: [None] * D.k for b in fronts}
+        acts = {b: np.empty((D.k, D.I)) for b in fronts}
+        for e in sorted(users):
+            gu, dn = self._experts.get(e) or synth.host_expert(self.seed, D, e, self.layer)
+            for b, j in users[e]:
+                a, y = self.o.expert(gu, dn, fronts[b]["x"][0], D.I)
+                ys[b][j] = y
+                acts[b][j] = a
+        out = {}
+        for b, f in fronts.items():
+            ref, ob = self.o.combine(f["h"][0], f["gate"][0], ys[b])
+            out[b] = (ref, ob, acts[b])
+        return out
+
 
 def token_attn(seed, dims, layer, b, attempt):
     return synth.host_token(seed, synth.ATTN, dims.d_o, layer=layer, token=b, attempt=attempt)
@@ -70,7 +109,7 @@ def token_resid(seed, dims, b, attempt):
 
 def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=None,
                min_gap: float = 1e-3, max_attempts: int = 200, resid0=None, attn0=None,
-               refs=None, moe_tokens=None, min_boundary_gap=None) -> dict:
+               refs=None, moe_tokens=None, min_boundary_gap=None, gap_fn=None) -> dict:
     """Seeded inputs for a B-token, n_layers-deep step and the oracle's answers.
 
     ``checked`` lists the tokens the oracle follows through every layer (all
@@ -82,7 +121,8 @@ def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=N
     subset of the checked tokens; the others get indices and gates only.
     ``min_boundary_gap`` (one value per layer) also asks of each checked token's draw
     that the k-th and (k+1)-th largest logits lie that far apart, so that an input
-    perturbed within half of it still selects the same experts.
+    perturbed within half of it still selects the same experts.  ``gap_fn`` replaces
+    ``top_gap`` as the gap rule (e.g. ``top_gap_distinct`` for routers with tied rows).
 
     Returns attn [L][B][d_o] and resid [B][d] (bf16 bits), the attempts used,
     and per layer the oracle's front results and outputs for checked tokens.
@@ -108,6 +148,7 @@ def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=N
         ref = refs[l]
         per = {"idx": {}, "gate": {}, "out_ref": {}, "out_bf16": {}, "h": {}, "x": {},
                "logits32": {}, "logits64": {}, "rstd": {}, "a": {}}
+        fronts = {}
         for b in checked:
             for att in range(max_attempts):
                 if att:
@@ -116,7 +157,7 @@ def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=N
                         cur[b] = token_resid(seed, dims, b, att)
                         resid[b] = cur[b]
                 f = ref.front(attn[l, b][None], cur[b][None])
-                ok = top_gap(f["logits64"][0], dims.k) >= min_gap
+                ok = (gap_fn or top_gap)(f["logits64"][0], dims.k) >= min_gap
                 if ok and min_boundary_gap is not None:
                     ok = boundary_gap(f["logits64"][0], dims.k) >= min_boundary_gap[l]
                 if ok:
@@ -129,9 +170,10 @@ def build_case(seed: int, dims: synth.Dims, B: int, n_layers: int = 1, checked=N
             for key in ("idx", "gate", "h", "x", "logits32", "logits64", "rstd"):
                 per[key][b] = f[key][0]
             if b in moe_set:
-                out_ref, out_bf16, a = ref.moe(f, 0)
-                per["out_ref"][b], per["out_bf16"][b], per["a"][b] = out_ref, out_bf16, a
-                cur[b] = out_bf16
+                fronts[b] = f
+        for b, (out_ref, out_bf16, a) in ref.moe_many(fronts).items():
+            per["out_ref"][b], per["out_bf16"][b], per["a"][b] = out_ref, out_bf16, a
+            cur[b] = out_bf16
         layers.append(per)
     return {"attn": attn, "resid": resid, "attempts": attempts, "layers": layers,
             "checked": checked, "refs": refs}

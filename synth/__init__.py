@@ -140,11 +140,28 @@ KIND_DIST = {W_O: "w", GAMMA: "gamma", W_R: "w", W_GU: "w", W_DOWN: "w",
              ATTN: "act", RESID: "act", LIFT_Z: "act"}
 
 
-def gen_bf16(seed: int, kind: int, count: int, *, layer: int = 0, token: int = 0,
-             attempt: int = 0, start: int = 0) -> np.ndarray:
-    """bf16 bits of elements ``start .. start+count-1`` of one seeded stream."""
+def gen_bf16_numpy(seed: int, kind: int, count: int, *, layer: int = 0, token: int = 0,
+                   attempt: int = 0, start: int = 0) -> np.ndarray:
+    """bf16 bits of elements ``start .. start+count-1`` of one seeded stream (numpy)."""
     u = draws_u16(seed, stream_id(kind, layer, token), attempt, start, count)
     return table(KIND_DIST[kind])[u]
+
+
+def gen_bf16(seed: int, kind: int, count: int, *, layer: int = 0, token: int = 0,
+             attempt: int = 0, start: int = 0) -> np.ndarray:
+    """bf16 bits of elements ``start .. start+count-1`` of one seeded stream.
+
+    Uses the C fill (synth_host.c, same bits) once it is built, else numpy."""
+    lib = _host_lib()
+    if lib is None or count <= 0:
+        return gen_bf16_numpy(seed, kind, count, layer=layer, token=token, attempt=attempt, start=start)
+    tab = table(KIND_DIST[kind])
+    out = np.empty(count, np.uint16)
+    rc = lib.synth_host_fill_bf16(out.ctypes.data, count, start, seed & 0xFFFFFFFFFFFFFFFF,
+                                  stream_id(kind, layer, token), attempt & 0xFFFFFFFF, tab.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"synth_host_fill_bf16 failed ({rc})")
+    return out
 
 
 def config_seed(config_id: int) -> int:
@@ -190,8 +207,36 @@ def host_token(seed: int, kind: int, n: int, *, layer: int = 0, token: int = 0, 
     return gen_bf16(seed, kind, n, layer=layer, token=token, attempt=attempt)
 
 
-# --- device fill (optional CUDA helper) -------------------------------------------
+# --- host fill (C, OpenMP) ------------------------------------------------------------
 _HERE = os.path.dirname(os.path.abspath(__file__))
+SYNTH_HOST_SO = os.path.join(_HERE, "libsynth_host.so")
+_host = None
+
+
+def build_host_fill(force: bool = False) -> str:
+    """Compile the host fill (plain C, gcc, OpenMP) next to this file."""
+    import subprocess
+    src = os.path.join(_HERE, "synth_host.c")
+    if force or not os.path.exists(SYNTH_HOST_SO) or os.path.getmtime(SYNTH_HOST_SO) < os.path.getmtime(src):
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o",
+                               SYNTH_HOST_SO, src])
+    return SYNTH_HOST_SO
+
+
+def _host_lib():
+    global _host
+    if _host is None and os.path.exists(SYNTH_HOST_SO):
+        import ctypes
+        lib = ctypes.CDLL(SYNTH_HOST_SO)
+        lib.synth_host_fill_bf16.restype = ctypes.c_int
+        lib.synth_host_fill_bf16.argtypes = [ctypes.c_void_p, ctypes.c_ulonglong, ctypes.c_ulonglong,
+                                             ctypes.c_ulonglong, ctypes.c_uint, ctypes.c_uint,
+                                             ctypes.c_void_p]
+        _host = lib
+    return _host
+
+
+# --- device fill (optional CUDA helper) -------------------------------------------
 SYNTH_SO = os.path.join(_HERE, "libsynth.so")
 
 

@@ -39,6 +39,7 @@ def check_case(stack: H.GpuStack, case: dict, sampled=None, check_intermediates=
         for b in per["idx"]:
             if l == 0:
                 assert np.array_equal(idx[l, b], per["idx"][b]), (l, b, idx[l, b], per["idx"][b])
+                H.note("gate_abs", np.abs(gate[l, b] - per["gate"][b]).max())
                 assert np.allclose(gate[l, b], per["gate"][b], atol=H.GATE_ATOL, rtol=0), (l, b)
             else:
                 H.check_route_stacked(idx[l, b], gate[l, b], per["idx"][b], per["gate"][b],
@@ -59,6 +60,7 @@ def check_case(stack: H.GpuStack, case: dict, sampled=None, check_intermediates=
             assert np.allclose(hg[b], last["h"][b], atol=1e-4, rtol=1e-5)
             assert abs(rs[b] - last["rstd"][b]) <= 1e-5 * last["rstd"][b]
             assert np.allclose(xg[b], last["x"][b], atol=1e-5, rtol=1e-5)
+            H.note("logit_abs", np.abs(lg[b] - last["logits64"][b]).max())
             assert np.allclose(lg[b], last["logits64"][b], atol=1e-4, rtol=0)
     return out, idx, gate, res
 
@@ -110,8 +112,9 @@ def test_ragged_shapes(B):
 
 # --- the largest shapes the library accepts, one dimension at a time -----------------------
 #   d = d_o = 8192 with k = 32 and I = 512 (64 experts keep the weights at ~1.2 GB), and
-#   E = 1024 with k = 32 on d = 1024 (large enough a logit spread for gapped draws).  Batch 1 (the fused kernel, or the large-batch kernels
-#   where its shared memory does not fit), 2 and 64.
+#   E = 1024 with k = 32 on d = 1024 (large enough a logit spread for gapped draws).  Batch 1
+#   (the fused kernel, or the large-batch kernels where its shared memory does not fit), 2
+#   and 64; every token is checked.
 @pytest.mark.slow
 @pytest.mark.parametrize("B", [1, 2, 64])
 @pytest.mark.parametrize("dims", [synth.Dims(8192, 8192, 64, 32, 512), synth.Dims(1024, 256, 1024, 32, 32)],
@@ -120,11 +123,62 @@ def test_maximum_sizes(dims, B):
     seed = synth.config_seed(13) + B + dims.E
     st = H.GpuStack(seed, dims, max_batch=64)
     try:
-        sampled = [0] if B == 1 else [0, B - 1]
-        case = build_case(seed, dims, B, checked=sampled, moe_tokens=sampled)
-        check_case(st, case, sampled=sampled)
+        check_case(st, build_case(seed, dims, B))
     finally:
         st.close()
+
+
+# --- ties: the selection order is (logit descending, expert index ascending) ---------------
+#   x = 0 makes every logit exactly 0 (every candidate ties: the routing falls back to k
+#   rounds of arg-max), and a router whose rows come in identical pairs makes pairs of
+#   logits bitwise equal (the lower index must come first).  TP16 shapes, at batch 1
+#   (fused kernel), 2 (small-batch expert kernel) and 16 (router's routing tables).
+@pytest.fixture(scope="module")
+def tp16_tied():
+    import torch
+    seed = synth.config_seed(5)
+    w = H.device_weights(seed, synth.TP16, 1)
+    wr = w[0][2].view(synth.TP16.E, synth.TP16.d)
+    wr[1::2] = wr[0::2]  # rows 2m and 2m + 1 identical
+    torch.cuda.synchronize()
+    ref = LayerRef(seed, synth.TP16, 0)
+    wr_h = ref.W_r.reshape(synth.TP16.E, synth.TP16.d).copy()
+    wr_h[1::2] = wr_h[0::2]
+    ref.W_r = wr_h.reshape(-1)
+    st = H.GpuStack(seed, synth.TP16, max_batch=16, weights=w)
+    yield seed, st, ref
+    st.close()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("B", [1, 2, 16])
+def test_ties_all_logits_zero(tp16_tied, B):
+    seed, st, ref = tp16_tied
+    D = synth.TP16
+    attn = np.zeros((1, B, D.d_o), np.uint16)
+    resid = np.zeros((B, D.d), np.uint16)
+    out, idx, gate = st.step(attn, resid)
+    f = ref.front(attn[0], resid)
+    assert np.all(f["logits32"] == 0) and np.array_equal(f["idx"], np.tile(np.arange(D.k), (B, 1)))
+    for b in range(B):
+        assert np.array_equal(idx[0, b], np.arange(D.k)), idx[0, b]
+        assert np.allclose(gate[0, b], 1.0 / D.k, atol=H.GATE_ATOL, rtol=0)
+    assert np.all(synth.bf16_bits_to_f32(out) == 0.0)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("B", [1, 2, 16])
+def test_ties_duplicated_router_rows(tp16_tied, B):
+    from oracle.layer import top_gap_distinct
+    seed, st, ref = tp16_tied
+    case = build_case(seed + B, synth.TP16, B, refs=[ref], gap_fn=top_gap_distinct)
+    out, idx, gate, _ = check_case(st, case)
+    for b in range(B):  # every selected pair of tied experts comes lower index first
+        sel = idx[0, b].tolist()
+        assert sum(1 for e in sel if e % 2 == 0 and e + 1 in sel) >= 1
+        for e in sel:
+            if e % 2 == 1 and e - 1 in sel:
+                assert sel.index(e - 1) == sel.index(e) - 1, sel
 
 
 @pytest.mark.parametrize("B", [1, 3])
@@ -190,14 +244,7 @@ def tp8():
 @pytest.mark.parametrize("B", [16, 64])
 def test_tp8_batches(tp8, B):
     seed, st, ref = tp8
-    sampled = [0, B // 2, B - 1]
-    case = build_case(seed, synth.TP8, B, refs=[ref], moe_tokens=sampled)
-    out, idx, gate, _ = check_case(st, case, sampled=sampled)
-    # every token: valid, distinct, and gates a descending distribution
-    assert np.all((idx >= 0) & (idx < synth.TP8.E))
-    for b in range(B):
-        assert len(set(idx[0, b])) == synth.TP8.k
-        assert abs(gate[0, b].sum() - 1) < 1e-5 and np.all(np.diff(gate[0, b]) <= 0)
+    check_case(st, build_case(seed, synth.TP8, B, refs=[ref]))  # every token
 
 
 # --- stack of 8 full-size layers, batch 1 and 64, prefetch on and off -----------------------------
@@ -206,7 +253,7 @@ def stack8():
     seed = synth.config_seed(4)
     w = H.device_weights(seed, synth.TP16, 8)
     refs = [LayerRef(seed, synth.TP16, l) for l in range(8)]
-    yield seed, w, refs
+    yield seed, w, refs, {}
     del w
 
 
@@ -214,12 +261,12 @@ def stack8():
 @pytest.mark.parametrize("prefetch", [0, 1])
 @pytest.mark.parametrize("B", [1, 64])
 def test_stack8(stack8, B, prefetch):
-    seed, w, refs = stack8
+    seed, w, refs, cases = stack8
     st = H.GpuStack(seed, synth.TP16, n_layers=8, max_batch=64, prefetch=prefetch, weights=w)
     try:
-        sampled = [0] if B == 1 else [0, 37]
-        case = build_case(seed, synth.TP16, B, n_layers=8, checked=sampled, refs=refs,
-                          min_boundary_gap=[2 * H.stack_tau(l) for l in range(8)])
-        check_case(st, case, sampled=sampled)
+        if B not in cases:  # every token, every layer
+            cases[B] = build_case(seed, synth.TP16, B, n_layers=8, refs=refs,
+                                  min_boundary_gap=[2 * H.stack_tau(l) for l in range(8)])
+        check_case(st, cases[B])
     finally:
         st.close()

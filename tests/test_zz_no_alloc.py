@@ -9,7 +9,6 @@ import synth
 pytestmark = pytest.mark.gpu
 
 RAGGED = synth.Dims(320, 192, 40, 5, 96)
-GATE_ATOL = 1e-6  # same kernels on both sides: gates agree to rounding
 
 
 def _torch():
@@ -26,23 +25,20 @@ def _inputs(torch, seed, dims, B):
     return to_dev(attn), to_dev(resid)
 
 
-def _bf16_close(torch, got, ref):
-    """|got - ref| <= 2e-2 + ulp_bf16(ref) / 2, element by element."""
-    g, r = got.float(), ref.float()
-    ulp = torch.ldexp(torch.ones_like(r), torch.frexp(r)[1] - 8)
-    return bool(((g - r).abs() <= 2e-2 + 0.5 * ulp).all())
-
-
-@pytest.mark.parametrize("dims,B", [(synth.TINY, 1), (synth.TINY, 2), (RAGGED, 1), (RAGGED, 2),
-                                    (synth.TP16, 1), (synth.TP16, 2)])
-def test_static_step_matches_step_twice(dims, B):
+# Both entry points launch the same deterministic kernels on the same inputs, so their
+# outputs, indices and gates must agree bit for bit; force_variant 1 at batch 1 selects the
+# three small-batch kernels in both.
+@pytest.mark.parametrize("dims,B,variant", [(synth.TINY, 1, 0), (synth.TINY, 2, 0), (RAGGED, 1, 0),
+                                            (RAGGED, 2, 0), (synth.TINY, 1, 1), (RAGGED, 1, 1),
+                                            (synth.TP16, 1, 0), (synth.TP16, 2, 0)])
+def test_static_step_matches_step_twice(dims, B, variant):
     torch = _torch()
     import moe_decode_layer_02_b200 as md
     from tests.harness import device_weights
     synth.build_device_fill()
     seed = 41
     w = device_weights(seed, dims, 1)[0]
-    cfg = md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, 2)
+    cfg = md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, 2, force_variant=variant)
     s = torch.cuda.current_stream()
     attn, resid = _inputs(torch, seed, dims, B)
     h = md.moe_decode_create(cfg, [w], s)
@@ -65,19 +61,21 @@ def test_static_step_matches_step_twice(dims, B):
     for out, idx, gate, err in zip(outs, idxs, gates, errs):
         assert int(err[0]) == 0
         assert torch.equal(idx, idx_ref)
-        assert float((gate - gate_ref).abs().max()) <= GATE_ATOL
-        assert _bf16_close(torch, out, out_ref)
+        assert torch.equal(gate, gate_ref)
+        assert torch.equal(out.view(torch.int16), out_ref.view(torch.int16))
 
 
 def test_static_step_rejects_what_it_cannot_run():
     torch = _torch()
     import moe_decode_layer_02_b200 as md
     s = torch.cuda.current_stream()
-    # d = 8192, top_k * inter = 32 * 512: batch 2 needs more than MOE_STATIC_SCRATCH_BYTES
+    # d = 8192, top_k * inter = 32 * 512: batch 2 needs more than MOE_STATIC_SCRATCH_BYTES.
+    # The size checks run before anything is launched or read, so small dummy buffers stand
+    # in for the weights and activations.
     d, d_o, E, k, I = 8192, 64, 32, 32, 512
     z = lambda n: torch.zeros(n, dtype=torch.bfloat16, device="cuda")
-    w = (z(d * d_o), z(d), z(E * d), z(E * 2 * I * d), z(E * d * I))
-    attn, resid, out = z(2 * d_o), z(2 * d), z(2 * d)
+    w = tuple(z(64) for _ in range(5))
+    attn, resid, out = z(64), z(64), z(64)
     cfg = md.config(d, d_o, E, k, I, 2)
     with pytest.raises(md.MoeError) as ei:
         md.moe_decode_step_static(cfg, w, 2, attn, resid, out, stream=s)
