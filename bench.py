@@ -14,9 +14,15 @@ layer (or of the 8-layer stack) on one batch of seeded synthetic inputs.
 Workloads (seeded synthetic inputs shaped like one GPU's tensor-parallel shard):
   tp16_b1        d=7168, d_o=8192, E=896, k=16, I=128, batch 1     (default)
   tp16_b2_ov0    same shapes, batch 2, two independent tokens (overlap ~0)
+  tp16_b2_ov8    same shapes, batch 2, two tokens constructed to share 8 of their 16 experts
   tp16_b2_ov16   same shapes, batch 2, one token twice (overlap 16)
+  tp16_spec4/8   same shapes, 4 / 8 tokens of one sequence (3 / 7 draft tokens + 1) sharing 12 experts
   tp8_b16/b64    d=7168, d_o=8192, E=896, k=16, I=256, batch 16 / 64
   stack8_b1/b64  8 layers of the tp16 shape in one step, batch 1 / 64
+
+The default run (tp16_b1) also measures batch 2 (overlap 0/8/16), the 4- and 8-token
+speculative-verification steps and TP8 batch 16/64 at one
+GPU and reports them in the same line under "per_workload" (--no-per-workload skips them).
 
 Multi-GPU: the step does not shard (one GPU per layer-step), so N ranks run N
 independent replicas; the value is the whole job's time per layer-step
@@ -42,7 +48,11 @@ UNIT = "us/layer-step"
 WORKLOADS = {
     "tp16_b1": ("TP16", 1, 1, "indep"),
     "tp16_b2_ov0": ("TP16", 2, 1, "indep"),
+    "tp16_b2_ov8": ("TP16", 2, 1, "ov8"),
     "tp16_b2_ov16": ("TP16", 2, 1, "dup"),
+    # speculative verification: 1 sequence x (3 or 7 drafts + 1) tokens sharing 12 of 16 experts
+    "tp16_spec4": ("TP16", 4, 1, "spec"),
+    "tp16_spec8": ("TP16", 8, 1, "spec"),
     "tp8_b16": ("TP8", 16, 1, "indep"),
     "tp8_b64": ("TP8", 64, 1, "indep"),
     "stack8_b1": ("TP16", 1, 8, "indep"),
@@ -57,6 +67,9 @@ WORKLOADS = {
 }
 
 KERNEL_DIR = os.path.join(ROOT, "moe_decode_layer_02_b200", "csrc")
+# host-only sources (handle, graphs, the C ABI): not part of the kernels' hash
+HOST_SOURCES = {"moe_decode.cu", "static_step.cu"}
+PER_WORKLOAD = ("tp16_b2_ov0", "tp16_b2_ov8", "tp16_b2_ov16", "tp16_spec4", "tp16_spec8", "tp8_b16", "tp8_b64")
 
 
 def peaks():
@@ -80,14 +93,46 @@ def seed_of(dname, L):
     return synth.config_seed({"TP16": 1, "TP8": 3, "TP16E64": 21, "TP8E64": 23, "TP8E224K4": 25}[dname] + (10 if L > 1 else 0))
 
 
-def rotation(L):
-    """Weight copies a single-layer step cycles over (4 x >= 218 MB > 2 x the 126 MB L2)."""
-    return 4 if L == 1 else 1
+def rotation(dname, L):
+    """Weight copies a one-layer step cycles over so that no step finds its weights in L2:
+    4 x >= 218 MB > 2 x the 126 MB L2 for the TP16 shard; a TP8 batch-16/64 step streams
+    2.6-6.9 GB of distinct weights by itself, as does a stack."""
+    return 4 if (L == 1 and dname.startswith("TP16")) else 1
 
 
-def token_inputs(seed, dims, B, L, mode):
+def constructed_sets(seed_w, dims, B, core, lift=15.0):
+    """B tokens whose top-k sets share `core` experts (each token adds k - core of its own),
+    for the weights of seed `seed_w`: batch 2 with a chosen overlap, or a draft-verification
+    step whose tokens mostly route alike.
+
+    attn_out = 0, so h = residual_in; residual_in = bf16(x* / gamma) with
+    x* = z + lift * sum_{e in S_b} W_r[e] / |W_r[e]|^2 (z ~ N(0, 1) from the seeded
+    generator), which lifts the chosen k router rows' logits ~6 sigma above the rest.
+    Input construction only: the kernels do all of the layer's arithmetic."""
     import numpy as np
     import synth
+    E, k, d = dims.E, dims.k, dims.d
+    Wr = synth.bf16_bits_to_f32(synth.gen_bf16(seed_w, synth.W_R, E * d)).astype(np.float64).reshape(E, d)
+    gam = synth.bf16_bits_to_f32(synth.gen_bf16(seed_w, synth.GAMMA, d)).astype(np.float64)
+    rng = np.random.default_rng(seed_w * 1000 + 17 * B + core)
+    C = rng.choice(E, core, replace=False)
+    priv = rng.permutation(np.setdiff1d(np.arange(E), C))[:B * (k - core)].reshape(B, k - core)
+    resid = []
+    for b in range(B):
+        S = np.concatenate([C, priv[b]])
+        z = synth.bf16_bits_to_f32(synth.host_token(seed_w, synth.LIFT_Z, d, token=b)).astype(np.float64)
+        xs = z + lift * (Wr[S] / (Wr[S] ** 2).sum(1, keepdims=True)).sum(0)
+        resid.append(synth.f64_to_bf16_bits(xs / gam))
+    return np.zeros((1, B, dims.d_o), np.uint16), np.stack(resid)
+
+
+def token_inputs(seed, dims, B, L, mode, seed_w=None):
+    import numpy as np
+    import synth
+    if mode == "ov8":
+        return constructed_sets(seed if seed_w is None else seed_w, dims, 2, 8)
+    if mode == "spec":  # one sequence's draft tokens: a core of 12 shared experts
+        return constructed_sets(seed if seed_w is None else seed_w, dims, B, 12)
     attn = np.stack([np.stack([synth.host_token(seed, synth.ATTN, dims.d_o, layer=l, token=(0 if mode == "dup" else b))
                                for b in range(B)]) for l in range(L)])
     resid = np.stack([synth.host_token(seed, synth.RESID, dims.d, token=(0 if mode == "dup" else b)) for b in range(B)])
@@ -202,13 +247,13 @@ def job_us_per_layer_step(t_max_ms, world, steps, layers):
 
 
 def kernels_sha(kernel_dir=None):
-    """Hash of the kernel code (comments ignored): ncu traffic figures are valid only for the
-    code they were taken on."""
+    """Hash of the device code (comments ignored; host-only sources excluded): ncu traffic
+    figures are valid only for the kernel code they were taken on."""
     import hashlib
     kdir = kernel_dir or KERNEL_DIR
     hs = hashlib.sha256()
     for f in sorted(os.listdir(kdir)):
-        if f.endswith((".cu", ".cuh")):
+        if f.endswith((".cu", ".cuh")) and f not in HOST_SOURCES:
             hs.update(f.encode())
             hs.update(code_only(open(os.path.join(kdir, f), encoding="utf-8").read()).encode())
     return hs.hexdigest()[:16]
@@ -228,6 +273,117 @@ def traffic_for(kernel_name, B, workload):
     return ent.get("bytes_per_launch")
 
 
+def setup_workload(md, torch, name, args):
+    """Seeded weights (R copies), per-copy inputs and handles of one workload."""
+    import numpy as np
+    import synth
+    dname, B, L, mode = WORKLOADS[name]
+    dims = dims_of(dname)
+    seed = seed_of(dname, L)
+    sz = dims.sizes()
+    R = rotation(dname, L)
+    cfg = md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, max(B, 1), L, enable_prefetch=args.prefetch,
+                    force_variant=args.force_variant)
+    s = torch.cuda.current_stream()
+    weight_sets, inputs, hs = [], [], []
+    for r in range(R):  # independently seeded copies; a timed step uses copy i % R
+        seed_w = seed + 1000 * r
+        weights = []
+        for l in range(L):
+            t = {}
+            for kind in (synth.W_O, synth.GAMMA, synth.W_R, synth.W_GU, synth.W_DOWN):
+                x = torch.empty(sz[kind], dtype=torch.bfloat16, device="cuda")
+                synth.device_fill(x, seed_w, kind, layer=l)
+                t[kind] = x
+            weights.append((t[synth.W_O], t[synth.GAMMA], t[synth.W_R], t[synth.W_GU], t[synth.W_DOWN]))
+        weight_sets.append(weights)
+        attn_np, resid_np = token_inputs(seed, dims, B, L, mode, seed_w=seed_w)
+        inputs.append((attn_np, resid_np, torch.from_numpy(attn_np.view(np.int16)).cuda().view(torch.bfloat16),
+                       torch.from_numpy(resid_np.view(np.int16)).cuda().view(torch.bfloat16)))
+        hs.append(md.moe_decode_create(cfg, weights, s))
+    out = torch.empty((B, dims.d), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((L, B, dims.k), dtype=torch.int32, device="cuda")
+    gate = torch.empty((L, B, dims.k), dtype=torch.float32, device="cuda")
+    return {"name": name, "B": B, "L": L, "R": R, "dims": dims, "s": s, "hs": hs, "weights": weight_sets,
+            "inputs": inputs, "out": out, "idx": idx, "gate": gate, "kps": md.moe_decode_kernels_per_step(hs[0], B)}
+
+
+def step_fn(md, ctx):
+    B, R, s, hs = ctx["B"], ctx["R"], ctx["s"], ctx["hs"]
+    out, idx, gate, inputs = ctx["out"], ctx["idx"], ctx["gate"], ctx["inputs"]
+
+    def step(i=0):
+        _, _, attn, resid = inputs[i % R]
+        md.moe_decode_step(hs[i % R], B, attn, resid, out, idx, gate, s)
+    return step
+
+
+def check_status(md, ctx):
+    rc = max(abs(md.moe_decode_sync_status(x, ctx["s"])) for x in ctx["hs"])
+    if rc:
+        raise RuntimeError(md.strerror(-rc))
+
+
+def union_sizes(md, ctx, step):
+    """Distinct experts each weight copy's step touches, per layer (from the kernels' indices)."""
+    import numpy as np
+    n_union = []
+    for r in range(ctx["R"]):
+        step(r)
+        check_status(md, ctx)
+        idx_np = ctx["idx"].cpu().numpy()
+        n_union += [len(np.unique(idx_np[l])) for l in range(ctx["L"])]
+    return n_union
+
+
+def timed_steps(torch, ctx, step, K):
+    """K steps bracketed by events on the launching stream; returns per-step milliseconds."""
+    s = ctx["s"]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        ev[i][0].record(s)
+        step(i)
+        ev[i][1].record(s)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def per_kernel(md, torch, ctx, reps):
+    """Eager, event-bracketed launches of every kernel of the step (weights rotated)."""
+    per = {}
+    for i in range(reps * ctx["R"]):
+        torch.cuda.synchronize()
+        _, _, attn, resid = ctx["inputs"][i % ctx["R"]]
+        for name, ms in md.moe_decode_profile_step(ctx["hs"][i % ctx["R"]], ctx["B"], attn, resid, ctx["out"],
+                                                   ctx["idx"], ctx["gate"], ctx["s"]):
+            per.setdefault(name, []).append(ms)
+    return per
+
+
+def release(md, torch, ctx):
+    for x in ctx["hs"]:
+        md.moe_decode_destroy(x)
+    ctx.clear()
+    torch.cuda.empty_cache()
+
+
+def summarize(dims, B, L, R, step_ms_total, K, n_union, per, hbm):
+    """µs per layer-step, weight GB/s and the dominant kernel's roofline from raw timings."""
+    us_per_layer = step_ms_total * 1000.0 / (K * L)
+    wbytes = weight_bytes(dims, n_union) / R  # n_union holds R copies x L layers
+    gbs = wbytes / (step_ms_total / K * 1e-3) / 1e9
+    avg = {n: statistics.mean(v) for n, v in per.items()}
+    dom = max(avg, key=avg.get)
+    ab = algorithmic_bytes(dims, B, statistics.mean(n_union))
+    ach = ab.get(dom, 0) / (avg[dom] * 1e-3) / 1e9
+    return {"us_per_layer_step": round(us_per_layer, 3), "weight_gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm, 4),
+            "weight_bytes_per_step": wbytes, "experts_touched": n_union,
+            "kernels_us": {n: round(v * 1000, 2) for n, v in avg.items()},
+            "dominant": {"kernel": dom, "achieved_gbs": round(ach, 1), "frac": round(ach / hbm, 4),
+                         "algorithmic_bytes": ab.get(dom, 0), "avg_launch_us": round(avg[dom] * 1000, 3),
+                         "share": round(avg[dom] / sum(avg.values()), 3)}}
+
+
 def run_ours(args, rank, world):
     import numpy as np
     import torch
@@ -241,39 +397,12 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(dev)
     mdb.build()
     synth.build_device_fill()
+    synth.build_host_fill()
     md.load()
-    dname, B, L, mode = WORKLOADS[args.workload]
-    dims = dims_of(dname)
-    seed = seed_of(dname, L)
-    sz = dims.sizes()
-    R = rotation(L)
-    weight_sets = []
-    for r in range(R):  # independently seeded copies; a timed step uses copy i % R
-        weights = []
-        for l in range(L):
-            t = {}
-            for kind in (synth.W_O, synth.GAMMA, synth.W_R, synth.W_GU, synth.W_DOWN):
-                x = torch.empty(sz[kind], dtype=torch.bfloat16, device="cuda")
-                synth.device_fill(x, seed + 1000 * r, kind, layer=l)
-                t[kind] = x
-            weights.append((t[synth.W_O], t[synth.GAMMA], t[synth.W_R], t[synth.W_GU], t[synth.W_DOWN]))
-        weight_sets.append(weights)
-    attn_np, resid_np = token_inputs(seed, dims, B, L, mode)
-    attn = torch.from_numpy(attn_np.view(np.int16)).cuda().view(torch.bfloat16)
-    resid = torch.from_numpy(resid_np.view(np.int16)).cuda().view(torch.bfloat16)
-    out = torch.empty((B, dims.d), dtype=torch.bfloat16, device="cuda")
-    idx = torch.empty((L, B, dims.k), dtype=torch.int32, device="cuda")
-    gate = torch.empty((L, B, dims.k), dtype=torch.float32, device="cuda")
-    cfg = md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, max(B, 1), L, enable_prefetch=args.prefetch,
-                    force_variant=args.force_variant)
-    s = torch.cuda.current_stream()
-    hs = [md.moe_decode_create(cfg, w, s) for w in weight_sets]
-    h = hs[0]
+    ctx = setup_workload(md, torch, args.workload, args)
+    B, L, R, dims, s = ctx["B"], ctx["L"], ctx["R"], ctx["dims"], ctx["s"]
+    step = step_fn(md, ctx)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")  # 256 MiB > 126 MB L2
-    kps = md.moe_decode_kernels_per_step(h, B)
-
-    def step(i=0):
-        md.moe_decode_step(hs[i % R], B, attn, resid, out, idx, gate, s)
 
     for i in range(max(args.warmup, 3) * R):
         step(i)
@@ -281,42 +410,24 @@ def run_ours(args, rank, world):
         # Profiling mode (for ncu): a few plain graph replays, no timing.
         for i in range(args.profile_run):
             step(i)
-        rc = max(abs(md.moe_decode_sync_status(x, s)) for x in hs)
-        for x in hs:
-            md.moe_decode_destroy(x)
-        if rc:
-            raise RuntimeError(md.strerror(-rc))
+        check_status(md, ctx)
+        release(md, torch, ctx)
         return None
-    n_union = []
-    for r in range(R):
-        step(r)
-        rc = md.moe_decode_sync_status(hs[r], s)
-        if rc:
-            raise RuntimeError(md.strerror(rc))
-        idx_np = idx.cpu().numpy()
-        n_union += [len(np.unique(idx_np[l])) for l in range(L)]
+    n_union = union_sizes(md, ctx, step)
 
     # ---- timed region: K steps; no step reuses weights that can still be in L2 -----------------
-    # (one layer: the step cycles over R weight copies, R x bytes per step > 2 x L2; a stack of
-    # layers streams more than 2 x L2 per step by itself)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # (a TP16 layer cycles over R weight copies, R x bytes per step > 2 x L2; TP8 batch >= 16
+    # and stacks stream more than 2 x L2 per step by themselves)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     with Clocks(dev) as clk:
         time.sleep(0.3)
-        for i in range(args.steps):
-            ev[i][0].record(s)
-            step(i)
-            ev[i][1].record(s)
-        torch.cuda.synchronize()
+        step_ms = timed_steps(torch, ctx, step, args.steps)
         time.sleep(0.2)
     if world > 1:
         dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    rc = max(abs(md.moe_decode_sync_status(x, s)) for x in hs)
-    if rc:
-        raise RuntimeError(md.strerror(-rc))
+    check_status(md, ctx)
     t_max_ms = max_over_ranks(sum(step_ms), world, "cuda")
 
     # ---- secondary: the same weights back to back (warm L2), and a 256 MiB L2 flush before each
@@ -339,39 +450,57 @@ def run_ours(args, rank, world):
         torch.cuda.synchronize()
         fl.append(f0.elapsed_time(f1))
     flushed_us = statistics.median(fl) * 1000 / L
+    del flush
 
     # ---- end to end through the host-buffer entry point (pinned host memory) -----------------
-    a_h = torch.from_numpy(attn_np.view(np.int16)).pin_memory()
-    r_h = torch.from_numpy(resid_np.view(np.int16)).pin_memory()
+    attn_np, resid_np = ctx["inputs"][0][0], ctx["inputs"][0][1]
+    host_in = [(torch.from_numpy(a.view(np.int16)).pin_memory(), torch.from_numpy(r.view(np.int16)).pin_memory())
+               for a, r, _, _ in ctx["inputs"]]
     o_h = torch.empty((B, dims.d), dtype=torch.int16).pin_memory()
     i_h = torch.empty((L, B, dims.k), dtype=torch.int32).pin_memory()
     g_h = torch.empty((L, B, dims.k), dtype=torch.float32).pin_memory()
-    for x in hs:
-        md.moe_decode_step_host(x, B, a_h, r_h, o_h, i_h, g_h, s)
+    for r, x in enumerate(ctx["hs"]):
+        md.moe_decode_step_host(x, B, host_in[r][0], host_in[r][1], o_h, i_h, g_h, s)
     e_ms = []
     for i in range(args.steps):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s)
-        md.moe_decode_step_host(hs[i % R], B, a_h, r_h, o_h, i_h, g_h, s)
+        md.moe_decode_step_host(ctx["hs"][i % R], B, host_in[i % R][0], host_in[i % R][1], o_h, i_h, g_h, s)
         e1.record(s)
         e1.synchronize()
         e_ms.append(e0.elapsed_time(e1))
     h2d = attn_np.nbytes + resid_np.nbytes
     d2h = B * dims.d * 2 + 2 * L * B * dims.k * 4
 
-    # ---- per-kernel durations (eager, event-bracketed launches, weights rotated as above) ------
-    per = {}
-    for i in range(max(5, min(args.steps, 20)) * R):
-        torch.cuda.synchronize()
-        for name, ms in md.moe_decode_profile_step(hs[i % R], B, attn, resid, out, idx, gate, s):
-            per.setdefault(name, []).append(ms)
-    for x in hs:
-        md.moe_decode_destroy(x)
+    per = per_kernel(md, torch, ctx, max(5, min(args.steps, 20)))
+    kps = ctx["kps"]
+    release(md, torch, ctx)
+
+    # ---- the metric's other batch sizes at one GPU, same method (timed steps, eager per-kernel
+    # launches); reported under "per_workload" of the same line
+    per_wl, clk_wl = {}, None
+    if world == 1 and args.per_workload and args.workload == "tp16_b1":
+        hbm = peaks()[0]
+        with Clocks(dev) as ck:
+            for name in PER_WORKLOAD:
+                c2 = setup_workload(md, torch, name, args)
+                st2 = step_fn(md, c2)
+                for i in range(max(args.warmup, 3) * c2["R"]):
+                    st2(i)
+                nu2 = union_sizes(md, c2, st2)
+                K2 = min(args.steps, 20)
+                ms2 = timed_steps(torch, c2, st2, K2)
+                check_status(md, c2)
+                per2 = per_kernel(md, torch, c2, 5)
+                per_wl[name] = summarize(c2["dims"], c2["B"], c2["L"], c2["R"], sum(ms2), K2, nu2, per2, hbm)
+                per_wl[name]["steps"] = K2
+                release(md, torch, c2)
+        clk_wl = ck.summary()
     return {"B": B, "L": L, "R": R, "dims": dims, "step_ms": step_ms, "t_max_ms": t_max_ms, "warm_us": warm_us,
             "flushed_us": flushed_us,
             "e2e_ms": e_ms, "h2d": h2d, "d2h": d2h, "per_kernel": per, "n_union": n_union,
-            "clocks": clk.summary(), "kps": kps}
+            "clocks": clk.summary(), "kps": kps, "per_workload": per_wl, "per_workload_clocks": clk_wl}
 
 
 def cpu_baseline(args, budget_s=12.0):
@@ -421,6 +550,8 @@ def main():
                     help="kernel choice: 0 by batch size, 1 unfused batch <= 2 kernels, 2 large-batch "
                          "kernels at every batch (comparison runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", dest="per_workload", action="store_false",
+                    help="skip the batch-2 and TP8 batch-16/64 entries of the default run")
     ap.add_argument("--profile-run", type=int, default=0,
                     help="profiling mode: warm up, replay the step N times, print nothing")
     args = ap.parse_args()
@@ -432,9 +563,10 @@ def main():
     config = {"workload": args.workload, "batch": B, "layers": L, "shape": dname,
               "prefetch": bool(args.prefetch and L > 1),
               "force_variant": args.force_variant,
-              "l2": (f"inputs larger than L2: the step cycles over {rotation(L)} independently seeded weight "
-                     "copies, no flush" if rotation(L) > 1 else
-                     f"inputs larger than L2: {L} layers of distinct weights per step, no flush"),
+              "l2": (f"inputs larger than L2: the step cycles over {rotation(dname, L)} independently seeded "
+                     "weight copies, no flush" if rotation(dname, L) > 1 else
+                     "inputs larger than L2: each step streams more than twice the L2 of distinct weights, "
+                     "no flush"),
               "parallelism": f"replicas x{args.gpus}"}
 
     if args.impl == "reference":
@@ -465,17 +597,16 @@ def main():
     dims = r["dims"]
     K = args.steps
     us_per_layer = job_us_per_layer_step(r["t_max_ms"], world, K, L)
-    wbytes = weight_bytes(dims, r["n_union"]) / r["R"]  # n_union holds R copies x L layers
     per_step_ms = r["t_max_ms"] / K
-    gbs = wbytes / (per_step_ms * 1e-3) / 1e9
-    # dominant kernel by time share
-    avg = {n: statistics.mean(v) for n, v in r["per_kernel"].items()}
-    tot = sum(avg.values())
-    dom = max(avg, key=avg.get)
-    ab = algorithmic_bytes(dims, B, statistics.mean(r["n_union"]))
-    key = dom
-    dom_bytes = ab.get(key, 0)
-    ach = dom_bytes / (avg[dom] * 1e-3) / 1e9
+    sm = summarize(dims, B, L, r["R"], r["t_max_ms"], K, r["n_union"], r["per_kernel"], hbm)
+    wbytes, gbs = sm["weight_bytes_per_step"], sm["weight_gbs"]
+    dom = sm["dominant"]["kernel"]
+    for name, w in r["per_workload"].items():
+        d2 = w.pop("dominant")
+        w["roofline"] = {"kernel": d2["kernel"], "achieved": d2["achieved_gbs"], "peak": hbm, "unit": "GB/s",
+                         "frac": d2["frac"], "traffic": traffic_for(d2["kernel"], WORKLOADS[name][1], name),
+                         "algorithmic_bytes": d2["algorithmic_bytes"], "avg_launch_us": d2["avg_launch_us"],
+                         "share": d2["share"]}
     e2e_us = statistics.mean(r["e2e_ms"]) * 1000 / L
     cb = None
     if world == 1 and not args.no_cpu_baseline:
@@ -485,7 +616,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16 weights, fp32 accumulate", "data": "synthetic",
         "config": config,
-        "weight_gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm, 4), "hbm_peak_gbs": hbm, "peak_source": src,
+        "weight_gbs": gbs, "hbm_frac": round(gbs / hbm, 4), "hbm_peak_gbs": hbm, "peak_source": src,
         "weight_bytes_per_step": wbytes, "experts_touched": r["n_union"],
         "us_per_layer_step_p10_p50_p90": [round(x * 1000 / L, 2) for x in
                                           (sorted(r["step_ms"])[int(0.1 * (K - 1))],
@@ -493,17 +624,21 @@ def main():
                                            sorted(r["step_ms"])[int(0.9 * (K - 1))])],
         "warm_us_per_layer_step": round(r["warm_us"], 3),
         "l2_flushed_us_per_layer_step": round(r["flushed_us"], 3),
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(ach / hbm, 4), "traffic": traffic_for(dom, B, args.workload),
-                     "algorithmic_bytes": dom_bytes, "avg_launch_us": round(avg[dom] * 1000, 3),
-                     "share": round(avg[dom] / tot, 3), "peak_kind": f"{src} burst copy"},
-        "kernels_us": {n: round(v * 1000, 2) for n, v in avg.items()},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": sm["dominant"]["achieved_gbs"], "peak": hbm,
+                     "unit": "GB/s", "frac": sm["dominant"]["frac"], "traffic": traffic_for(dom, B, args.workload),
+                     "algorithmic_bytes": sm["dominant"]["algorithmic_bytes"],
+                     "avg_launch_us": sm["dominant"]["avg_launch_us"], "share": sm["dominant"]["share"],
+                     "peak_kind": f"{src} burst copy"},
+        "kernels_us": sm["kernels_us"],
         "e2e": {"value": round(e2e_us, 3), "unit": UNIT, "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["kps"] * K,
         "clocks": r["clocks"],
         "cpu_baseline": cb,
     }
+    if r["per_workload"]:
+        line["per_workload"] = r["per_workload"]
+        line["per_workload_clocks"] = r["per_workload_clocks"]
     print(json.dumps(line))
 
 

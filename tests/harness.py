@@ -188,3 +188,42 @@ def constructed_b2(seed: int, dims: synth.Dims, overlap: int, lift: float = 15.0
         attn0.append(attn)
         resid0.append(resid)
     return np.stack(attn0), np.stack(resid0), (S0, S1)
+
+
+# --- speculative-verification batches: B tokens sharing a core of experts -------------------------
+def constructed_shared(seed: int, dims: synth.Dims, B: int, core: int, lift: float = 15.0,
+                       ref: LayerRef | None = None):
+    """B tokens whose top-k sets share `core` experts (a draft-verification step: one sequence's
+    next tokens mostly route alike); each token adds k - core experts of its own.
+
+    Same construction as constructed_b2: x* = z + lift * sum_{e in S_b} W_r[e] / |W_r[e]|^2,
+    h* = x* / gamma, residual_in = bf16(h* - W_o . attn_out); the oracle confirms each token's
+    set and the gap rule, else z is redrawn."""
+    from oracle import get as get_oracle
+    o = get_oracle()
+    ref = ref or LayerRef(seed, dims, 0)
+    E, k, d = dims.E, dims.k, dims.d
+    rng = np.random.default_rng(seed * 7919 + 131 * B + core)
+    C = rng.choice(E, core, replace=False)
+    rest = rng.permutation(np.setdiff1d(np.arange(E), C))
+    priv = rest[:B * (k - core)].reshape(B, k - core)
+    Wr = synth.bf16_bits_to_f32(ref.W_r).astype(np.float64).reshape(E, d)
+    gam = synth.bf16_bits_to_f32(ref.gamma).astype(np.float64)
+    attn0, resid0, sets = [], [], []
+    for b in range(B):
+        S = np.concatenate([C, priv[b]])
+        for att in range(50):
+            attn = token_attn(seed, dims, 0, b, att)
+            z = synth.bf16_bits_to_f32(synth.host_token(seed, synth.LIFT_Z, d, token=b, attempt=att)).astype(np.float64)
+            xs = z + lift * (Wr[S] / (Wr[S] ** 2).sum(1, keepdims=True)).sum(0)
+            wo_attn = o.oproj_residual(ref.W_o, attn, np.zeros(d, np.uint16), 1, d, dims.d_o)[0]
+            resid = synth.f64_to_bf16_bits(xs / gam - wo_attn)
+            f = ref.front(attn[None], resid[None])
+            if set(f["idx"][0].tolist()) == set(S.tolist()) and top_gap(f["logits64"][0], k) >= 1e-3:
+                break
+        else:
+            raise RuntimeError("construction failed")
+        attn0.append(attn)
+        resid0.append(resid)
+        sets.append(S)
+    return np.stack(attn0), np.stack(resid0), sets

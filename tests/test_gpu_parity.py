@@ -230,6 +230,17 @@ def test_tp16_b2_overlap(tp16, overlap):
     assert len(set(idx[0, 0]) & set(idx[0, 1])) == overlap
 
 
+# --- speculative verification: 1 sequence x (3 or 7 drafts + 1) tokens sharing 12 experts ------
+@pytest.mark.slow
+@pytest.mark.parametrize("B", [4, 8])
+def test_tp16_speculative_shapes(tp16, B):
+    seed, st, ref = tp16
+    attn0, resid0, sets = H.constructed_shared(seed, synth.TP16, B, core=12, ref=ref)
+    case = build_case(seed, synth.TP16, B, attn0=attn0, resid0=resid0, refs=[ref])
+    out, idx, gate, _ = check_case(st, case)  # every token
+    assert len(set(idx[0].ravel().tolist())) == 12 + B * (synth.TP16.k - 12)
+
+
 # --- full-size layer (1/8 shard, I=256), batch 16 and 64 -------------------------------------
 @pytest.fixture(scope="module")
 def tp8():

@@ -91,3 +91,21 @@ def test_fused_kernel_bytes_are_every_weight_once():
     weights = D.d * D.d_o * 2 + D.E * D.d * 2 + D.d * 2 + 16 * 3 * D.I * D.d * 2
     assert ab["layer_fused_small_m"] == weights + D.d_o * 2 + D.d * 4
     assert bench.weight_bytes(D, [16]) == weights
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("B,core", [(2, 8), (4, 12), (8, 12)])
+def test_bench_constructed_sets_route_as_built(B, core):
+    """The benchmark's constructed inputs (attn_out = 0, residual steered towards chosen expert
+    sets sharing `core` experts) select exactly those sets in the oracle."""
+    import bench
+    from oracle.layer import LayerRef
+    D = synth.TP16
+    seed_w = bench.seed_of("TP16", 1) + 1000  # the second weight copy of the rotation
+    attn, resid = bench.constructed_sets(seed_w, D, B, core)
+    assert attn.shape == (1, B, D.d_o) and not attn.any()
+    f = LayerRef(seed_w, D, 0).front(attn[0], resid)
+    sets = [set(f["idx"][b].tolist()) for b in range(B)]
+    common = set.intersection(*sets)
+    assert all(len(x) == D.k for x in sets) and len(common) == core
+    assert len(set.union(*sets)) == core + B * (D.k - core)
