@@ -546,9 +546,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="tp16_b1", choices=sorted(WORKLOADS))
     ap.add_argument("--prefetch", type=int, default=1)
-    ap.add_argument("--force-variant", type=int, default=0, choices=[0, 1, 2],
+    ap.add_argument("--force-variant", type=int, default=0, choices=[0, 1, 2, 3],
                     help="kernel choice: 0 by batch size, 1 unfused batch <= 2 kernels, 2 large-batch "
-                         "kernels at every batch (comparison runs)")
+                         "kernels at every batch, 3 counter-ordered batch <= 2 layer kernel "
+                         "(comparison runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-workload", dest="per_workload", action="store_false",
                     help="skip the batch-2 and TP8 batch-16/64 entries of the default run")

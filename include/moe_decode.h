@@ -82,7 +82,9 @@ enum {
  *                    o_proj, router, small-M expert kernel; above: o_proj, router,
  *                    gate/up, down);
  *                    1: at B = 1 too the three small-batch kernels (testing);
- *                    2: the large-batch kernels at every batch size (testing)             */
+ *                    2: the large-batch kernels at every batch size (testing);
+ *                    3: at B <= 2 the layer kernel whose expert phase is ordered by
+ *                       per-expert counters instead of a grid barrier (testing)           */
 typedef struct {
   int d, d_o, n_experts, top_k, inter, max_batch, n_layers;
   float rms_eps;
@@ -196,9 +198,9 @@ MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void*
  * `stream` (no graph, no handle), with every intermediate in one static device array of
  * MOE_STATIC_SCRATCH_BYTES that is part of the loaded library (one per device).
  *   cfg          layer shapes as for moe_decode_create (host, checked against the same
- *                supported set); n_layers must be 1 and force_variant 0 or 1 (1: the three
- *                small-batch kernels at batch 1 too, as in moe_decode_step); enable_prefetch
- *                is ignored
+ *                supported set); n_layers must be 1 and force_variant 0, 1 or 3 (as in
+ *                moe_decode_step: 1 the three small-batch kernels at batch 1 too, 3 the
+ *                counter-ordered layer kernel); enable_prefetch is ignored
  *   w            the layer's weights (host struct of device pointers, as for create)
  *   batch        1 or 2, and <= cfg->max_batch
  *   attn_out     [batch][d_o] bf16, residual_in [batch][d] bf16, out [batch][d] bf16 (device)

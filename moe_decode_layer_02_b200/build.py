@@ -9,8 +9,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmoe_decode.so")
-SOURCES = ["kernels.cu", "kernels_small.cu", "kernels_large.cu", "kernels_tc.cu", "moe_decode.cu", "static_step.cu"]
-HEADERS = ["common.cuh", "kernels.cuh", "gemv_mma.cuh", "topk.cuh", "rowdot.cuh"]
+SOURCES = ["kernels.cu", "kernels_small.cu", "kernels_layer.cu", "kernels_router.cu", "kernels_large.cu",
+           "kernels_tc.cu", "moe_decode.cu", "static_step.cu"]
+HEADERS = ["common.cuh", "kernels.cuh", "gemv_mma.cuh", "topk.cuh", "rowdot.cuh", "mma.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]

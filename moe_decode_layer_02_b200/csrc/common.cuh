@@ -151,6 +151,38 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// ---- cross-CTA signalling ------------------------------------------------------------
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Every lane of the warp waits (bounded) until *p >= target; each lane's own acquire load
+// orders its later reads after the writes released before the count was reached.
+__device__ __forceinline__ bool warp_wait_count(const unsigned* p, unsigned target, volatile int* abort_flag,
+                                                uint32_t* err) {
+  if (__all_sync(0xffffffffu, ld_acquire_u32(p) >= target)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (__all_sync(0xffffffffu, ld_acquire_u32(p) >= target)) return true;
+    int expired = (globaltimer() - t0 > kWaitLimitNs) || *abort_flag;
+    if (__any_sync(0xffffffffu, expired)) {
+      if ((threadIdx.x & 31) == 0) {
+        *abort_flag = 1;
+        atomicOr(err, kErrTimeout);
+      }
+      __syncwarp();
+      return false;
+    }
+    __nanosleep(32);
+  }
+}
+
 // ---- loads --------------------------------------------------------------------------
 // Activations / tables written earlier in the same graph: L2-coherent loads.
 __device__ __forceinline__ float ld_act(const float* p) { return __ldcg(p); }

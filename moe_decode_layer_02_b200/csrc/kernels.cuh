@@ -13,7 +13,12 @@ int check_config(const moe_decode_config* c);
 // Device counters: fused layer kernel's exit ticket, router ticket, expert-kernel grid
 // barrier count, fused layer kernel's grid barrier count.  All are zero between launches.
 // kCntProbe: the error-path probe's grid-barrier count.
-enum Counter { kCntLayerExit = 0, kCntRouter = 1, kCntGateUp = 2, kCntLayer = 3, kCntProbe = 4, kNumCounters = 5 };
+enum Counter {
+  kCntLayerExit = 0, kCntRouter = 1, kCntGateUp = 2, kCntLayer = 3, kCntProbe = 4,
+  kCntRouterBar = 5,   // the split-K router's grid barriers
+  kCntRouterExit = 6,  // its exit ticket (the last CTA out clears 1, 5 and 6)
+  kNumCounters = 7
+};
 
 // Library-owned device workspace (one per handle).
 struct Workspace {
@@ -32,7 +37,14 @@ struct Workspace {
   float* a;          // [maxB*k][I] SwiGLU activations per entry
   unsigned* counters;  // [kNumCounters]
   unsigned* err;       // error word (kErrTimeout | kErrBounds)
+  // batch <= 2 layer kernel: per union expert, rows of its SwiGLU activations published so far
+  // (zero between launches), and the activations [kMaxUnion][B][I]
+  unsigned* ecnt;      // [kMaxUnion]
+  float* a_u;          // [kMaxUnion][2][I]
+  float* rpart;        // split-K router: per-CTA partial logits [G][E][8 * ceil(maxB / 8)]
 };
+
+constexpr int kMaxUnion = 64;  // union experts of a batch <= 2 step (2 tokens x top_k <= 32)
 
 struct KTune {
   int stages = 0;          // ring stages
@@ -88,6 +100,19 @@ cudaError_t set_kernel_attributes(size_t smem_optin);
 // The error-path probe (what 1: bounded waits run out; 2: an out-of-range index is clamped).
 cudaError_t launch_error_probe(unsigned* count, unsigned* err, int what, unsigned long long limit_ns, int E,
                                int* sink, cudaStream_t s);
+
+// The batch <= 2 layer kernel with per-expert counters instead of a barrier between the
+// gate/up and down projections (kernels_layer.cu).
+bool plan_layer2(LayerArgs& a, int grid, size_t smem_optin);
+bool layer2_ok(const LayerArgs& a, size_t smem_optin);
+cudaError_t set_layer2_attributes(size_t smem_optin);
+cudaError_t launch_layer2(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
+
+// The router above batch 2 with K split over the CTAs, partial logits on the tensor cores,
+// and the routing tables (kernels_router.cu).
+bool router_ks_ok(const LayerArgs& a, int grid, size_t smem_optin);
+cudaError_t set_router_ks_attributes(size_t smem_optin);
+cudaError_t launch_router_ks(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
 
 // o_proj above batch 2 on the tensor cores with 2-D TMA tiles (kernels_tc.cu).
 bool oproj_tc_ok(const LayerArgs& a, int grid, size_t smem_optin);

@@ -4,8 +4,9 @@
 // (224 experts x 512 gate/up rows at batch 16 with I = 256), far more than the 148 SMs
 // need, so the rows are not split along K: every row is one contiguous bulk copy and every
 // dot product is finished inside one CTA, with no partial sums in global memory.  Each
-// expert's tokens (about 1.1-1.7 per expert under uniform routing) are taken NT at a time
-// against the row staged in shared memory.
+// expert's tokens (about 1.1-1.7 per expert under uniform routing) are taken up to four at a
+// time against the row staged in shared memory (their x held in registers, so an expert with
+// at most four tokens loads x once).
 //
 //   k_gateup_rows  a[entry][p] = silu(W_g[e][p] . x_t) * (W_u[e][p] . x_t) for every entry
 //                  (expert e, token t): the (expert, row) pairs of the union are split evenly
@@ -79,10 +80,12 @@ __device__ __forceinline__ void load_tables(const LayerArgs& a, int U, int n_ent
 //   (fewer, larger copies stream faster).  The partial sums of a chunk are reduced once its
 //   up stage is done.
 // =============================================================================
-template <int NT>
+// CPL: 8-element chunks of x per lane (2 covers d <= 7680: the unused third chunk of a wider
+// template would cost a third more unpack and FMA instructions on zeros).
+template <int NT, int CPL>
 __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kRI = 4 / NT;  // rows per interleaved pass
+  static_assert(NT == 2 || NT == 4, "token groups of two or four");
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, I = a.I, E = a.E, B = a.B;
   const int SA = a.k3.stages, PC = a.k3.rows_per_stage;
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
   csync();
 
   const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
-  float xr[NT][kCPLf][8];
+  float xr[NT][CPL][8];
   int cached_u = -1, cached_g = -1;
   int it = 0, ch = 0, u = q0 / I, p = q0 - (q0 / I) * I;
   for (int q = q0; q < q1; ++ch) {
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
           for (int t = 0; t < NT; ++t) {
             const int tok = (g0 + t < m) ? tb.etok[off + g0 + t] : -1;
 #pragma unroll
-            for (int j = 0; j < kCPLf; ++j) {
+            for (int j = 0; j < CPL; ++j) {
               if (tok >= 0 && cvalid(qpw, j, lane)) {
                 const float* xp = a.ws.x + (size_t)tok * d + (size_t)(qbase + j * 32 + lane) * 8;
                 const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
@@ -195,8 +198,9 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
           waited = true;
         }
         const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SA_B);
-        if (m - g0 == 1) {  // a single token: half the FMAs, four rows per pass
-          const float(&x1)[1][kCPLf][8] = reinterpret_cast<const float(&)[1][kCPLf][8]>(xr[0]);
+        const int mg = min(NT, m - g0);  // tokens of this group
+        if (mg == 1) {  // a single token: four rows per pass
+          const float(&x1)[1][CPL][8] = reinterpret_cast<const float(&)[1][CPL][8]>(xr[0]);
           for (int i0 = 0; i0 < np; i0 += 4) {
             const uint16_t* rp[4];
 #pragma unroll
@@ -209,16 +213,33 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
           }
           continue;
         }
-        for (int i0 = 0; i0 < np; i0 += kRI) {
-          const uint16_t* rp[kRI];
+        if (NT == 2 || mg == 2) {  // two tokens: two rows per pass
+          const float(&x2)[2][CPL][8] = reinterpret_cast<const float(&)[2][CPL][8]>(xr[0]);
+          for (int i0 = 0; i0 < np; i0 += 2) {
+            const uint16_t* rp[2];
 #pragma unroll
-          for (int k = 0; k < kRI; ++k) rp[k] = st + (size_t)min(i0 + k, np - 1) * d;
-          float v[kRI * NT];
-          rows_dot<NT, kRI>(rp, np - i0, xr, qbase, qpw, lane, v);
-          const float tot = warp_reduce_multi<kRI * NT>(v, lane);
-          const int vi = multi_index<kRI * NT>(lane), i = i0 + vi / NT, t = vi % NT;
-          if (multi_writer<kRI * NT>(lane) && i < np && g0 + t < m)
-            pb[((size_t)(gu * PC + i) * B + g0 + t) * kCW + warp] = tot;
+            for (int k = 0; k < 2; ++k) rp[k] = st + (size_t)min(i0 + k, np - 1) * d;
+            float v[4];
+            rows_dot<2, 2>(rp, np - i0, x2, qbase, qpw, lane, v);
+            const float tot = warp_reduce_multi<4>(v, lane);
+            const int vi = multi_index<4>(lane), i = i0 + vi / 2, t = vi % 2;
+            if (multi_writer<4>(lane) && i < np && g0 + t < m)
+              pb[((size_t)(gu * PC + i) * B + g0 + t) * kCW + warp] = tot;
+          }
+          continue;
+        }
+        if constexpr (NT >= 4) {  // three or four tokens against each row: one unpack per chunk
+          for (int i0 = 0; i0 < np; i0 += 2) {
+            const uint16_t* rp[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) rp[k] = st + (size_t)min(i0 + k, np - 1) * d;
+            float v[2 * NT];
+            rows_dot<NT, 2>(rp, np - i0, xr, qbase, qpw, lane, v);
+            const float tot = warp_reduce_multi<2 * NT>(v, lane);
+            const int vi = multi_index<2 * NT>(lane), i = i0 + vi / NT, t = vi % NT;
+            if (multi_writer<2 * NT>(lane) && i < np && g0 + t < m)
+              pb[((size_t)(gu * PC + i) * B + g0 + t) * kCW + warp] = tot;
+          }
         }
       }
       if (!waited) mbar_wait(&full[s], (it / SA) & 1, abort_flag, a.ws.err);
@@ -446,7 +467,8 @@ cudaError_t set_large_attributes(size_t optin) {
 #define SETL(k)                                                                                         \
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, v); \
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100)
-  SETL(k_gateup_rows<2>);
+  SETL((k_gateup_rows<4, 2>));
+  SETL((k_gateup_rows<2, 3>));
   SETL(k_down_rows<4>);
   SETL(k_down_rows<8>);
   SETL(k_down_rows<0>);
@@ -457,7 +479,10 @@ cudaError_t set_large_attributes(size_t optin) {
 cudaError_t launch_gateup_rows(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   LayerArgs a = a0;
   plan_large(a, grid, optin);
-  return launch_l(k_gateup_rows<2>, grid, a.k3.smem, s, pdl, a);
+  // x of up to four tokens in registers where two chunks per lane cover d (an expert's tokens
+  // rarely exceed four at batch <= 64); pairs of tokens where three chunks are needed
+  return a.d <= 8 * 32 * 2 * kCW ? launch_l(k_gateup_rows<4, 2>, grid, a.k3.smem, s, pdl, a)
+                                 : launch_l(k_gateup_rows<2, 3>, grid, a.k3.smem, s, pdl, a);
 }
 
 cudaError_t launch_down_rows(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {

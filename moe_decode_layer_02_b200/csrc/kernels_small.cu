@@ -495,16 +495,6 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_big(const LayerArgs a) 
 // =============================================================================
 namespace {
 
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 // `count` is zero when the kernel starts and only grows during a launch: the n-th barrier
 // of a launch opens when it reaches n * gridDim.x (`target`), so the last arrival's add is
 // the release (no second round trip).  Who clears it: for the expert kernel, the router

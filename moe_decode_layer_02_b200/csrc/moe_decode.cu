@@ -39,9 +39,38 @@ namespace {
 struct GraphEntry {
   int batch;
   const void *attn, *resid, *out, *idx, *gate;
+  bool host;  // host-buffer step: staging copies in the graph around the layer kernels
   cudaGraphExec_t exec;
   int kernels;
 };
+
+// Staging copy of the host-buffer step: n 16-byte words from src to dst, one side pinned host
+// memory (through its device address), the other device memory.  The copy-in runs first in the
+// graph and lets the first layer kernel launch at once (its producer streams weights while the
+// inputs arrive; its consumers wait for this grid); the copy-out waits for the last kernel.
+__global__ void k_stage_copy(const uint4* __restrict__ src, uint4* __restrict__ dst, unsigned long long n,
+                             int after_previous) {
+  if (after_previous) asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
+  for (unsigned long long i = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    dst[i] = src[i];
+}
+
+cudaError_t launch_stage_copy(const void* src, void* dst, size_t bytes, bool after_previous, cudaStream_t s) {
+  const unsigned long long n = (bytes + 15) / 16;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::min<unsigned long long>(148, std::max<unsigned long long>(1, (n + 1023) / 1024)));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_previous ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_stage_copy, static_cast<const uint4*>(src), static_cast<uint4*>(dst), n,
+                            after_previous ? 1 : 0);
+}
 
 constexpr size_t kPrefetchWoBytes = 16ull << 20;  // bytes of the next W_o prefetched into L2
 constexpr int kGraphCacheMax = 16;
@@ -60,6 +89,7 @@ struct moe_decode_handle {
   // group contiguous, and pinned host mirrors of them, so a step moves one copy each way
   void *h_in = nullptr, *h_outs = nullptr;      // device: inputs, outputs
   void *pin_in = nullptr, *pin_out = nullptr;   // pinned host mirrors
+  void *pin_in_dev = nullptr, *pin_out_dev = nullptr;  // their device addresses
   size_t in_bytes = 0, out_bytes = 0;           // capacities (max_batch)
   LayerArgs plan_base{};
   cudaStream_t cap = nullptr;
@@ -102,17 +132,19 @@ bool use_large(const moe_decode_handle* h, int B) {
 struct Variant {
   bool oproj_small;   // whole-row o_proj (batch <= 2)
   bool experts_small; // small-M gate/up and down with per-CTA routing (batch <= 2)
-  bool fused;         // the three batch <= 2 kernels as one launch
+  bool layer2;        // the batch <= 2 layer kernel with per-expert counters (one launch)
+  bool fused;         // the three batch <= 2 kernels as one launch with three grid barriers
 };
 
 Variant variant_of(const moe_decode_handle* h, const LayerArgs& a) {
   Variant v;
   v.experts_small = !use_large(h, a.B) && small_path_ok(a, h->smem_optin);
   v.oproj_small = v.experts_small && oproj_small_ok(a, h->smem_optin);
-  // One fused launch per layer at batch 1 (measured: on par with the three kernels for one
-  // layer, ahead in stacks); at batch 2 the three kernels are ahead (one token twice: by
-  // ~1.5 us), so they stay.
-  v.fused = v.oproj_small && a.B == 1 && h->cfg.force_variant != 1 && layer_fused_ok(a, h->smem_optin);
+  const bool by_batch = !use_large(h, a.B) && h->cfg.force_variant == 0;
+  v.layer2 = !use_large(h, a.B) && h->cfg.force_variant == 3 && layer2_ok(a, h->smem_optin);
+  // Where the counter-based kernel does not fit: one fused launch at batch 1; at batch 2 the
+  // three kernels were measured ahead of that fused launch, so they stay.
+  v.fused = !v.layer2 && by_batch && v.oproj_small && a.B == 1 && layer_fused_ok(a, h->smem_optin);
   return v;
 }
 
@@ -147,8 +179,9 @@ LayerArgs layer_args(const moe_decode_handle* h, int l, int B, const void* attn,
 }
 
 // Records the whole step on h->cap (which is in capture mode).  Returns kernels launched.
+// first_pdl: the first kernel follows another kernel of the same graph (programmatic launch).
 int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid, void* out,
-                int32_t* idx, float* gate, cudaError_t* err) {
+                int32_t* idx, float* gate, cudaError_t* err, bool first_pdl = false) {
   const moe_decode_config& c = h->cfg;
   const int G = h->num_sms;
   int kernels = 0;
@@ -156,17 +189,20 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
   for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
     LayerArgs a = layer_args(h, l, B, attn, resid, out, idx, gate);
     const Variant v = variant_of(h, a);
-    if (v.fused) {
-      e = launch_layer_s(a, G, h->cap, l > 0, h->smem_optin);
+    if (v.layer2 || v.fused) {
+      const bool pdl = l > 0 || first_pdl;
+      e = v.layer2 ? launch_layer2(a, G, h->cap, pdl, h->smem_optin) : launch_layer_s(a, G, h->cap, pdl, h->smem_optin);
       kernels += 1;
       continue;
     }
-    e = v.oproj_small                         ? launch_oproj_s(a, G, h->cap, l > 0, h->smem_optin)
-        : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, h->cap, l > 0)
-                                            : launch_oproj(a, G, h->cap, l > 0);
+    const bool pdl = l > 0 || first_pdl;
+    e = v.oproj_small                         ? launch_oproj_s(a, G, h->cap, pdl, h->smem_optin)
+        : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, h->cap, pdl)
+                                            : launch_oproj(a, G, h->cap, pdl);
     if (e == cudaSuccess)
-      e = (!v.experts_small && router_big_ok(a, h->smem_optin)) ? launch_router_big(a, G, h->cap, true, h->smem_optin)
-                                                                : launch_router_s(a, G, h->cap, true, h->smem_optin);
+      e = (!v.experts_small && router_ks_ok(a, G, h->smem_optin))    ? launch_router_ks(a, G, h->cap, true)
+          : (!v.experts_small && router_big_ok(a, h->smem_optin)) ? launch_router_big(a, G, h->cap, true, h->smem_optin)
+                                                                  : launch_router_s(a, G, h->cap, true, h->smem_optin);
     kernels += 2;
     if (v.experts_small) {
       if (e == cudaSuccess) e = launch_experts_s(a, G, h->cap, true, h->smem_optin);
@@ -181,10 +217,14 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
   return kernels;
 }
 
+// host: the step reads its inputs from, and writes its outputs to, the handle's pinned
+// staging (in_bytes from pin_in_dev to attn; out_bytes from out to pin_out_dev).
 int get_graph(moe_decode_handle* h, int B, const void* attn, const void* resid, void* out,
-              int32_t* idx, float* gate, GraphEntry** ge) {
+              int32_t* idx, float* gate, GraphEntry** ge, bool host = false, size_t in_bytes = 0,
+              size_t out_bytes = 0) {
   for (auto& g : h->graphs)
-    if (g.batch == B && g.attn == attn && g.resid == resid && g.out == out && g.idx == idx && g.gate == gate) {
+    if (g.batch == B && g.attn == attn && g.resid == resid && g.out == out && g.idx == idx && g.gate == gate &&
+        g.host == host) {
       *ge = &g;
       return MOE_OK;
     }
@@ -195,7 +235,10 @@ int get_graph(moe_decode_handle* h, int B, const void* attn, const void* resid, 
   cudaGraph_t graph = nullptr;
   if (cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return MOE_ERR_CUDA;
   cudaError_t rec = cudaSuccess;
-  const int kernels = record_step(h, B, attn, resid, out, idx, gate, &rec);
+  int kernels = 0;
+  if (host) rec = launch_stage_copy(h->pin_in_dev, const_cast<void*>(attn), in_bytes, false, h->cap);
+  if (rec == cudaSuccess) kernels = record_step(h, B, attn, resid, out, idx, gate, &rec, host);
+  if (host && rec == cudaSuccess) rec = launch_stage_copy(out, h->pin_out_dev, out_bytes, true, h->cap);
   const cudaError_t end = cudaStreamEndCapture(h->cap, &graph);
   if (rec != cudaSuccess || end != cudaSuccess || !graph) {
     if (graph) cudaGraphDestroy(graph);
@@ -209,7 +252,7 @@ int get_graph(moe_decode_handle* h, int B, const void* attn, const void* resid, 
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
-  h->graphs.push_back(GraphEntry{B, attn, resid, out, idx, gate, exec, kernels});
+  h->graphs.push_back(GraphEntry{B, attn, resid, out, idx, gate, host, exec, kernels});
   *ge = &h->graphs.back();
   return MOE_OK;
 }
@@ -227,7 +270,7 @@ int moe::check_config(const moe_decode_config* c) {
   if (c->max_batch < 1 || c->max_batch > 64) return MOE_ERR_UNSUPPORTED_CONFIG;
   if (c->n_layers < 1 || c->n_layers > 64) return MOE_ERR_UNSUPPORTED_CONFIG;
   if (!(c->rms_eps > 0.f)) return MOE_ERR_UNSUPPORTED_CONFIG;
-  if (c->force_variant < 0 || c->force_variant > 2) return MOE_ERR_INVALID_ARG;
+  if (c->force_variant < 0 || c->force_variant > 3) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
 
@@ -304,7 +347,9 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
                o_uo = take(sizeof(int) * (E + 1)), o_et = take(sizeof(int) * entries),
                o_es = take(sizeof(int) * entries), o_a = take(sizeof(float) * entries * I),
                o_cnt = take(sizeof(unsigned) * kNumCounters),
-               o_err = take(sizeof(unsigned)), o_r0 = take(2ull * maxB * d), o_r1 = take(2ull * maxB * d);
+               o_err = take(sizeof(unsigned)), o_r0 = take(2ull * maxB * d), o_r1 = take(2ull * maxB * d),
+               o_ec = take(sizeof(unsigned) * kMaxUnion), o_au = take(sizeof(float) * kMaxUnion * 2 * I),
+               o_rp = take(sizeof(float) * G * E * ((maxB + 7) / 8 * 8));
   if (cudaMalloc(&h->ws_base, off) != cudaSuccess) {
     cudaGetLastError();
     delete h;
@@ -327,6 +372,9 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   ws.a = (float*)(b + o_a);
   ws.counters = (unsigned*)(b + o_cnt);
   ws.err = (unsigned*)(b + o_err);
+  ws.ecnt = (unsigned*)(b + o_ec);
+  ws.a_u = (float*)(b + o_au);
+  ws.rpart = (float*)(b + o_rp);
   h->resid_pp[0] = (uint16_t*)(b + o_r0);
   h->resid_pp[1] = (uint16_t*)(b + o_r1);
   h->plan_base.ws = ws;
@@ -338,6 +386,8 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   if (e == cudaSuccess) e = set_small_attributes(h->smem_optin);
   if (e == cudaSuccess) e = set_large_attributes(h->smem_optin);
   if (e == cudaSuccess) e = set_tc_attributes(h->smem_optin);
+  if (e == cudaSuccess) e = set_layer2_attributes(h->smem_optin);
+  if (e == cudaSuccess) e = set_router_ks_attributes(h->smem_optin);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -379,6 +429,8 @@ int moe_decode_step_host(moe_decode_handle* h, int batch, const void* attn_out_h
   if (!h || !is_live(h) || h->poisoned) return MOE_ERR_INVALID_ARG;
   if (batch < 1 || batch > h->cfg.max_batch) return MOE_ERR_INVALID_ARG;
   if (!attn_out_host || !residual_in_host || !out_host) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev != h->device) return MOE_ERR_INVALID_ARG;
   const moe_decode_config& c = h->cfg;
   const size_t maxB = c.max_batch;
   // Layout for `batch` tokens: inputs [attn_out | residual_in], outputs [out | idx | gate],
@@ -391,10 +443,11 @@ int moe_decode_step_host(moe_decode_handle* h, int batch, const void* attn_out_h
   if (!h->h_in) {
     h->in_bytes = up256(2ull * c.n_layers * maxB * c.d_o) + up256(2ull * maxB * c.d);
     h->out_bytes = up256(2ull * maxB * c.d) + 2 * up256(4ull * c.n_layers * maxB * c.top_k);
-    void *di = nullptr, *dout = nullptr, *pi = nullptr, *po = nullptr;
+    void *di = nullptr, *dout = nullptr, *pi = nullptr, *po = nullptr, *pid = nullptr, *pod = nullptr;
     if (cudaMalloc(&di, h->in_bytes) != cudaSuccess || cudaMalloc(&dout, h->out_bytes) != cudaSuccess ||
-        cudaHostAlloc(&pi, h->in_bytes, cudaHostAllocDefault) != cudaSuccess ||
-        cudaHostAlloc(&po, h->out_bytes, cudaHostAllocDefault) != cudaSuccess) {
+        cudaHostAlloc(&pi, h->in_bytes, cudaHostAllocMapped) != cudaSuccess ||
+        cudaHostAlloc(&po, h->out_bytes, cudaHostAllocMapped) != cudaSuccess ||
+        cudaHostGetDevicePointer(&pid, pi, 0) != cudaSuccess || cudaHostGetDevicePointer(&pod, po, 0) != cudaSuccess) {
       cudaGetLastError();
       if (di) cudaFree(di);
       if (dout) cudaFree(dout);
@@ -406,28 +459,29 @@ int moe_decode_step_host(moe_decode_handle* h, int batch, const void* attn_out_h
     h->h_outs = dout;
     h->pin_in = pi;
     h->pin_out = po;
+    h->pin_in_dev = pid;
+    h->pin_out_dev = pod;
   }
   char* din = static_cast<char*>(h->h_in);
   char* dout = static_cast<char*>(h->h_outs);
   char* pin = static_cast<char*>(h->pin_in);
   char* pout = static_cast<char*>(h->pin_out);
+  // One graph per (batch, outputs wanted): copy-in kernel -> the step's kernels -> copy-out
+  // kernel, so a call is one graph launch and one synchronisation.
+  GraphEntry* ge = nullptr;
+  int rc = get_graph(h, batch, din, din + o_res, dout, topk_idx_host ? (int32_t*)(dout + o_idx) : nullptr,
+                     topk_gate_host ? (float*)(dout + o_gate) : nullptr, &ge, true, in_used, out_used);
+  if (rc) return rc;
   std::memcpy(pin, attn_out_host, n_attn);
   std::memcpy(pin + o_res, residual_in_host, n_res);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemcpyAsync(din, pin, in_used, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return MOE_ERR_CUDA;
-  }
-  int rc = moe_decode_step(h, batch, din, din + o_res, dout, topk_idx_host ? (int32_t*)(dout + o_idx) : nullptr,
-                           topk_gate_host ? (float*)(dout + o_gate) : nullptr, stream);
-  if (rc) return rc;
-  e = cudaMemcpyAsync(pout, dout, out_used, cudaMemcpyDeviceToHost, s);
+  cudaError_t e = cudaGraphLaunch(ge->exec, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
+  h->last_batch = batch;
   std::memcpy(out_host, pout, n_res);
   if (topk_idx_host) std::memcpy(topk_idx_host, pout + o_idx, n_tk);
   if (topk_gate_host) std::memcpy(topk_gate_host, pout + o_gate, n_tk);
@@ -447,8 +501,9 @@ int moe_decode_sync_status(moe_decode_handle* h, void* stream) {
     return MOE_ERR_CUDA;
   }
   if (word) {
-    // a bounded wait that ran out may leave a grid-barrier count behind
+    // a bounded wait that ran out may leave a grid-barrier or expert count behind
     cudaMemset(h->ws.counters, 0, sizeof(unsigned) * kNumCounters);
+    cudaMemset(h->ws.ecnt, 0, sizeof(unsigned) * kMaxUnion);
     cudaMemset(h->ws.err, 0, sizeof word);
     cudaDeviceSynchronize();
     return (word & kErrTimeout) ? MOE_ERR_DEVICE_TIMEOUT : MOE_ERR_DEVICE_BOUNDS;
@@ -497,7 +552,7 @@ int moe_decode_kernels_per_step(moe_decode_handle* h, int batch) {
   a.B = batch;
   plan_layer(a, h->num_sms, h->smem_optin);
   const Variant v = variant_of(h, a);
-  const int per_layer = v.fused ? 1 : v.experts_small ? 3 : 4;
+  const int per_layer = (v.layer2 || v.fused) ? 1 : v.experts_small ? 3 : 4;
   return per_layer * L;
 }
 
@@ -529,8 +584,10 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
   for (int l = 0; l < c.n_layers; ++l) {
     LayerArgs a = layer_args(h, l, batch, attn_out, residual_in, out, topk_idx, topk_gate);
     const Variant v = variant_of(h, a);
-    if (v.fused) {
-      timed(6, s, [&](cudaStream_t st) { return launch_layer_s(a, G, st, false, h->smem_optin); });
+    if (v.layer2 || v.fused) {
+      timed(6, s, [&](cudaStream_t st) {
+        return v.layer2 ? launch_layer2(a, G, st, false, h->smem_optin) : launch_layer_s(a, G, st, false, h->smem_optin);
+      });
       continue;
     }
     timed(1, s, [&](cudaStream_t st) {
@@ -539,8 +596,9 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
                                                  : launch_oproj(a, G, st, false);
     });
     timed(2, s, [&](cudaStream_t st) {
-      return (!v.experts_small && router_big_ok(a, h->smem_optin)) ? launch_router_big(a, G, st, false, h->smem_optin)
-                                                                   : launch_router_s(a, G, st, false, h->smem_optin);
+      return (!v.experts_small && router_ks_ok(a, G, h->smem_optin))    ? launch_router_ks(a, G, st, false)
+             : (!v.experts_small && router_big_ok(a, h->smem_optin)) ? launch_router_big(a, G, st, false, h->smem_optin)
+                                                                     : launch_router_s(a, G, st, false, h->smem_optin);
     });
     if (v.experts_small) {
       timed(3, s, [&](cudaStream_t st) { return launch_experts_s(a, G, st, false, h->smem_optin); });

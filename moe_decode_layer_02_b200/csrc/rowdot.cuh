@@ -47,15 +47,16 @@ __device__ __forceinline__ void ffma2(float2& d, float a0, float a1, float b0, f
 // rows are issued before the first FMA; the accumulators are independent chains of packed
 // FMAs (an even and an odd element per instruction, kA pairs per row and token), so a
 // warp's pass over a stage is one short chain instead of R dependent ones.
-template <int NT, int R>
-__device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr, const float (&x)[NT][kCPLf][8],
+// CPL: 8-element chunks per lane of the activation slice (deduced from x).
+template <int NT, int R, int CPL>
+__device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr, const float (&x)[NT][CPL][8],
                                          int qbase, int qpw, int lane, float (&out)[R * NT]) {
   constexpr int kA = (R * NT >= 4) ? 1 : 4 / (R * NT);  // accumulator pairs per (row, token)
-  uint4 w[R][kCPLf];
+  uint4 w[R][CPL];
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
-    for (int j = 0; j < kCPLf; ++j)
+    for (int j = 0; j < CPL; ++j)
       w[r][j] = (r < nr && cvalid(qpw, j, lane))
                     ? *reinterpret_cast<const uint4*>(rp[r] + (size_t)(qbase + j * 32 + lane) * 8)
                     : make_uint4(0, 0, 0, 0);
@@ -67,7 +68,7 @@ __device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr,
 #pragma unroll
       for (int e = 0; e < kA; ++e) acc[r][t][e] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int j = 0; j < kCPLf; ++j)
+  for (int j = 0; j < CPL; ++j)
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       float wf[8];

@@ -8,8 +8,8 @@
 //   - code that runs under a hard per-process memory cap, where one more allocation can be
 //     the one that fails in the middle of serving.
 // For them this entry point runs the same kernels as the batch <= 2 path of moe_decode_step
-// (at batch 1 the fused layer kernel: o_proj + residual + RMS statistics, router + top-k,
-// experts; at batch 2 the o_proj, router and small-M expert kernels), launched directly on
+// (one layer kernel: o_proj + residual + RMS statistics, router + top-k, experts; with
+// force_variant 1 the o_proj, router and small-M expert kernels), launched directly on
 // the caller's stream, with every intermediate in one file-scope device array of
 // MOE_STATIC_SCRATCH_BYTES.  Nothing is allocated per call: no
 // cudaMalloc/cudaFree and no library routine that allocates.  The array is part of the
@@ -20,9 +20,9 @@
 // later calls on that device reuse both.  That first call should come before any stream
 // capture begins.
 //
-// Zero start.  The grid barriers need their arrival counts at zero and the error word
-// must start at zero; every call clears them (one cudaMemsetAsync on the caller's stream)
-// before its kernels run.  Nothing else in the array needs a known value.
+// Zero start.  The grid barriers and the per-expert counters need their counts at zero and
+// the error word must start at zero; every call clears them (one cudaMemsetAsync on the
+// caller's stream) before its kernels run.  Nothing else in the array needs a known value.
 //
 // Sharing.  Every call on a device uses the same array.  Calls whose executions overlap
 // (issued on different streams, or from different threads without ordering between them)
@@ -73,7 +73,7 @@ int setup_device(int dev, DeviceSetup* out) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
-    if (set_small_attributes((size_t)optin) != cudaSuccess) {
+    if (set_small_attributes((size_t)optin) != cudaSuccess || set_layer2_attributes((size_t)optin) != cudaSuccess) {
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
@@ -98,7 +98,8 @@ size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, Work
     return base ? base + o : nullptr;
   };
   const size_t entries = (size_t)B * K;
-  unsigned char* cnt = take(sizeof(unsigned) * kNumCounters + sizeof(unsigned));
+  // grid-barrier counters, the error word and the per-expert counters: cleared by every call
+  unsigned char* cnt = take(sizeof(unsigned) * (kNumCounters + 1 + kMaxUnion));
   unsigned char* h = take(sizeof(float) * B * d);
   unsigned char* x = take(sizeof(float) * B * d);
   unsigned char* rstd = take(sizeof(float) * B);
@@ -112,6 +113,7 @@ size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, Work
   unsigned char* et = take(sizeof(int) * entries);
   unsigned char* es = take(sizeof(int) * entries);
   unsigned char* act = take(sizeof(float) * entries * I);
+  unsigned char* au = take(sizeof(float) * kMaxUnion * 2 * I);
   if (ws) {
     ws->counters = reinterpret_cast<unsigned*>(cnt);
     ws->err = reinterpret_cast<unsigned*>(cnt) + kNumCounters;
@@ -128,6 +130,8 @@ size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, Work
     ws->entry_tok = reinterpret_cast<int*>(et);
     ws->entry_slot = reinterpret_cast<int*>(es);
     ws->a = reinterpret_cast<float*>(act);
+    ws->ecnt = reinterpret_cast<unsigned*>(cnt) + kNumCounters + 1;
+    ws->a_u = reinterpret_cast<float*>(au);
   }
   return off;
 }
@@ -192,10 +196,13 @@ int moe_decode_step_static(const moe_decode_config* cfg, const moe_decode_layer_
   if (!small_path_ok(a, ds.smem_optin) || !router_ok(a, ds.smem_optin)) return MOE_ERR_UNSUPPORTED_CONFIG;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(a.ws.counters, 0, sizeof(unsigned) * (kNumCounters + 1), s);
-  // the kernels moe_decode_step picks: the fused layer kernel at batch 1 unless force_variant 1
-  // asks for the three small-batch kernels
-  if (batch == 1 && c.force_variant != 1 && layer_fused_ok(a, ds.smem_optin)) {
+  cudaError_t e = cudaMemsetAsync(a.ws.counters, 0, sizeof(unsigned) * (kNumCounters + 1 + kMaxUnion), s);
+  // the kernels moe_decode_step picks: one layer kernel (or, where it does not fit, the fused
+  // kernel at batch 1), unless force_variant 1 asks for the three small-batch kernels
+  const bool by_batch = c.force_variant == 0;
+  if (c.force_variant == 3 && layer2_ok(a, ds.smem_optin)) {
+    if (e == cudaSuccess) e = launch_layer2(a, G, s, false, ds.smem_optin);
+  } else if (by_batch && batch == 1 && layer_fused_ok(a, ds.smem_optin)) {
     if (e == cudaSuccess) e = launch_layer_s(a, G, s, false, ds.smem_optin);
   } else {
     if (e == cudaSuccess) e = launch_oproj_s(a, G, s, false, ds.smem_optin);

@@ -25,20 +25,31 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
 }
 
 // Exact top-K (K <= 32, E <= 1024) of one token's logits by one warp; lane j < K receives the
-// j-th selection.  Threshold pass: the K-th largest of the 32 lane maxima, T, is a lower
+// j-th selection.  Lane l holds the logits of experts 128 i + 4 l + c (float4 loads when E is
+// a multiple of 4).  Threshold pass: the K-th largest of the 32 lane maxima, T, is a lower
 // bound of the K-th largest logit, so every selected expert is among the logits >= T.  Those
-// candidates are ranked exactly; with more than kCandMax of them (mass ties) the warp falls
-// back to K rounds of arg-max.  cand_v / cand_i: kCandStride floats / ints each.
+// C candidates are ranked exactly: with C <= 32 one per lane, through shuffles; with
+// C <= kCandMax through shared memory; with more (mass ties) the warp falls back to K
+// rounds of arg-max.  cand_v / cand_i: kCandStride floats / ints each.
 __device__ void warp_topk(const float* logits, int E, int K, float* cand_v, int* cand_i, int lane, float& my_v,
                           int& my_i) {
   float v[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = (lane + 32 * i < E) ? ld_act(logits + lane + 32 * i) : -INFINITY;
+  for (int i = 0; i < 8; ++i) {
+    const int e0 = 128 * i + 4 * lane;
+    if ((E & 3) == 0 && e0 + 3 < E) {
+      const float4 f = ld_act4(logits + e0);
+      v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[4 * i + c] = (e0 + c < E) ? ld_act(logits + e0 + c) : -INFINITY;
+    }
+  }
   float lm = -INFINITY;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     if (v[i] != v[i]) v[i] = -INFINITY;  // NaN never outranks a number
-    if (lane + 32 * i < E) lm = fmaxf(lm, v[i]);
+    if (128 * (i >> 2) + 4 * lane + (i & 3) < E) lm = fmaxf(lm, v[i]);
   }
   int rank = 0;
 #pragma unroll
@@ -50,7 +61,7 @@ __device__ void warp_topk(const float* logits, int E, int K, float* cand_v, int*
   const float T = __shfl_sync(0xffffffffu, lm, __ffs(who) - 1);
   int cnt = 0;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) cnt += (lane + 32 * i < E && v[i] >= T);
+  for (int i = 0; i < 32; ++i) cnt += (128 * (i >> 2) + 4 * lane + (i & 3) < E && v[i] >= T);
   int incl = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -61,27 +72,42 @@ __device__ void warp_topk(const float* logits, int E, int K, float* cand_v, int*
   if (C <= kCandMax) {
     int w = incl - cnt;
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (lane + 32 * i < E && v[i] >= T) {
+    for (int i = 0; i < 32; ++i) {
+      const int e = 128 * (i >> 2) + 4 * lane + (i & 3);
+      if (e < E && v[i] >= T) {
         cand_v[w] = v[i];
-        cand_i[w] = lane + 32 * i;
+        cand_i[w] = e;
         ++w;
       }
-    __syncwarp();
-    // The rank of a candidate among the candidates is its rank among all experts.
-    for (int c = lane; c < C; c += 32) {
-      const float cv = cand_v[c];
-      const int ci = cand_i[c];
-      int r = 0;
-      for (int o = 0; o < C; ++o) r += better(cand_v[o], cand_i[o], cv, ci);
-      cand_i[kCandMax + c] = r;
     }
     __syncwarp();
-    for (int c = lane; c < C; c += 32) {
-      const int r = cand_i[kCandMax + c];
-      if (r < K) {
-        cand_v[2 * kCandMax + r] = cand_v[c];
-        cand_i[2 * kCandMax + r] = cand_i[c];
+    if (C <= 32) {  // one candidate per lane, ranked through shuffles
+      const float x = (lane < C) ? cand_v[lane] : -INFINITY;
+      const int xi = (lane < C) ? cand_i[lane] : 0x7FFFFFFF;  // empty lanes rank last
+      int r = 0;
+#pragma unroll
+      for (int o = 0; o < 32; ++o)
+        r += better(__shfl_sync(0xffffffffu, x, o), __shfl_sync(0xffffffffu, xi, o), x, xi);
+      if (lane < C && r < K) {
+        cand_v[2 * kCandMax + r] = x;
+        cand_i[2 * kCandMax + r] = xi;
+      }
+    } else {
+      // The rank of a candidate among the candidates is its rank among all experts.
+      for (int c = lane; c < C; c += 32) {
+        const float cv = cand_v[c];
+        const int ci = cand_i[c];
+        int r = 0;
+        for (int o = 0; o < C; ++o) r += better(cand_v[o], cand_i[o], cv, ci);
+        cand_i[kCandMax + c] = r;
+      }
+      __syncwarp();
+      for (int c = lane; c < C; c += 32) {
+        const int r = cand_i[kCandMax + c];
+        if (r < K) {
+          cand_v[2 * kCandMax + r] = cand_v[c];
+          cand_i[2 * kCandMax + r] = cand_i[c];
+        }
       }
     }
     __syncwarp();
@@ -95,12 +121,14 @@ __device__ void warp_topk(const float* logits, int E, int K, float* cand_v, int*
   uint32_t taken = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i)
-    if (lane + 32 * i >= E) taken |= 1u << i;
+    if (128 * (i >> 2) + 4 * lane + (i & 3) >= E) taken |= 1u << i;
   float lbv = -INFINITY;
   int lbi = 0x7fffffff;
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if (!((taken >> i) & 1u) && better(v[i], lane + 32 * i, lbv, lbi)) { lbv = v[i]; lbi = lane + 32 * i; }
+  for (int i = 0; i < 32; ++i) {
+    const int e = 128 * (i >> 2) + 4 * lane + (i & 3);
+    if (!((taken >> i) & 1u) && better(v[i], e, lbv, lbi)) { lbv = v[i]; lbi = e; }
+  }
   for (int j = 0; j < K; ++j) {
     float bv = lbv;
     int bi = lbi;
@@ -111,13 +139,16 @@ __device__ void warp_topk(const float* logits, int E, int K, float* cand_v, int*
       if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
     }
     if (lane == j) { my_v = bv; my_i = bi; }
-    if ((bi & 31) == lane) {
-      taken |= 1u << (bi >> 5);
+    if (((bi & 127) >> 2) == lane) {  // the winner's lane marks it taken
+      const int slot = 4 * (bi >> 7) + (bi & 3);
+      taken |= 1u << slot;
       lbv = -INFINITY;
       lbi = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (!((taken >> i) & 1u) && better(v[i], lane + 32 * i, lbv, lbi)) { lbv = v[i]; lbi = lane + 32 * i; }
+      for (int i = 0; i < 32; ++i) {
+        const int e = 128 * (i >> 2) + 4 * lane + (i & 3);
+        if (!((taken >> i) & 1u) && better(v[i], e, lbv, lbi)) { lbv = v[i]; lbi = e; }
+      }
     }
   }
 }
@@ -146,8 +177,10 @@ __device__ __forceinline__ bool last_cta_s(unsigned* counter, int* s_flag) {
 
 // Routing tables in global memory for the large-batch expert kernels (every thread of one
 // CTA): per-token top-k and gates, the union of selected experts in ascending order, and the
-// entries (token, slot) of each union expert in CSR form, tokens ascending.
-__device__ void topk_route(const LayerArgs& a, unsigned char* scratch) {
+// entries (token, slot) of each union expert in CSR form, tokens ascending.  selected: the
+// per-token top-k is already in ws.topk_idx / ws.topk_gate (and the caller's outputs), only
+// the tables remain.
+__device__ void topk_route(const LayerArgs& a, unsigned char* scratch, bool selected = false) {
   const int B = a.B, E = a.E, K = a.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   unsigned long long* mask = reinterpret_cast<unsigned long long*>(scratch);  // [1024] token bitmaps
@@ -160,7 +193,10 @@ __device__ void topk_route(const LayerArgs& a, unsigned char* scratch) {
   int* ci = reinterpret_cast<int*>(cv + kCandStride);
 
   for (int e = threadIdx.x; e < E; e += blockDim.x) mask[e] = 0ull;
-  for (int t = warp; t < B; t += nwarps) {
+  if (selected) {
+    for (int p = threadIdx.x; p < B * K; p += blockDim.x) sidx[p] = ld_act_i(&a.ws.topk_idx[p]);
+  }
+  for (int t = warp; t < B && !selected; t += nwarps) {
     float my_v = 0.f;
     int my_i = 0;
     warp_topk(a.ws.logits + (size_t)t * E, E, K, cv, ci, lane, my_v, my_i);

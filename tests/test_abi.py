@@ -98,17 +98,18 @@ def test_step_argument_checks():
             md.moe_decode_get_intermediate(h, 9, out, 16)
         md.moe_decode_step(h, 2, attn, res, out)
         assert md.moe_decode_sync_status(h) == 0
-        assert md.moe_decode_kernels_per_step(h, 1) == 1  # batch 1: one fused layer kernel
-        assert md.moe_decode_kernels_per_step(h, 2) == 3  # o_proj, router, small-M experts
+        assert md.moe_decode_kernels_per_step(h, 1) == 1  # batch 1: one layer kernel
+        assert md.moe_decode_kernels_per_step(h, 2) == 3  # batch 2: o_proj, router, small-M experts
         assert md.moe_decode_kernels_per_step(h, 4) == 4  # o_proj, router, gate/up, down
     finally:
         assert md.moe_decode_destroy(h) == 0
     assert md.moe_decode_destroy(h) == md.MOE_ERR_INVALID_ARG  # destroyed twice: rejected
-    for variant, per_b1 in ((1, 3), (2, 4)):  # unfused small-batch kernels; large-batch kernels
+    for variant, per_b in ((1, 3), (2, 4), (3, 1)):  # unfused small-batch; large-batch; counter-ordered
         h = md.moe_decode_create(md.config(dims.d, dims.d_o, dims.E, dims.k, dims.I, 4,
                                            force_variant=variant), w)
         try:
-            assert md.moe_decode_kernels_per_step(h, 1) == per_b1
+            assert md.moe_decode_kernels_per_step(h, 1) == per_b
+            assert md.moe_decode_kernels_per_step(h, 2) == per_b
         finally:
             assert md.moe_decode_destroy(h) == 0
 
@@ -140,5 +141,37 @@ def test_host_buffer_step_matches_device_step():
         st.md.moe_decode_step_host(st.h, 1, np.ascontiguousarray(case1["attn"]),
                                    np.ascontiguousarray(case1["resid"]), out1_h)
         assert np.array_equal(out1_h, out1_d)
+        # the same batch again (the cached graph with its staging copies), new inputs
+        case2 = build_case(seed + 2, synth.TINY, 3, checked=[0])
+        out2_d, idx2_d, gate2_d = st.step(case2["attn"], case2["resid"])
+        st.md.moe_decode_step_host(st.h, 3, np.ascontiguousarray(case2["attn"]),
+                                   np.ascontiguousarray(case2["resid"]), out_h, idx_h, gate_h)
+        assert np.array_equal(out_h, out2_d) and np.array_equal(idx_h, idx2_d) and np.array_equal(gate_h, gate2_d)
+    finally:
+        st.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B", [1, 2, 5])
+def test_host_buffer_step_two_layer_stack(B):
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import synth
+    from oracle.layer import build_case
+    from tests.harness import GpuStack
+    synth.build_device_fill()
+    seed = synth.config_seed(0) + 77 + B
+    st = GpuStack(seed, synth.TINY, n_layers=2, max_batch=8)
+    try:
+        case = build_case(seed, synth.TINY, B, n_layers=2, checked=[0])
+        out_d, idx_d, gate_d = st.step(case["attn"], case["resid"])
+        out_h = np.zeros((B, synth.TINY.d), np.uint16)
+        idx_h = np.zeros((2, B, synth.TINY.k), np.int32)
+        gate_h = np.zeros((2, B, synth.TINY.k), np.float32)
+        for _ in range(2):
+            st.md.moe_decode_step_host(st.h, B, np.ascontiguousarray(case["attn"]),
+                                       np.ascontiguousarray(case["resid"]), out_h, idx_h, gate_h)
+            assert np.array_equal(out_h, out_d) and np.array_equal(idx_h, idx_d) and np.array_equal(gate_h, gate_d)
     finally:
         st.close()

@@ -77,7 +77,7 @@ def test_tiny_b1():
 
 
 @pytest.mark.parametrize("B", [1, 2, 3, 5, 16, 64])
-@pytest.mark.parametrize("variant", [0, 1, 2])
+@pytest.mark.parametrize("variant", [0, 1, 2, 3])
 def test_tiny_batches_and_variants(B, variant):
     seed = synth.config_seed(0) + 100 * B
     st = H.GpuStack(seed, synth.TINY, max_batch=64, force_variant=variant)
@@ -218,6 +218,18 @@ def tp16():
 def test_tp16_b1(tp16):
     seed, st, ref = tp16
     check_case(st, build_case(seed, synth.TP16, 1, refs=[ref]))
+
+
+@pytest.mark.slow
+def test_tp16_b1_counter_ordered_kernel(tp16):
+    seed, _, ref = tp16
+    st = H.GpuStack(seed, synth.TP16, max_batch=2, force_variant=3, weights=H.device_weights(seed, synth.TP16, 1))
+    try:
+        check_case(st, build_case(seed, synth.TP16, 1, refs=[ref]))
+        attn0, resid0, _ = H.constructed_b2(seed, synth.TP16, 8, ref=ref)
+        check_case(st, build_case(seed, synth.TP16, 2, attn0=attn0, resid0=resid0, refs=[ref]))
+    finally:
+        st.close()
 
 
 @pytest.mark.slow

@@ -30,6 +30,7 @@ def _inputs(torch, seed, dims, B):
 # three small-batch kernels in both.
 @pytest.mark.parametrize("dims,B,variant", [(synth.TINY, 1, 0), (synth.TINY, 2, 0), (RAGGED, 1, 0),
                                             (RAGGED, 2, 0), (synth.TINY, 1, 1), (RAGGED, 1, 1),
+                                            (synth.TINY, 1, 3), (RAGGED, 2, 3),
                                             (synth.TP16, 1, 0), (synth.TP16, 2, 0)])
 def test_static_step_matches_step_twice(dims, B, variant):
     torch = _torch()
