@@ -117,7 +117,7 @@ cudaError_t launch_router_ks(const LayerArgs& a, int grid, cudaStream_t s, bool 
 // o_proj above batch 2 on the tensor cores with 2-D TMA tiles (kernels_tc.cu).
 bool oproj_tc_ok(const LayerArgs& a, int grid, size_t smem_optin);
 cudaError_t set_tc_attributes(size_t smem_optin);
-cudaError_t launch_oproj_tc(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_oproj_tc(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 
 // Expert kernels above batch 2 (kernels_large.cu): whole rows, tokens grouped per expert.
 bool plan_large(LayerArgs& a, int grid, size_t smem_optin);

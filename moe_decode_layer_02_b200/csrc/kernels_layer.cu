@@ -38,8 +38,11 @@
 #include <algorithm>
 #include <type_traits>
 
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.cuh"
+#include "mma.cuh"
 #include "rowdot.cuh"
 #include "topk.cuh"
 
@@ -47,8 +50,11 @@ namespace moe {
 
 namespace {
 
+constexpr int kRBox = 224;                // experts per W_r box (one 2-D tensor-map copy)
+constexpr int kRBoxBytes = kRBox * 128;   // 64 bf16 columns per expert
 constexpr int kPS = 2;       // gate/up row pairs per chunk
-constexpr int kDownLag = 1;  // rounds between an expert's last chunk and the use of its down block
+constexpr int kDownLag = 2;  // rounds between an expert's last chunk and the use of its down block
+constexpr int kDownPrefetch = 2;  // rounds ahead of its copy that a down block is prefetched into L2
 constexpr int kRPW = 4;      // output rows per consumer warp (rows per CTA <= 60)
 
 // Routing state of one CTA (shared memory).
@@ -60,6 +66,8 @@ struct alignas(16) Route2 {
   int U;
   int pad[3];
   float cand[2][2 * kCandStride];  // warp_topk scratch of the two routing warps
+  int dry_i[32];                   // outputs of the producer's warm-up pass
+  float dry_g[32];
 };
 
 // Shared-memory layout (byte offsets), the same on host and device.
@@ -74,9 +82,11 @@ __host__ __device__ inline size_t up128(size_t x) { return (x + 127) & ~size_t(1
 __host__ __device__ inline Smem2 smem2(int NT, const LayerArgs& a) {
   Smem2 L;
   const size_t orow = (size_t)a.d_o * 2, row = (size_t)a.d * 2;
-  const int RM = a.k1.rows_max, RMr = a.k2.rows_max;
+  const int RM = a.k1.rows_max;
+  // an O-ring stage holds W_o rows or one W_r box (1024-aligned for the 128-byte swizzle)
   L.so_b = up128((size_t)a.k1.rows_per_stage * orow);
-  if (L.so_b < up128(row)) L.so_b = up128(row);
+  if (L.so_b < (size_t)kRBoxBytes) L.so_b = kRBoxBytes;
+  L.so_b = (L.so_b + 1023) & ~size_t(1023);
   L.sp_b = up128((size_t)2 * kPS * row);
   L.sd_b = up128((size_t)RM * a.I * 2);
   L.pring = 0;
@@ -84,7 +94,7 @@ __host__ __device__ inline Smem2 smem2(int NT, const LayerArgs& a) {
   size_t region = (size_t)a.k1.stages * L.so_b;
   if (L.dring + (size_t)a.k4.stages * L.sd_b > region) region = L.dring + (size_t)a.k4.stages * L.sd_b;
   size_t pf = (size_t)RM * kCW * NT;                               // o_proj partials
-  if ((size_t)RMr * kCW * NT > pf) pf = (size_t)RMr * kCW * NT;    // router partials
+  if ((size_t)NT * 64 > pf) pf = (size_t)NT * 64;                 // h * gamma of the router columns
   if ((size_t)2 * 2 * kPS * kCW * NT > pf) pf = (size_t)2 * 2 * kPS * kCW * NT;  // chunk partials
   L.part = region;
   L.sq = L.part + up128(pf * 4);
@@ -92,7 +102,7 @@ __host__ __device__ inline Smem2 smem2(int NT, const LayerArgs& a) {
   L.route = L.hs + up128((size_t)NT * RM * 4);
   L.bars = L.route + up128(sizeof(Route2));
   L.misc = L.bars + (6 * kMaxStages + 2 + kMaxUnion + 4) * 8;
-  L.total = L.misc + 64;
+  L.total = L.misc + 64 + 1024;  // + alignment of the dynamic shared memory to 1024
   return L;
 }
 
@@ -125,23 +135,24 @@ __device__ __forceinline__ void grid_barrier2(unsigned* count, unsigned target, 
   csync();
 }
 
-// Top-k and gates of token t by one warp into rt->sel_*[t] (and the caller's outputs in CTA 0).
-__device__ __forceinline__ void route_token(const LayerArgs& a, int t, Route2* rt, int lane, bool write_user) {
+// Top-k and gates of one token by one warp: lane j < K writes the j-th selection (descending
+// logit) and its gate to sel_i / sel_g, and to the caller's outputs when given.  Not inlined,
+// so one copy of the code serves every call: the producer warp runs it once on stale data
+// during the o_proj tail (its instructions are then resident when the real selection runs
+// right after barrier 2, where every SM would otherwise fetch them cold at the same moment).
+__device__ __noinline__ void route_token(const float* logits, int E, int K, float* cand, int* sel_i, float* sel_g,
+                                         int* user_idx, float* user_gate, uint32_t* err, int lane) {
   float my_v = 0.f;
   int my_i = 0;
-  float* cv = rt->cand[t];
-  warp_topk(a.ws.logits + (size_t)t * a.E, a.E, a.k, cv, reinterpret_cast<int*>(cv + kCandStride), lane, my_v,
-            my_i);
-  const float g = warp_gate(my_v, lane, a.k);
-  if (lane < a.k) {
-    const int e = (my_i >= 0 && my_i < a.E) ? my_i : 0;
-    if (e != my_i) atomicOr(a.ws.err, kErrBounds);
-    rt->sel_i[t][lane] = e;
-    rt->sel_g[t][lane] = g;
-    if (write_user) {
-      if (a.user_idx) a.user_idx[t * a.k + lane] = e;
-      if (a.user_gate) a.user_gate[t * a.k + lane] = g;
-    }
+  warp_topk(logits, E, K, cand, reinterpret_cast<int*>(cand + kCandStride), lane, my_v, my_i);
+  const float g = warp_gate(my_v, lane, K);
+  if (lane < K) {
+    const int e = (my_i >= 0 && my_i < E) ? my_i : 0;
+    if (e != my_i && err) atomicOr(err, kErrBounds);
+    sel_i[lane] = e;
+    sel_g[lane] = g;
+    if (user_idx) user_idx[lane] = e;
+    if (user_gate) user_gate[lane] = g;
   }
   __syncwarp();
 }
@@ -167,13 +178,13 @@ __device__ __forceinline__ float rstd_of(const LayerArgs& a, int t, int G, int l
 }  // namespace
 
 template <int NT, int CPLX, int EPL>
-__global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const LayerArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
+__global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const __grid_constant__ CUtensorMap tmR, const LayerArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int CPLO = kCPLf;
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, d_o = a.d_o, I = a.I, B = a.B, E = a.E;
   const int SO = a.k1.stages, RS = a.k1.rows_per_stage, RM = a.k1.rows_max;
-  const int RSr = a.k2.rows_per_stage;
   const int SP = a.k3.stages, SD = a.k4.stages;
   const uint32_t orow_bytes = (uint32_t)d_o * 2u, row_bytes = (uint32_t)d * 2u, drow_bytes = (uint32_t)I * 2u;
   const Smem2 L = smem2(NT, a);
@@ -181,7 +192,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const LayerArgs a) {
   split_range(d, G, c, lo, hi);
   const int i0 = (int)lo, nrows = (int)(hi - lo);  // o_proj rows = output rows
   split_range(E, G, c, lo, hi);
-  const int e0 = (int)lo, nr = (int)(hi - lo);      // router rows
+  const int e0 = (int)lo, nr = (int)(hi - lo);      // experts whose logits this CTA finishes
+  const int x0 = i0 & ~7, nbox = (E + kRBox - 1) / kRBox;  // W_r columns [x0, x0 + 64) in boxes
 
   unsigned char* ring = smem;
   float* part = reinterpret_cast<float*>(smem + L.part);
@@ -239,12 +251,13 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const LayerArgs a) {
         mbar_arrive_expect_tx(&fullO[s], n * orow_bytes);
         bulk_g2s(ring + s * L.so_b, a.w_o + (size_t)r * d_o, n * orow_bytes, &fullO[s], pol);
       }
-      for (int j = 0; j < nr && !*abort_flag; j += RSr, ++itO) {
-        const int n = min(RSr, nr - j);
+      // W_r[:, x0 .. x0 + 64) for every expert, one box of kRBox experts per stage (columns past
+      // d and experts past E read as zeros)
+      for (int j = 0; j < nbox && !*abort_flag; ++j, ++itO) {
         if (!ring_acquire(emptyO, itO, SO, abort_flag, err)) break;
         const int s = itO % SO;
-        mbar_arrive_expect_tx(&fullO[s], n * row_bytes);
-        bulk_g2s(ring + s * L.so_b, a.w_r + (size_t)(e0 + j) * d, n * row_bytes, &fullO[s], pol);
+        mbar_arrive_expect_tx(&fullO[s], (uint32_t)kRBoxBytes);
+        tma_load_2d(ring + s * L.so_b, &tmR, x0, j * kRBox, &fullO[s]);
       }
       if (a.pf_w_o) {  // next layer: what the same CTA reads first, into L2
         if (nr > 0) bulk_prefetch_l2(a.pf_w_r + (size_t)e0 * d, nr * row_bytes);
@@ -259,16 +272,21 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const LayerArgs a) {
         }
       }
     }
+    __syncwarp();
+    // warm-up pass of the selection code on whatever the logits buffer holds (nothing is
+    // written outside this CTA's shared memory)
+    route_token(a.ws.logits, E, a.k, rt->cand[0], rt->dry_i, rt->dry_g, nullptr, nullptr, nullptr, lane);
     pdl_wait();  // the previous kernel (counters, logits of an earlier launch) is complete
     if (lane == 0) {
-      // every O-ring fill has landed and been read (the router rows, before barrier 2), so
-      // the region may take the expert rings
+      // every O-ring fill has landed and been read (the W_r boxes, before barrier 1), so the
+      // region may take the expert rings
       ring_drain(fullO, itO, SO, err);
       for (int i = itO - SO < 0 ? 0 : itO - SO; i < itO; ++i) mbar_drain(&emptyO[i % SO], (i / SO) & 1, err);
     }
     __syncwarp();
     warp_wait_count(bar_count, 2u * (unsigned)G, abort_flag, err);  // barrier 2: every logit written
-    route_token(a, 0, rt, lane, c == 0);
+    route_token(a.ws.logits, E, a.k, rt->cand[0], rt->sel_i[0], rt->sel_g[0], c == 0 ? a.user_idx : nullptr,
+                c == 0 ? a.user_gate : nullptr, err, lane);
     if (B == 2) mbar_wait(tok1_ready, 0, abort_flag, err);  // every lane: token 1's selection
     // union: token 0's selections in rank order, then token 1's experts that token 0 lacks
     const int K = a.k;
@@ -304,24 +322,22 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const LayerArgs a) {
     if (lane == 0) {
       rt->U = U;
       mbar_arrive(route_ready);  // releases the routing state to the consumers
-      // ---- expert phase: copies in the consumers' order ----
-      const int Z = U * cpe, Mc = (Z > c) ? (Z - c + G - 1) / G : 0;
-      const uint32_t blk = (uint32_t)nrows * drow_bytes;
-      int itP = 0, itD = 0, nu = 0;
-      bool ok = true;
-      auto issue_down = [&](int u) {
-        if (nrows == 0 || !ok) return;
-        if (!ring_acquire(emptyD, itD, SD, abort_flag, err)) {
-          ok = false;
-          return;
-        }
-        const int s = itD % SD;
-        mbar_arrive_expect_tx(&fullD[s], blk);
-        bulk_g2s(ring + L.dring + s * L.sd_b, a.w_down + ((size_t)rt->un_e[u] * d + i0) * I, blk, &fullD[s], pol);
-        ++itD;
+    }
+    // ---- expert phase: lane 0 streams the gate/up chunks (and sends down blocks to L2 ahead
+    // of their turn), lane 1 streams the down blocks into their own ring, each in the order the
+    // consumers use them; the two rings are independent, so neither stream waits on the other.
+    const int Z = U * cpe, Mc = (Z > c) ? (Z - c + G - 1) / G : 0;
+    const uint32_t blk = (uint32_t)nrows * drow_bytes;
+    if (lane == 0) {
+      int itP = 0, npf = 0;
+      auto prefetch_down = [&](int upto_round) {
+        for (; npf < U && nrows > 0 && down_round(npf, cpe, G) <= upto_round; ++npf)
+          bulk_prefetch_l2(a.w_down + ((size_t)rt->un_e[npf] * d + i0) * I, blk);
       };
-      for (int m = 0; m < Mc && ok; ++m) {
+      prefetch_down(kDownPrefetch - 1);
+      for (int m = 0; m < Mc; ++m) {
         const int z = c + m * G, u = z / cpe, t0 = (z - u * cpe) * kPS;
+        prefetch_down(m + kDownPrefetch);
         if (!ring_acquire(emptyP, itP, SP, abort_flag, err)) break;
         const int s = itP % SP;
         const uint16_t* g_rows = a.w_gu + ((size_t)rt->un_e[u] * 2 * I + t0) * d;
@@ -330,10 +346,17 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const LayerArgs a) {
         bulk_g2s(ring + L.pring + s * L.sp_b + (size_t)kPS * row_bytes, g_rows + (size_t)I * d, kPS * row_bytes,
                  &fullP[s], pol);
         ++itP;
-        while (nu < U && down_round(nu, cpe, G) <= m) issue_down(nu++);
       }
-      while (nu < U) issue_down(nu++);
+      prefetch_down(1 << 30);
       ring_drain(fullP, itP, SP, err);
+    } else if (lane == 1 && nrows > 0) {
+      int itD = 0;
+      for (int u = 0; u < U; ++u, ++itD) {
+        if (!ring_acquire(emptyD, itD, SD, abort_flag, err)) break;
+        const int s = itD % SD;
+        mbar_arrive_expect_tx(&fullD[s], blk);
+        bulk_g2s(ring + L.dring + s * L.sd_b, a.w_down + ((size_t)rt->un_e[u] * d + i0) * I, blk, &fullD[s], pol);
+      }
       ring_drain(fullD, itD, SD, err);
     }
     return;
@@ -400,10 +423,87 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const LayerArgs a) {
     ss = warp_sum(ss);
     if (lane == 0) a.ws.ss_part[(size_t)c * a.maxB + warp] = ss;
   }
+  // Router, split over K: logits[t][e] = rstd[t] * sum_i W_r[e][i] (h[t][i] gamma[i]); this
+  // CTA's share is the sum over its own rows i in [i0, i0 + nrows), for every expert, formed
+  // here before barrier 1 (it needs no other CTA's h).  h * gamma of columns x0 .. x0 + 63
+  // (zero outside the CTA's rows) goes to shared memory (the o_proj partials are spent).
+  float* hg = part;  // [NT][64]
+  for (int z = tid; z < NT * 64; z += kCT) {
+    const int t = z >> 6, k = z & 63, i = x0 + k;
+    hg[z] = (t < B && i >= i0 && i < i0 + nrows) ? hs[(i - i0) * NT + t] * bf16f(a.gamma[i]) : 0.f;
+  }
+  csync();
+  {
+    for (int j = 0; j < nbox; ++j) mbar_wait(&fullO[(itO + j) % SO], ((itO + j) / SO) & 1, abort_flag, err);
+    const int Bp = (a.maxB + 7) & ~7;
+    float* P = a.ws.rpart + (size_t)c * E * Bp;  // [E][Bp]: this CTA's partial logits
+#pragma unroll 1
+    for (int e = tid; e < E; e += kCT) {
+      const int j = e / kRBox, r = e - j * kRBox;
+      const unsigned char* tile = ring + ((itO + j) % SO) * L.so_b;
+      float acc[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+#pragma unroll 1
+      for (int q = 0; q < 8; ++q) {
+        float w[8];
+        unpack8f(*reinterpret_cast<const uint4*>(tile + swz(r, q)), w);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const float4 g0 = *reinterpret_cast<const float4*>(hg + t * 64 + 8 * q);
+          const float4 g1 = *reinterpret_cast<const float4*>(hg + t * 64 + 8 * q + 4);
+          acc[t] = fmaf(w[0], g0.x, acc[t]); acc[t] = fmaf(w[1], g0.y, acc[t]);
+          acc[t] = fmaf(w[2], g0.z, acc[t]); acc[t] = fmaf(w[3], g0.w, acc[t]);
+          acc[t] = fmaf(w[4], g1.x, acc[t]); acc[t] = fmaf(w[5], g1.y, acc[t]);
+          acc[t] = fmaf(w[6], g1.z, acc[t]); acc[t] = fmaf(w[7], g1.w, acc[t]);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < NT; ++t) P[(size_t)e * Bp + t] = acc[t];
+    }
+    __syncwarp();
+    if (lane == 0)
+      for (int j = 0; j < nbox; ++j) mbar_arrive(&emptyO[(itO + j) % SO]);
+  }
   grid_barrier2(bar_count, (unsigned)G, abort_flag, err);
 
-  // ---- router: x = h * rstd * gamma (kept in registers), logits of this CTA's rows ----
+  // ---- after barrier 1: logits of this CTA's experts, then x = h * rstd * gamma ----
   float x[NT][CPLX][8];
+  {
+    // one warp per (expert, token): lanes sum the CTAs' partials in a fixed lane-strided order,
+    // then a butterfly (the loads of all lanes are in flight together)
+    const int Bp = (a.maxB + 7) & ~7;
+    for (int z = warp; z < nr * NT; z += kCW) {
+      const int e = e0 + z / NT, t = z % NT;
+      float sacc = 0.f, ss = 0.f;  // the partials and, in the same round trips, the sums of h^2
+      for (int c0 = 0; c0 < G; c0 += 8 * 32) {
+        float pv[8], qv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int cc = c0 + k * 32 + lane;
+          pv[k] = cc < G ? ld_act(a.ws.rpart + ((size_t)cc * E + e) * Bp + t) : 0.f;
+          qv[k] = cc < G ? ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          sacc += pv[k];
+          ss += qv[k];
+        }
+      }
+      sacc = warp_sum(sacc);
+      ss = warp_sum(ss);  // the fixed-order sum of rstd_of: the same rstd bits everywhere
+      const float r = 1.0f / sqrtf(ss / (float)a.d + a.eps);
+      if (lane == 0) a.ws.logits[(size_t)t * E + e] = r * sacc;
+    }
+  }
+  grid_arrive(bar_count);  // barrier 2: the producer warps wait for it
+  if (NT == 2 && warp == 1) {  // token 1's selection, in parallel with the producer's token 0
+    warp_wait_count(bar_count, 2u * (unsigned)G, abort_flag, err);
+    route_token(a.ws.logits + E, E, a.k, rt->cand[1], rt->sel_i[1], rt->sel_g[1],
+                c == 0 && a.user_idx ? a.user_idx + a.k : nullptr, c == 0 && a.user_gate ? a.user_gate + a.k : nullptr,
+                err, lane);
+    if (lane == 0) mbar_arrive(tok1_ready);
+  }
   {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
@@ -439,40 +539,6 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const LayerArgs a) {
         }
       }
     }
-    // the router rows' fills (landed during the o_proj tail), then passes of 8 / NT rows
-    const int itR = itO, nfr = (nr + RSr - 1) / RSr;
-    for (int f = 0; f < nfr; ++f) mbar_wait(&fullO[(itR + f) % SO], ((itR + f) / SO) & 1, abort_flag, err);
-    constexpr int kRI = 8 / NT;
-    for (int j0 = 0; j0 < nr; j0 += kRI) {
-      const uint16_t* rp[kRI];
-#pragma unroll
-      for (int k = 0; k < kRI; ++k) {
-        const int j = min(j0 + k, nr - 1), f = j / RSr;
-        rp[k] = reinterpret_cast<const uint16_t*>(ring + ((itR + f) % SO) * L.so_b) + (size_t)(j - f * RSr) * d;
-      }
-      float v[kRI * NT];
-      rows_dot<NT, kRI>(rp, nr - j0, x, qbase, qpw, lane, v);
-      const float tot = warp_reduce_multi<kRI * NT>(v, lane);
-      const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
-      if (multi_writer<kRI * NT>(lane) && j < nr) part[(j * kCW + warp) * NT + t] = tot;
-    }
-    __syncwarp();
-    if (lane == 0)
-      for (int f = 0; f < nfr; ++f) mbar_arrive(&emptyO[(itR + f) % SO]);
-    csync();
-    for (int z = tid; z < nr * B; z += kCT) {
-      const int j = z / B, t = z % B;
-      float sacc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kCW; ++w) sacc += part[(j * kCW + w) * NT + t];
-      a.ws.logits[(size_t)t * E + e0 + j] = sacc;
-    }
-  }
-  grid_arrive(bar_count);  // barrier 2: the producer warps wait for it
-  if (NT == 2 && warp == 0) {  // token 1's selection, in parallel with the producer's token 0
-    warp_wait_count(bar_count, 2u * (unsigned)G, abort_flag, err);
-    route_token(a, 1, rt, lane, c == 0);
-    if (lane == 0) mbar_arrive(tok1_ready);
   }
   mbar_wait(route_ready, 0, abort_flag, err);
   const int U = rt->U;
@@ -649,15 +715,14 @@ bool plan_layer2(LayerArgs& a, int G, size_t optin) {
   if (a.B < 1 || a.B > 2 || a.k > 32 || a.E > 1024 || a.I % 32 || a.I / 32 > 16) return false;
   if ((long long)a.d > 8LL * 32 * kCPLf * kCW || (long long)a.d_o > 8LL * 32 * kCPLf * kCW) return false;
   const int NT = a.B;
-  const size_t budget = optin - 1024 - 256;
+  const size_t budget = optin - 256;
   KTune& o = a.k1;
-  KTune& r = a.k2;
   KTune& p = a.k3;
   KTune& dn = a.k4;
-  const size_t orow = (size_t)a.d_o * 2, row = (size_t)a.d * 2;
+  const size_t orow = (size_t)a.d_o * 2;
   o.rows_max = (a.d + G - 1) / G;
-  if (o.rows_max > kRPW * kCW) return false;
-  r.rows_max = (a.E + G - 1) / G;
+  // rows per CTA: at most kRPW per consumer warp, and inside one 64-column W_r box from x0
+  if (o.rows_max > kRPW * kCW || o.rows_max > 57) return false;
   o.rows_per_stage = (int)std::max<size_t>(1, std::min<size_t>(32768 / orow, (size_t)o.rows_max));
   p.rows_per_stage = kPS;
   dn.rows_max = o.rows_max;
@@ -667,28 +732,31 @@ bool plan_layer2(LayerArgs& a, int G, size_t optin) {
   const size_t fixed = L0.total;  // region 0
   if (fixed >= budget) return false;
   const size_t cap = budget - fixed;
-  r.rows_per_stage = (int)(L0.so_b / row);
   o.stages = (int)std::min<size_t>(kMaxStages, cap / L0.so_b);
-  if (o.stages < 2 || (r.rows_max + r.rows_per_stage - 1) / r.rows_per_stage > o.stages) return false;
+  if (o.stages < 2 || (a.E + kRBox - 1) / kRBox > o.stages) return false;  // every W_r box resident at once
   dn.stages = 3;
   if ((size_t)dn.stages * L0.sd_b >= cap) return false;
   p.stages = (int)std::min<size_t>(kMaxStages, (cap - (size_t)dn.stages * L0.sd_b) / L0.sp_b);
   if (p.stages < 2) return false;
   const Smem2 L = smem2(NT, a);
   o.smem = L.total;
-  r.smem = p.smem = dn.smem = o.smem;
+  p.smem = dn.smem = o.smem;
   return o.smem <= budget;
 }
 
 bool layer2_ok(const LayerArgs& a0, size_t optin) {
   LayerArgs a = a0;
-  return plan_layer2(a, 148, optin);
+  CUtensorMap probe;
+  return plan_layer2(a, 148, optin) &&
+         make_map_2d(&probe, a.w_r ? a.w_r : reinterpret_cast<const uint16_t*>(256), (uint64_t)a.d, (uint64_t)a.E,
+                     64, kRBox);
 }
 
 namespace {
 
 template <typename Kern>
-cudaError_t launch_coop(Kern k, int grid, size_t smem, cudaStream_t s, bool pdl, const LayerArgs& a) {
+cudaError_t launch_coop(Kern k, int grid, size_t smem, cudaStream_t s, bool pdl, const CUtensorMap& tmR,
+                        const LayerArgs& a) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreadsS);
@@ -706,15 +774,15 @@ cudaError_t launch_coop(Kern k, int grid, size_t smem, cudaStream_t s, bool pdl,
   ++n;
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, k, a);
+  return cudaLaunchKernelEx(&cfg, k, tmR, a);
 }
 
 template <int NT, int CPLX>
-cudaError_t launch_by_epl(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
+cudaError_t launch_by_epl(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, const CUtensorMap& tmR) {
   const int epl = a.I / 32;
-  if (epl == 4) return launch_coop(k_layer2<NT, CPLX, 4>, grid, a.k1.smem, s, pdl, a);
-  if (epl == 8) return launch_coop(k_layer2<NT, CPLX, 8>, grid, a.k1.smem, s, pdl, a);
-  return launch_coop(k_layer2<NT, CPLX, 0>, grid, a.k1.smem, s, pdl, a);
+  if (epl == 4) return launch_coop(k_layer2<NT, CPLX, 4>, grid, a.k1.smem, s, pdl, tmR, a);
+  if (epl == 8) return launch_coop(k_layer2<NT, CPLX, 8>, grid, a.k1.smem, s, pdl, tmR, a);
+  return launch_coop(k_layer2<NT, CPLX, 0>, grid, a.k1.smem, s, pdl, tmR, a);
 }
 
 }  // namespace
@@ -722,9 +790,12 @@ cudaError_t launch_by_epl(const LayerArgs& a, int grid, cudaStream_t s, bool pdl
 cudaError_t launch_layer2(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   LayerArgs a = a0;
   if (!plan_layer2(a, grid, optin)) return cudaErrorInvalidConfiguration;
+  CUtensorMap tmR;  // W_r [E][d]: boxes of 64 columns x kRBox experts
+  if (!make_map_2d(&tmR, a.w_r, (uint64_t)a.d, (uint64_t)a.E, 64, kRBox)) return cudaErrorInvalidValue;
   const bool small_x = a.d <= 8 * 32 * 2 * kCW;  // two 8-element chunks per lane cover d
-  if (a.B == 1) return small_x ? launch_by_epl<1, 2>(a, grid, s, pdl) : launch_by_epl<1, 3>(a, grid, s, pdl);
-  return small_x ? launch_by_epl<2, 2>(a, grid, s, pdl) : launch_by_epl<2, 3>(a, grid, s, pdl);
+  if (a.B == 1)
+    return small_x ? launch_by_epl<1, 2>(a, grid, s, pdl, tmR) : launch_by_epl<1, 3>(a, grid, s, pdl, tmR);
+  return small_x ? launch_by_epl<2, 2>(a, grid, s, pdl, tmR) : launch_by_epl<2, 3>(a, grid, s, pdl, tmR);
 }
 
 cudaError_t set_layer2_attributes(size_t optin) {

@@ -8,11 +8,13 @@
 //      map, boxes of 224 experts x 64 columns, 128-byte swizzle; columns outside [r0, r1) meet
 //      zeros below), issued before the dependency wait since W_r is static;
 //   2. consumers compute rstd of every token (the same fixed-order sum as every other kernel),
-//      write x for their slice, and place h * gamma of the slice, split into bf16 hi + lo
-//      (exact to 2^-17 of the fp32 value), in two swizzled tiles;
-//   3. the tensor cores (mma.sync m16n8k16, experts as M, tokens as N, hi and lo into the same
-//      fp32 accumulator over the 64 columns) give the CTA's partial logits of every expert and
-//      token, stored to a per-CTA slab;
+//      write x for their slice, and place h * gamma of the slice, split into three bf16 terms
+//      hi + mid + lo (together within 2^-26 of the fp32 value; two terms leave 2^-18, which
+//      over d = 8192 columns moves a logit by ~1e-5), in three swizzled tiles;
+//   3. the tensor cores (mma.sync m16n8k16, experts as M, tokens as N; each term's 16-column
+//      product in a fresh accumulator, summed in fp32 on the CUDA cores so that the tensor
+//      core's own accumulation never carries a long sum) give the CTA's partial logits of
+//      every expert and token, stored to a per-CTA slab;
 //   4. grid barrier; CTA c sums its 6-7 experts' partials over the CTAs in a fixed order and
 //      scales by rstd (the logits);
 //   5. grid barrier; CTA t (t < B) selects token t's top-k and gates; the last CTA to finish
@@ -50,7 +52,7 @@ __host__ __device__ inline size_t rk_smem(int E) {
   size_t w = (size_t)rk_boxes(E) * kRkBoxBytes;
   if (w < (size_t)kTopkScratch) w = kTopkScratch;
   w = (w + 1023) & ~size_t(1023);
-  return 1024 + w + 2 * kRkTileBytes + 64 * 4 + 64;
+  return 1024 + w + 3 * kRkTileBytes + 64 * 4 + 64;
 }
 
 // Fixed-order RMS statistics (the same sum as the other router kernels).
@@ -106,7 +108,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
   wbytes = (wbytes + 1023) & ~size_t(1023);
   unsigned char* wr = smem;
   unsigned char* th = smem + wbytes;       // h * gamma, bf16 hi  [64 tokens][64 columns], swizzled
-  unsigned char* tl = th + kRkTileBytes;   // bf16 lo
+  unsigned char* tm = th + kRkTileBytes;   // bf16 mid
+  unsigned char* tl = tm + kRkTileBytes;   // bf16 lo
   float* rstd_s = reinterpret_cast<float*>(tl + kRkTileBytes);
   uint64_t* bar = reinterpret_cast<uint64_t*>(rstd_s + 64);
   int* s_misc = reinterpret_cast<int*>(bar + 1);
@@ -152,9 +155,12 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
         a.ws.x[(size_t)t * d + i] = hv * rstd_s[t] * g;
       }
       const __nv_bfloat16 vh = __float2bfloat16_rn(v);
-      const __nv_bfloat16 vl = __float2bfloat16_rn(v - __bfloat162float(vh));
+      const float r1 = v - __bfloat162float(vh);
+      const __nv_bfloat16 vm = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 vl = __float2bfloat16_rn(r1 - __bfloat162float(vm));
       const uint32_t off = swz(t, k >> 3) + (uint32_t)(k & 7) * 2;
       *reinterpret_cast<__nv_bfloat16*>(th + off) = vh;
+      *reinterpret_cast<__nv_bfloat16*>(tm + off) = vm;
       *reinterpret_cast<__nv_bfloat16*>(tl + off) = vl;
     }
     csync();
@@ -165,14 +171,15 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
       const int arow = ((ai & 1) << 3) + (lane & 7), achk = ai >> 1;      // A: expert +8 (i & 1), chunk +(i >> 1)
       const int brow0 = ((ai >> 1) << 3) + (lane & 7), bchk = ai & 1;     // B: token tile +(i >> 1), chunk +(i & 1)
       const int g = lane >> 2, q = lane & 3;
-      const uint32_t hbase = smem_addr(th), lbase = smem_addr(tl);
+      const uint32_t hbase = smem_addr(th), mbase = smem_addr(tm), lbase = smem_addr(tl);
       float* P = a.ws.rpart + (size_t)c * E * Bp;
       const int nmt = (E + 15) / 16, ntp = (B + 15) / 16;
       for (int np = 0; np < ntp; ++np) {
-        uint32_t bh[4][4], bl[4][4];
+        uint32_t bh[4][4], bm[4][4], bl[4][4];
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           ldsm4(bh[kk], hbase + swz(16 * np + brow0, 2 * kk + bchk));
+          ldsm4(bm[kk], mbase + swz(16 * np + brow0, 2 * kk + bchk));
           ldsm4(bl[kk], lbase + swz(16 * np + brow0, 2 * kk + bchk));
         }
         for (int mt = warp; mt < nmt; mt += kCW) {
@@ -183,10 +190,18 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
           for (int kk = 0; kk < 4; ++kk) {
             uint32_t af[4];
             ldsm4(af, wt + swz(rb + arow, 2 * kk + achk));
-            mma16816(d0, af, bh[kk][0], bh[kk][1]);
-            mma16816(d0, af, bl[kk][0], bl[kk][1]);
-            mma16816(d1, af, bh[kk][2], bh[kk][3]);
-            mma16816(d1, af, bl[kk][2], bl[kk][3]);
+            // each term's 16-column product in a fresh accumulator, summed in fp32:
+            // (hi + (mid + lo)) per k-step, k-steps in order
+#pragma unroll
+            for (int tile = 0; tile < 2; ++tile) {
+              float ph[4] = {0.f, 0.f, 0.f, 0.f}, pm[4] = {0.f, 0.f, 0.f, 0.f}, pl[4] = {0.f, 0.f, 0.f, 0.f};
+              mma16816(ph, af, bh[kk][2 * tile], bh[kk][2 * tile + 1]);
+              mma16816(pm, af, bm[kk][2 * tile], bm[kk][2 * tile + 1]);
+              mma16816(pl, af, bl[kk][2 * tile], bl[kk][2 * tile + 1]);
+              float* dd = tile ? d1 : d0;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) dd[e] += ph[e] + (pm[e] + pl[e]);
+            }
           }
           // D: lane (g, q) holds experts 16 mt + g (+8), tokens 2q, 2q + 1 of each token tile
 #pragma unroll

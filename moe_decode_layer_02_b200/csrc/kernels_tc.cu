@@ -32,19 +32,28 @@ constexpr int kTcBK = 64;        // K of one k-block (128 bytes of bf16: one swi
 constexpr int kTcKB = 4;         // k-blocks per stage: 256 of K per pair of TMA copies
 constexpr int kTcRows = 56;      // weight rows per box (a CTA owns at most 49; 56 keeps tiles 1024-aligned)
 constexpr int kTcTok = 64;       // most token rows per activation box
-constexpr int kTcStages = 3;
+constexpr int kTcMaxStages = 8;
 constexpr int kTcWTile = kTcRows * kTcBK * 2;          // 7168 bytes per weight k-block tile
 constexpr int kTcAOff = kTcKB * kTcWTile;              // 28672: activation tiles follow
-constexpr int kTcStageBytes = kTcAOff + kTcKB * kTcTok * kTcBK * 2;  // 61440
+constexpr size_t kTcFixed = 1024 + (size_t)kTcTok * kTcRows * 4 + 2 * kTcMaxStages * 8 + 64;
+
+// A stage holds the weight tiles and tokb activation rows per k-block, rounded up to 1 KB for
+// the swizzle; as many stages as fit the shared memory keep W_o in flight (5 at 16 tokens,
+// 3 at 64).
+int tc_stage_bytes(int tokb) { return (kTcAOff + kTcKB * tokb * kTcBK * 2 + 1023) & ~1023; }
+int tc_stages(int tokb, size_t optin) {
+  const size_t room = optin > kTcFixed ? optin - kTcFixed : 0;
+  return std::min<int>(kTcMaxStages, (int)(room / (size_t)tc_stage_bytes(tokb)));
+}
 
 }  // namespace
 
 // Tensor maps view W_o [d][d_o] and attn_out [B][d_o] as 3-D {64 (k), rows, d_o / 64
 // (k-block)} so one copy brings four 64-wide k-blocks of 56 weight rows (28 KB) or of the
-// tokens; tokb = the activation box height (B rounded up to 16).
+// tokens; tokb = the activation box height (B rounded up to 16); NS stages of sb bytes each.
 __global__ void __launch_bounds__(kThreads, 1)
     k_oproj_tc(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA, const LayerArgs a,
-               int tokb) {
+               int tokb, int NS, int sb) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = gridDim.x, c = blockIdx.x;
@@ -55,16 +64,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = (d_o + kTcKB * kTcBK - 1) / (kTcKB * kTcBK);
   const uint32_t stage_tx = (uint32_t)(kTcAOff + kTcKB * tokb * kTcBK * 2);
 
-  unsigned char* ring = smem;                                                      // [S][60 KB]
-  float* sq = reinterpret_cast<float*>(ring + (size_t)kTcStages * kTcStageBytes);  // [kTcTok][kTcRows]
+  unsigned char* ring = smem;                                          // [NS][sb]
+  float* sq = reinterpret_cast<float*>(ring + (size_t)NS * sb);        // [kTcTok][kTcRows]
   uint64_t* full = reinterpret_cast<uint64_t*>(sq + kTcTok * kTcRows);
-  uint64_t* empty = full + kTcStages;
-  int* s_misc = reinterpret_cast<int*>(empty + kTcStages);
+  uint64_t* empty = full + NS;
+  int* s_misc = reinterpret_cast<int*>(empty + NS);
   volatile int* abort_flag = s_misc;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   if (tid == 0) {
-    init_ring(full, empty, kTcStages);
+    init_ring(full, empty, NS);
     s_misc[0] = 0;
     fence_barrier_init();
   }
@@ -75,23 +84,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       // W_o is static: the first stages' weight copies go out before the dependency wait; the
       // activation copies (attn_out comes from the previous kernel) only after it.
-      const int pre = nk < kTcStages ? nk : kTcStages;
+      const int pre = nk < NS ? nk : NS;
       for (int ks = 0; ks < pre; ++ks) {
         mbar_arrive_expect_tx(&full[ks], stage_tx);
-        tma_load_3d(ring + (size_t)ks * kTcStageBytes, &tmW, 0, r0, ks * kTcKB, &full[ks]);
+        tma_load_3d(ring + (size_t)ks * sb, &tmW, 0, r0, ks * kTcKB, &full[ks]);
       }
       pdl_wait();
       for (int ks = 0; ks < pre; ++ks)
-        tma_load_3d(ring + (size_t)ks * kTcStageBytes + kTcAOff, &tmA, 0, 0, ks * kTcKB, &full[ks]);
+        tma_load_3d(ring + (size_t)ks * sb + kTcAOff, &tmA, 0, 0, ks * kTcKB, &full[ks]);
       int it = pre;
       for (int ks = pre; ks < nk; ++ks, ++it) {
-        if (!ring_acquire(empty, it, kTcStages, abort_flag, a.ws.err)) break;
-        const int s = it % kTcStages;
+        if (!ring_acquire(empty, it, NS, abort_flag, a.ws.err)) break;
+        const int s = it % NS;
         mbar_arrive_expect_tx(&full[s], stage_tx);
-        tma_load_3d(ring + (size_t)s * kTcStageBytes, &tmW, 0, r0, ks * kTcKB, &full[s]);
-        tma_load_3d(ring + (size_t)s * kTcStageBytes + kTcAOff, &tmA, 0, 0, ks * kTcKB, &full[s]);
+        tma_load_3d(ring + (size_t)s * sb, &tmW, 0, r0, ks * kTcKB, &full[s]);
+        tma_load_3d(ring + (size_t)s * sb + kTcAOff, &tmA, 0, 0, ks * kTcKB, &full[s]);
       }
-      ring_drain(full, it, kTcStages, a.ws.err);
+      ring_drain(full, it, NS, a.ws.err);
     }
     return;
   }
@@ -110,9 +119,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int brow0 = 32 * nh + ((ai >> 1) << 3) + (lane & 7), bchk = ai & 1;
   const int ntile2 = (32 * nh + 16 < kTcRows) ? 2 : 1;  // tile pairs inside the 56-row box
   for (int ks = 0; ks < nk; ++ks) {
-    const int s = ks % kTcStages;
-    mbar_wait(&full[s], (ks / kTcStages) & 1, abort_flag, a.ws.err);
-    const uint32_t wbase = smem_addr(ring + (size_t)s * kTcStageBytes);
+    const int s = ks % NS;
+    mbar_wait(&full[s], (ks / NS) & 1, abort_flag, a.ws.err);
+    const uint32_t wbase = smem_addr(ring + (size_t)s * sb);
     const uint32_t abase = wbase + kTcAOff;
     if (active) {
 #pragma unroll
@@ -222,16 +231,9 @@ bool make_map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t oute
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-namespace {
-
-constexpr size_t kTcSmem = 1024 + (size_t)kTcStages * kTcStageBytes + (size_t)kTcTok * kTcRows * 4 +
-                           2 * kTcStages * 8 + 64;
-
-}  // namespace
-
 bool oproj_tc_ok(const LayerArgs& a, int grid, size_t optin) {
   return encode_fn() != nullptr && a.B <= kTcTok && a.d_o % kTcBK == 0 && (a.d + grid - 1) / grid <= 49 &&
-         kTcSmem <= optin;
+         tc_stages(std::min(kTcTok, (a.B + 15) / 16 * 16), optin) >= 3;
 }
 
 cudaError_t set_tc_attributes(size_t optin) {
@@ -240,7 +242,7 @@ cudaError_t set_tc_attributes(size_t optin) {
   return e;
 }
 
-cudaError_t launch_oproj_tc(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
+cudaError_t launch_oproj_tc(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t optin) {
   CUtensorMap tmW, tmA;
   const int tokb = std::min(kTcTok, (a.B + 15) / 16 * 16);
   if (!make_map(&tmW, a.w_o, (uint64_t)a.d_o, (uint64_t)a.d, kTcRows) ||
@@ -249,14 +251,15 @@ cudaError_t launch_oproj_tc(const LayerArgs& a, int grid, cudaStream_t s, bool p
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kTcSmem;
+  const int ns = tc_stages(tokb, optin), sb = tc_stage_bytes(tokb);
+  cfg.dynamicSmemBytes = kTcFixed + (size_t)ns * sb;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_oproj_tc, tmW, tmA, a, tokb);
+  return cudaLaunchKernelEx(&cfg, k_oproj_tc, tmW, tmA, a, tokb, ns, sb);
 }
 
 }  // namespace moe

@@ -197,7 +197,7 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
     }
     const bool pdl = l > 0 || first_pdl;
     e = v.oproj_small                         ? launch_oproj_s(a, G, h->cap, pdl, h->smem_optin)
-        : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, h->cap, pdl)
+        : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, h->cap, pdl, h->smem_optin)
                                             : launch_oproj(a, G, h->cap, pdl);
     if (e == cudaSuccess)
       e = (!v.experts_small && router_ks_ok(a, G, h->smem_optin))    ? launch_router_ks(a, G, h->cap, true)
@@ -592,7 +592,7 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
     }
     timed(1, s, [&](cudaStream_t st) {
       return v.oproj_small                         ? launch_oproj_s(a, G, st, false, h->smem_optin)
-             : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, st, false)
+             : oproj_tc_ok(a, G, h->smem_optin) ? launch_oproj_tc(a, G, st, false, h->smem_optin)
                                                  : launch_oproj(a, G, st, false);
     });
     timed(2, s, [&](cudaStream_t st) {

@@ -114,6 +114,8 @@ size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, Work
   unsigned char* es = take(sizeof(int) * entries);
   unsigned char* act = take(sizeof(float) * entries * I);
   unsigned char* au = take(sizeof(float) * kMaxUnion * 2 * I);
+  // the counter-ordered kernel's split-K router partials, [G][E][B rounded up to 8]
+  unsigned char* rp = take(sizeof(float) * G * E * ((B + 7) / 8 * 8));
   if (ws) {
     ws->counters = reinterpret_cast<unsigned*>(cnt);
     ws->err = reinterpret_cast<unsigned*>(cnt) + kNumCounters;
@@ -132,6 +134,7 @@ size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, Work
     ws->a = reinterpret_cast<float*>(act);
     ws->ecnt = reinterpret_cast<unsigned*>(cnt) + kNumCounters + 1;
     ws->a_u = reinterpret_cast<float*>(au);
+    ws->rpart = reinterpret_cast<float*>(rp);
   }
   return off;
 }

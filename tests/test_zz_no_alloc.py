@@ -70,10 +70,11 @@ def test_static_step_rejects_what_it_cannot_run():
     torch = _torch()
     import moe_decode_layer_02_b200 as md
     s = torch.cuda.current_stream()
-    # d = 8192, top_k * inter = 32 * 512: batch 2 needs more than MOE_STATIC_SCRATCH_BYTES.
+    # n_experts = 1024: the router's partial sums (SMs x 1024 x 8 floats) alone exceed
+    # MOE_STATIC_SCRATCH_BYTES on a 148-SM part.
     # The size checks run before anything is launched or read, so small dummy buffers stand
     # in for the weights and activations.
-    d, d_o, E, k, I = 8192, 64, 32, 32, 512
+    d, d_o, E, k, I = 8192, 64, 1024, 32, 512
     z = lambda n: torch.zeros(n, dtype=torch.bfloat16, device="cuda")
     w = tuple(z(64) for _ in range(5))
     attn, resid, out = z(64), z(64), z(64)
