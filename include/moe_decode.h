@@ -187,8 +187,8 @@ MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void*
                                     float* topk_gate, void* stream, float* kernel_ms,
                                     int* kernel_id, int max_kernels);
 
-/* Capacity of the static scratch array used by moe_decode_step_static (4 MiB per device). */
-#define MOE_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)
+/* Capacity of the static scratch array used by moe_decode_step_static (1.5 MiB per device). */
+#define MOE_STATIC_SCRATCH_BYTES (1536u * 1024u)
 
 /* One layer step for batch 1 or 2 that allocates no device memory.  The pages have no
  * counterpart of this entry point; it exists for callers that may not allocate when they
@@ -209,8 +209,9 @@ MOE_API int moe_decode_profile_step(moe_decode_handle* h, int batch, const void*
  *                bits (0 none, 1 a bounded wait ran out, 2 an index out of range)
  * Errors: MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_CONFIG / MOE_ERR_ALIGNMENT as for
  * create and step; MOE_ERR_SCRATCH_LIMIT when the scratch for (cfg, batch) exceeds
- * MOE_STATIC_SCRATCH_BYTES (e.g. n_experts = 1024 on 148 SMs: the router's partial sums alone,
- * SMs x n_experts x 8 floats, take 4.6 MiB); nothing is launched then.  MOE_ERR_CUDA on a failed CUDA call.
+ * MOE_STATIC_SCRATCH_BYTES (e.g. force_variant 3 with n_experts = 1024 at batch 2 on 148 SMs,
+ * whose split-K router partial sums, SMs x n_experts x batch floats, take 1.2 MB of the 1.7 MB
+ * needed); nothing is launched then.  MOE_ERR_CUDA on a failed CUDA call.
  * The first call on each device, with that device current, looks up the array's address
  * (cudaGetSymbolAddress) and sets kernel attributes; make that first call before any stream
  * capture begins.  Each call zeroes the barrier counters and error word at the head of the

@@ -23,7 +23,7 @@ MOE_ERR_CUDA = -5
 MOE_ERR_DEVICE_TIMEOUT = -6
 MOE_ERR_DEVICE_BOUNDS = -7
 MOE_ERR_SCRATCH_LIMIT = -8
-MOE_STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
+MOE_STATIC_SCRATCH_BYTES = 1536 * 1024
 
 EXPORTED = ("moe_decode_create", "moe_decode_step", "moe_decode_step_host", "moe_decode_sync_status",
             "moe_decode_get_intermediate", "moe_decode_kernels_per_step", "moe_decode_profile_step",

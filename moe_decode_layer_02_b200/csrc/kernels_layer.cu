@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const __grid_constant__
   csync();
   {
     for (int j = 0; j < nbox; ++j) mbar_wait(&fullO[(itO + j) % SO], ((itO + j) / SO) & 1, abort_flag, err);
-    const int Bp = (a.maxB + 7) & ~7;
+    const int Bp = a.maxB;
     float* P = a.ws.rpart + (size_t)c * E * Bp;  // [E][Bp]: this CTA's partial logits
 #pragma unroll 1
     for (int e = tid; e < E; e += kCT) {
@@ -472,7 +472,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer2(const __grid_constant__
   {
     // one warp per (expert, token): lanes sum the CTAs' partials in a fixed lane-strided order,
     // then a butterfly (the loads of all lanes are in flight together)
-    const int Bp = (a.maxB + 7) & ~7;
+    const int Bp = a.maxB;
     for (int z = warp; z < nr * NT; z += kCW) {
       const int e = e0 + z / NT, t = z % NT;
       float sacc = 0.f, ss = 0.f;  // the partials and, in the same round trips, the sums of h^2

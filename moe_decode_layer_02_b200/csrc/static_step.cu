@@ -90,7 +90,7 @@ size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Scratch layout for B tokens on G CTAs.  Counters and the error word come first so one
 // memset clears both.  Returns the bytes used; fills ws when base is non-null.
-size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, Workspace* ws) {
+size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, bool layer2, Workspace* ws) {
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -114,8 +114,8 @@ size_t carve(unsigned char* base, int B, int G, int d, int E, int K, int I, Work
   unsigned char* es = take(sizeof(int) * entries);
   unsigned char* act = take(sizeof(float) * entries * I);
   unsigned char* au = take(sizeof(float) * kMaxUnion * 2 * I);
-  // the counter-ordered kernel's split-K router partials, [G][E][B rounded up to 8]
-  unsigned char* rp = take(sizeof(float) * G * E * ((B + 7) / 8 * 8));
+  // the counter-ordered kernel's split-K router partials, [G][E][B]
+  unsigned char* rp = layer2 ? take(sizeof(float) * G * E * B) : nullptr;
   if (ws) {
     ws->counters = reinterpret_cast<unsigned*>(cnt);
     ws->err = reinterpret_cast<unsigned*>(cnt) + kNumCounters;
@@ -172,7 +172,8 @@ int moe_decode_step_static(const moe_decode_config* cfg, const moe_decode_layer_
   const int G = ds.num_sms;
   if ((long long)G * kConsumerThreads < c.d) return MOE_ERR_UNSUPPORTED_CONFIG;
 
-  const size_t need = carve(nullptr, batch, G, c.d, c.n_experts, c.top_k, c.inter, nullptr);
+  const bool layer2 = c.force_variant == 3;
+  const size_t need = carve(nullptr, batch, G, c.d, c.n_experts, c.top_k, c.inter, layer2, nullptr);
   if (need > (size_t)MOE_STATIC_SCRATCH_BYTES) return MOE_ERR_SCRATCH_LIMIT;
 
   LayerArgs a{};
@@ -195,7 +196,7 @@ int moe_decode_step_static(const moe_decode_config* cfg, const moe_decode_layer_
   a.out = static_cast<uint16_t*>(out);
   a.user_idx = topk_idx;
   a.user_gate = topk_gate;
-  carve(ds.scratch, batch, G, c.d, c.n_experts, c.top_k, c.inter, &a.ws);
+  carve(ds.scratch, batch, G, c.d, c.n_experts, c.top_k, c.inter, layer2, &a.ws);
   if (!small_path_ok(a, ds.smem_optin) || !router_ok(a, ds.smem_optin)) return MOE_ERR_UNSUPPORTED_CONFIG;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -31,7 +31,8 @@ def _inputs(torch, seed, dims, B):
 @pytest.mark.parametrize("dims,B,variant", [(synth.TINY, 1, 0), (synth.TINY, 2, 0), (RAGGED, 1, 0),
                                             (RAGGED, 2, 0), (synth.TINY, 1, 1), (RAGGED, 1, 1),
                                             (synth.TINY, 1, 3), (RAGGED, 2, 3),
-                                            (synth.TP16, 1, 0), (synth.TP16, 2, 0)])
+                                            (synth.TP16, 1, 0), (synth.TP16, 2, 0), (synth.TP16, 1, 3),
+                                            (synth.TP16, 2, 3)])
 def test_static_step_matches_step_twice(dims, B, variant):
     torch = _torch()
     import moe_decode_layer_02_b200 as md
@@ -70,15 +71,16 @@ def test_static_step_rejects_what_it_cannot_run():
     torch = _torch()
     import moe_decode_layer_02_b200 as md
     s = torch.cuda.current_stream()
-    # n_experts = 1024: the router's partial sums (SMs x 1024 x 8 floats) alone exceed
-    # MOE_STATIC_SCRATCH_BYTES on a 148-SM part.
+    # force_variant 3, n_experts = 1024, batch 2: the split-K router's partial sums
+    # (SMs x 1024 x 2 floats) and the rest need about 1.7 MB on a 148-SM part, more than
+    # MOE_STATIC_SCRATCH_BYTES.
     # The size checks run before anything is launched or read, so small dummy buffers stand
     # in for the weights and activations.
     d, d_o, E, k, I = 8192, 64, 1024, 32, 512
     z = lambda n: torch.zeros(n, dtype=torch.bfloat16, device="cuda")
     w = tuple(z(64) for _ in range(5))
     attn, resid, out = z(64), z(64), z(64)
-    cfg = md.config(d, d_o, E, k, I, 2)
+    cfg = md.config(d, d_o, E, k, I, 2, force_variant=3)
     with pytest.raises(md.MoeError) as ei:
         md.moe_decode_step_static(cfg, w, 2, attn, resid, out, stream=s)
     assert ei.value.code == md.MOE_ERR_SCRATCH_LIMIT
