@@ -17,7 +17,8 @@ enum Counter {
   kCntLayerExit = 0, kCntRouter = 1, kCntGateUp = 2, kCntLayer = 3, kCntProbe = 4,
   kCntRouterBar = 5,   // the split-K router's grid barriers
   kCntRouterExit = 6,  // its exit ticket (the last CTA out clears 1, 5 and 6)
-  kNumCounters = 7
+  kCntOUnit = 7,       // the fused layer kernel's o_proj unit counter (cleared after its barrier 1)
+  kNumCounters = 8
 };
 
 // Library-owned device workspace (one per handle).

@@ -844,12 +844,20 @@ namespace {
 // Scratch floats shared by the o_proj, router and phase A partial sums (each phase's use
 // ends before the next begins).  Phase B's gated activations live in the ring region, after
 // phase B's stages.
-__host__ __device__ constexpr size_t layer_scratch_floats(int NT, int RM, int RMr, int PM) {
-  const size_t o = (size_t)RM * kCW * NT + (size_t)NT * RM;   // o_proj partials + h^2
+__host__ __device__ constexpr size_t oproj_part_floats(int NT, int UC, int RS) {
+  return (((size_t)UC * RS * kCW * NT) + 3) & ~size_t(3);  // 16-byte multiple: the residual follows
+}
+__host__ __device__ constexpr size_t layer_scratch_floats(int NT, int UC, int RS, int RMr, int PM, int d) {
+  const size_t o = oproj_part_floats(NT, UC, RS) + (size_t)NT * d / 2 + UC;  // o_proj partials, residual, units
   const size_t r = (size_t)RMr * kCW * NT + 64;                // router partials + rstd
   const size_t pa = (size_t)PM * 2 * kCW * NT;                 // phase A partials
   const size_t m1 = o > r ? o : r;
   return m1 > pa ? m1 : pa;
+}
+
+// Most o_proj units (RS rows each) one CTA of G takes: twice an even share, plus one.
+__host__ __device__ constexpr int oproj_unit_cap(int d, int RS, int G) {
+  return 2 * (((d + RS - 1) / RS + G - 1) / G) + 1;
 }
 
 // Called by thread 0 after its CTA's last grid barrier.
@@ -880,7 +888,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   const size_t a_s_bytes = (size_t)std::min(E, B * a.k) * NT * I * 4;
   const size_t region =
       std::max(std::max((size_t)SO * SO_B, (size_t)SA * SA_B), (size_t)SBn * SB_B + a_s_bytes);
-  const size_t scratch_f = layer_scratch_floats(NT, RM, RMr, PM);
+  const int UC = oproj_unit_cap(d, RS, G);
+  const size_t scratch_f = layer_scratch_floats(NT, UC, RS, RMr, PM, d);
   long long lo, hi;
   split_range(d, G, c, lo, hi);
   const int i0 = (int)lo, nrows = (int)(hi - lo);  // o_proj rows = phase B output rows
@@ -889,7 +898,6 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
 
   unsigned char* ring = smem;
   float* part = reinterpret_cast<float*>(ring + region);
-  float* sq = part + RM * kCW * NT;   // o_proj: [NT][RM]
   float* rstd_s = part + RMr * kCW * NT;  // router
   // phase B: after phase B's stages (phase A's fills have all landed and been read by then)
   float* a_s = reinterpret_cast<float*>(ring + (size_t)SBn * SB_B);
@@ -903,7 +911,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   uint64_t* emptyA = fullA + kMaxStages;
   uint64_t* fullB = emptyA + kMaxStages;
   uint64_t* emptyB = fullB + kMaxStages;
-  int* s_misc = reinterpret_cast<int*>(emptyB + kMaxStages);
+  uint64_t* resbar = emptyB + kMaxStages;  // the residual's copy into shared memory
+  int* s_misc = reinterpret_cast<int*>(resbar + 1);
   volatile int* abort_flag = s_misc;
   unsigned* bar_count = &a.ws.counters[kCntLayer];
 
@@ -912,6 +921,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
     init_ring(fullO, emptyO, SO, kCW);
     init_ring(fullA, emptyA, SA, kCW);
     init_ring(fullB, emptyB, SBn, kCW);
+    mbar_init(resbar, 1);
     s_misc[0] = 0;
     fence_barrier_init();
   }
@@ -920,17 +930,68 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
 
   const int qbase_o = (d_o / 8) * warp / kCW, qpw_o = (d_o / 8) * (warp + 1) / kCW - qbase_o;
   const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
+  // o_proj work units: unit u = W_o rows [u RS, u RS + RS), one ring stage.  Three quarters
+  // of the units are split evenly and contiguously over the CTAs (S0 each); the rest are
+  // taken one at a time from a global counter, so a CTA whose copies stream faster takes more
+  // and the CTAs finish together.  A CTA takes at most UC units (its partial-sum buffers).
+  const int n_units = (d + RS - 1) / RS, S0 = (3 * n_units) / (4 * G);
+  float* opart = part;                                                         // [UC RS][kCW][NT]
+  uint16_t* res_s = reinterpret_cast<uint16_t*>(part + oproj_part_floats(NT, UC, RS));  // [B][d]
+  int* ouid = reinterpret_cast<int*>(part + oproj_part_floats(NT, UC, RS) + (size_t)NT * d / 2);  // [UC]
+  int* s_unit = s_misc + 8;  // [SO]: unit of each filled stage, -1 = no more units
   int itO = 0;  // O-ring fills (producer) / waits (consumers)
   if (warp == kCW) {
-    if (lane == 0) {  // weights are static: W_o, then W_r, before the dependency resolves
+    if (lane == 0) {  // weights are static: the first W_o fills go out before the dependency resolves
       const uint64_t pol = policy_evict_first();
       bulk_prefetch_l2(a.gamma, row_bytes);  // every CTA reads all of gamma after barrier 1
-      for (int r = i0; r < i0 + nrows; r += RS, ++itO) {
-        const int n = min(RS, i0 + nrows - r);
-        if (!ring_acquire(emptyO, itO, SO, abort_flag, a.ws.err)) break;
-        const int s = itO % SO;
+      int held = 0;  // units this CTA has been given (static fills and counter tickets)
+      auto fill_unit = [&](int u) -> bool {
+        if (!ring_acquire(emptyO, itO, SO, abort_flag, a.ws.err)) return false;
+        const int s = itO % SO, r = u * RS, n = min(RS, d - r);
+        s_unit[s] = u;
         mbar_arrive_expect_tx(&fullO[s], n * orow_bytes);
         bulk_g2s(ring + s * SO_B, a.w_o + (size_t)r * d_o, n * orow_bytes, &fullO[s], pol);
+        ++itO;
+        return true;
+      };
+      bool ok = true;
+      int nst = 0;  // static units filled
+      for (; nst < S0 && nst < SO && ok; ++nst) ok = fill_unit(c * S0 + nst);
+      held = S0;
+      // The counter was cleared by the previous launch after its barrier 1; griddepcontrol.wait
+      // makes that store visible.  The residual may come from the previous kernel too.
+      pdl_wait();
+      mbar_arrive_expect_tx(resbar, (uint32_t)B * row_bytes);
+      bulk_g2s(res_s, a.resid, (uint32_t)B * row_bytes, resbar, pol);
+      unsigned* unit_ctr = &a.ws.counters[kCntOUnit];
+      const int base = S0 * G;
+      // Two tickets in flight, each in a register of its own (a register array indexed at run
+      // time would sit in local memory, and storing a ticket there waits for its atomic).
+      int tA = 0, tB = 0;
+      bool hA = false, hB = false, more = base < n_units;
+      if (more && held < UC) { tA = (int)atomicAdd(unit_ctr, 1u); hA = true; ++held; }
+      if (more && held < UC) { tB = (int)atomicAdd(unit_ctr, 1u); hB = true; ++held; }
+      for (; nst < S0 && ok; ++nst) ok = fill_unit(c * S0 + nst);  // the tickets' round trips overlap these
+      auto use = [&](int& t, bool& h) {  // fill ticket t's unit and take the next ticket in its place
+        if (!h) return;
+        h = false;
+        const int u = base + t;
+        if (u < n_units && ok) {
+          if (more && held < UC) { t = (int)atomicAdd(unit_ctr, 1u); h = true; ++held; }
+          ok = fill_unit(u);
+        } else {
+          more = false;  // the other ticket is still read
+        }
+      };
+      while (hA || hB) {
+        use(tA, hA);
+        use(tB, hB);
+      }
+      if (ok && ring_acquire(emptyO, itO, SO, abort_flag, a.ws.err)) {  // end of the units
+        const int s = itO % SO;
+        s_unit[s] = -1;
+        mbar_arrive(&fullO[s]);
+        ++itO;
       }
       for (int j = 0; j < nr && !*abort_flag; j += RSr, ++itO) {
         const int n = min(RSr, nr - j);
@@ -942,29 +1003,21 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
       if (a.pf_w_o) {  // next layer: what the same CTA reads first, into L2
         if (nr > 0) bulk_prefetch_l2(a.pf_w_r + (size_t)e0 * d, nr * row_bytes);
         if (c == 0) bulk_prefetch_l2(a.pf_gamma, row_bytes);
-        size_t left = (size_t)min(a.pf_w_o_rows, nrows) * orow_bytes;
-        const unsigned char* src = reinterpret_cast<const unsigned char*>(a.pf_w_o + (size_t)i0 * d_o);
-        for (size_t off = 0; left > 0;) {
-          const uint32_t n = (uint32_t)min(left, (size_t)65536);
-          bulk_prefetch_l2(src + off, n);
-          off += n;
-          left -= n;
+        for (int j = 0; j < S0 && (size_t)j * RS < (size_t)a.pf_w_o_rows; ++j) {
+          const int u = c * S0 + j;
+          bulk_prefetch_l2(a.pf_w_o + (size_t)u * RS * d_o, (uint32_t)min(RS, d - u * RS) * orow_bytes);
         }
       }
       // The O ring's last fills land and are read (the router rows, after barrier 1) while
       // the consumers work towards barrier 2; phase A may then reuse the region at once.
       ring_drain(fullO, itO, SO, a.ws.err);
       for (int i = itO - SO < 0 ? 0 : itO - SO; i < itO; ++i) mbar_drain(&emptyO[i % SO], (i / SO) & 1, a.ws.err);
+      mbar_drain(resbar, 0, a.ws.err);
     }
   } else {
     // ---- o_proj (consumers) ----------------------------------------------------------
-    pdl_wait();  // attn_out and residual may come from the previous kernel
-    // this thread's residual element of the epilogue (rows x tokens <= 2 * 60 < kCT)
-    float res_v = 0.f;
-    if (tid < nrows * B) {
-      const int rr = tid / B, t = tid % B;
-      res_v = bf16f(__ldcg(reinterpret_cast<const unsigned short*>(a.resid + (size_t)t * d + i0 + rr)));
-    }
+    pdl_wait();  // attn_out may come from the previous kernel
+    int nslot = 0;
     {
       constexpr int kRI = 2;
       float xa[NT][kCPLf][8];
@@ -977,9 +1030,18 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
             u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)(qbase_o + j * 32 + lane) * 8);
           unpack8f(u, xa[t][j]);
         }
-      for (int r = i0; r < i0 + nrows; r += RS, ++itO) {
-        const int n = min(RS, i0 + nrows - r), s = itO % SO;
-        mbar_wait(&fullO[s], (itO / SO) & 1, abort_flag, a.ws.err);
+      while (true) {
+        const int s = itO % SO;
+        if (!mbar_wait(&fullO[s], (itO / SO) & 1, abort_flag, a.ws.err)) break;
+        const int u = s_unit[s];
+        if (u < 0 || nslot >= UC) {  // end of the units (the bound only guards the buffers)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&emptyO[s]);
+          ++itO;
+          break;
+        }
+        const int n = min(RS, d - u * RS);
+        if (warp == 0 && lane == 0) ouid[nslot] = u;
         const uint16_t* st = reinterpret_cast<const uint16_t*>(ring + s * SO_B);
         for (int j0 = 0; j0 < n; j0 += kRI) {
           const uint16_t* rp[kRI];
@@ -989,53 +1051,41 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
           rows_dot<NT, kRI>(rp, n - j0, xa, qbase_o, qpw_o, lane, v);
           const float tot = warp_reduce_multi<kRI * NT>(v, lane);
           const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
-          if (multi_writer<kRI * NT>(lane) && j < n) part[((r - i0 + j) * kCW + warp) * NT + t] = tot;
+          if (multi_writer<kRI * NT>(lane) && j < n) opart[(((size_t)nslot * RS + j) * kCW + warp) * NT + t] = tot;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&emptyO[s]);
+        ++itO;
+        ++nslot;
       }
     }
     csync();
-    if (tid < nrows * B) {
-      const int rr = tid / B, t = tid % B;
-      float sacc = 0.f;
+    mbar_wait(resbar, 0, abort_flag, a.ws.err);
+    for (int z = tid; z < nslot * RS * B; z += kCT) {  // h = residual + sum of the warps' partials
+      const int sl = z / (RS * B), rem = z - sl * RS * B, j = rem / B, t = rem - j * B;
+      const int row = ouid[sl] * RS + j;
+      if (row < d) {
+        float sacc = 0.f;
 #pragma unroll
-      for (int w = 0; w < kCW; ++w) sacc += part[(rr * kCW + w) * NT + t];
-      const float hv = res_v + sacc;
-      a.ws.h[(size_t)t * d + i0 + rr] = hv;
-      sq[t * RM + rr] = hv * hv;
-    }
-    csync();
-    if (warp < B) {  // per-CTA sum of h^2, fixed order
-      float ss = 0.f;
-      for (int rr = lane; rr < nrows; rr += 32) ss += sq[warp * RM + rr];
-      ss = warp_sum(ss);
-      if (lane == 0) a.ws.ss_part[(size_t)c * a.maxB + warp] = ss;
+        for (int w = 0; w < kCW; ++w) sacc += opart[(((size_t)sl * RS + j) * kCW + w) * NT + t];
+        a.ws.h[(size_t)t * d + row] = bf16f(res_s[(size_t)t * d + row]) + sacc;
+      }
     }
     grid_barrier(bar_count, (unsigned)G, abort_flag, a.ws.err);
+    if (c == 0 && tid == 0) a.ws.counters[kCntOUnit] = 0;  // every CTA has taken its last unit
 
     // ---- router (consumers) ----------------------------------------------------------
     {
-      for (int t = warp; t < B; t += kCW) {  // fixed order: same bits in every CTA
-        float ss = 0.f;
-        for (int c0 = 0; c0 < G; c0 += 8 * 32) {
-          float pv[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int cc = c0 + k * 32 + lane;
-            pv[k] = cc < G ? ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]) : 0.f;
-          }
-#pragma unroll
-          for (int k = 0; k < 8; ++k) ss += pv[k];
-        }
-        ss = warp_sum(ss);
-        if (lane == 0) {
-          const float rv = 1.0f / sqrtf(ss / (float)d + a.eps);
-          rstd_s[t] = rv;
-          if (c == 0) a.ws.rstd[t] = rv;
-        }
-      }
+      // h and gamma in one round of loads; the sum of h^2 over d from the same registers
+      // (per lane, per warp, then the 15 warps in a fixed order: the same bits in every CTA)
       float xr[NT][kCPLf][8];
+      float gam[kCPLf][8];
+#pragma unroll
+      for (int j = 0; j < kCPLf; ++j) {
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (cvalid(qpw, j, lane)) u = ld_weight_u4(a.gamma + (size_t)(qbase + j * 32 + lane) * 8);
+        unpack8f(u, gam[j]);
+      }
 #pragma unroll
       for (int t = 0; t < NT; ++t)
 #pragma unroll
@@ -1050,19 +1100,33 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
             for (int e = 0; e < 8; ++e) xr[t][j][e] = 0.f;
           }
         }
+      float* wss = rstd_s + 2;  // [kCW][NT]
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float s2 = 0.f;
+#pragma unroll
+        for (int j = 0; j < kCPLf; ++j)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s2 = fmaf(xr[t][j][e], xr[t][j][e], s2);
+        s2 = warp_sum(s2);
+        if (lane == 0) wss[warp * NT + t] = s2;
+      }
       csync();
+      float rv[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float ss = 0.f;
+        for (int w = 0; w < kCW; ++w) ss += wss[w * NT + t];
+        rv[t] = (t < B) ? 1.0f / sqrtf(ss / (float)d + a.eps) : 0.f;
+        if (c == 0 && tid == 0 && t < B) a.ws.rstd[t] = rv[t];
+      }
 #pragma unroll
       for (int j = 0; j < kCPLf; ++j) {
         const int q = qbase + j * 32 + lane;
-        float gam[8];
-        uint4 u = make_uint4(0, 0, 0, 0);
-        if (cvalid(qpw, j, lane)) u = ld_weight_u4(a.gamma + (size_t)q * 8);
-        unpack8f(u, gam);
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          const float rv = (t < B) ? rstd_s[t] : 0.f;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) xr[t][j][e] = xr[t][j][e] * rv * gam[e];
+          for (int e = 0; e < 8; ++e) xr[t][j][e] = xr[t][j][e] * rv[t] * gam[j][e];
           if (t < B && cvalid(qpw, j, lane) && q % G == c) {  // each chunk of x is written by one CTA
             float* xp = a.ws.x + (size_t)t * d + (size_t)q * 8;
             *reinterpret_cast<float4*>(xp) = make_float4(xr[t][j][0], xr[t][j][1], xr[t][j][2], xr[t][j][3]);
@@ -1388,12 +1452,13 @@ bool plan_fused(LayerArgs& a, int G, size_t optin) {
   const long long umax = std::min(a.E, std::max(a.B, 1) * a.k);
   pa.rows_max = (int)((umax * a.I + G - 1) / G);
   pb.rows_max = o.rows_max;
-  const size_t scratch_f = layer_scratch_floats(NT, o.rows_max, r.rows_max, pa.rows_max);
+  o.rows_per_stage = (int)std::max<size_t>(1, std::min<size_t>(32768 / orow, (size_t)o.rows_max));
+  const size_t scratch_f =
+      layer_scratch_floats(NT, oproj_unit_cap(a.d, o.rows_per_stage, G), o.rows_per_stage, r.rows_max, pa.rows_max, a.d);
   const size_t a_s_bytes = (size_t)umax * NT * a.I * 4;
-  const size_t extra = up128(scratch_f * 4) + kRouteBytes + 6 * kMaxStages * 8 + 64;
+  const size_t extra = up128(scratch_f * 4) + kRouteBytes + 6 * kMaxStages * 8 + 8 + 64;
   if (extra >= budget) return false;
   const size_t cap = budget - extra;
-  o.rows_per_stage = (int)std::max<size_t>(1, std::min<size_t>(32768 / orow, (size_t)o.rows_max));
   const size_t SO = std::max(up128((size_t)o.rows_per_stage * orow), up128(row));
   o.stages = (int)std::min<size_t>(kMaxStages, cap / SO);
   r.rows_per_stage = (int)(SO / row);
