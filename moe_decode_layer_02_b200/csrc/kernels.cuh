@@ -42,7 +42,8 @@ struct Workspace {
   // (zero between launches), and the activations [kMaxUnion][B][I]
   unsigned* ecnt;      // [kMaxUnion]
   float* a_u;          // [kMaxUnion][2][I]
-  float* rpart;        // split-K router: per-CTA partial logits [G][E][8 * ceil(maxB / 8)]
+  float* rpart;        // split-K routers' per-CTA partial logits: [G][E][8 ceil(B / 8)] above batch 2,
+                       // [G][E][maxB] in the counter-ordered kernel (8 ceil(maxB / 8) per CTA and expert allocated)
 };
 
 constexpr int kMaxUnion = 64;  // union experts of a batch <= 2 step (2 tokens x top_k <= 32)

@@ -349,7 +349,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
                o_cnt = take(sizeof(unsigned) * kNumCounters),
                o_err = take(sizeof(unsigned)), o_r0 = take(2ull * maxB * d), o_r1 = take(2ull * maxB * d),
                o_ec = take(sizeof(unsigned) * kMaxUnion), o_au = take(sizeof(float) * kMaxUnion * 2 * I),
-               o_rp = take(sizeof(float) * G * E * maxB);
+               o_rp = take(sizeof(float) * G * E * ((maxB + 7) / 8 * 8));  // the split-K router pads B to 8
   if (cudaMalloc(&h->ws_base, off) != cudaSuccess) {
     cudaGetLastError();
     delete h;

@@ -110,6 +110,19 @@ def test_ragged_shapes(B):
         st.close()
 
 
+# --- max_batch equal to the batch, not a multiple of 8: the workspace is sized for max_batch
+#     while the split-K router pads the batch to 8 per expert --------------------------------
+@pytest.mark.parametrize("B", [3, 5])
+def test_ragged_max_batch_equals_batch(B):
+    dims = synth.Dims(320, 192, 40, 5, 96)
+    seed = synth.config_seed(10) + B
+    st = H.GpuStack(seed, dims, max_batch=B)
+    try:
+        check_case(st, build_case(seed, dims, B))
+    finally:
+        st.close()
+
+
 # --- the largest shapes the library accepts, one dimension at a time -----------------------
 #   d = d_o = 8192 with k = 32 and I = 512 (64 experts keep the weights at ~1.2 GB), and
 #   E = 1024 with k = 32 on d = 1024 (large enough a logit spread for gapped draws).  Batch 1
@@ -251,6 +264,19 @@ def test_tp16_speculative_shapes(tp16, B):
     case = build_case(seed, synth.TP16, B, attn0=attn0, resid0=resid0, refs=[ref])
     out, idx, gate, _ = check_case(st, case)  # every token
     assert len(set(idx[0].ravel().tolist())) == 12 + B * (synth.TP16.k - 12)
+
+
+@pytest.mark.slow
+def test_tp16_speculative_max_batch_4(tp16):
+    """The speculative shape on a handle whose max_batch is the batch (4), as a verifier that
+    sizes its handle exactly would create it."""
+    seed, st0, ref = tp16
+    st = H.GpuStack(seed, synth.TP16, max_batch=4, weights=st0.weights)
+    try:
+        attn0, resid0, _ = H.constructed_shared(seed, synth.TP16, 4, core=12, ref=ref)
+        check_case(st, build_case(seed, synth.TP16, 4, attn0=attn0, resid0=resid0, refs=[ref]))
+    finally:
+        st.close()
 
 
 # --- full-size layer (1/8 shard, I=256), batch 16 and 64 -------------------------------------
