@@ -21,11 +21,13 @@ from oracle.layer import LayerRef, build_case, token_attn, top_gap  # noqa: F401
 
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
-# The router accumulates d = 7168 fp32 products in a different order than the fp64 oracle,
-# so a logit is off by ~1e-6; a gate moves by at most 1/4 of the largest logit difference
-# (sum over j of |d gate_i / d logit_j| = 2 g_i (1 - g_i) <= 1/2, applied to differences of
-# at most twice the logit error), plus fp32 rounding of the softmax itself (~1e-7).
-GATE_ATOL = 2e-6
+# A gate moves by at most the largest logit error: the sum over j of |d gate_i / d logit_j|
+# is 2 g_i (1 - g_i) <= 1/2, applied to logit differences of at most twice the logit error;
+# fp32 rounding of the softmax itself adds ~1e-7.  The logits differ from the fp64 oracle's
+# by the fp32 rounding of o_proj (d_o = 8192 products, on the tensor cores above batch 2),
+# RMSNorm and the router (d = 7168 products): up to 6.6e-6 measured at full size, every token
+# checked.  So gates are held to 1e-5.
+GATE_ATOL = 1e-5
 
 # Worst errors seen by the parity checks of this session (reported by conftest at the end).
 WORST = {"gate_abs": 0.0, "logit_abs": 0.0, "out_excess": -1.0, "out_rel_l2": 0.0}
