@@ -218,25 +218,38 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
       }
     }
     rk_barrier(bar_count, (unsigned)G, abort_flag, err);
-    // logits of this CTA's experts: the partials summed over the CTAs in order, times rstd
+    // logits of this CTA's experts: the partials summed over the CTAs, times rstd.  gl lanes
+    // share an (expert, token) item (as many as the CTA's threads allow), each lane summing
+    // every gl-th CTA's partial and the group adding its lanes' sums by shuffles, so that an
+    // item's G loads take one or two rounds to L2 instead of G / 8 (a fixed order for a given
+    // batch: the same bits on every run)
     {
       split_range(E, G, c, lo, hi);
-      const int e0 = (int)lo, ne = (int)(hi - lo);
-      for (int z = tid; z < ne * B; z += kCT) {
-        const int e = e0 + z / B, t = z % B;
-        const float* p = a.ws.rpart + (size_t)e * Bp + t;
-        const size_t stride = (size_t)E * Bp;
+      const int e0 = (int)lo, ne = (int)(hi - lo), items = ne * B;
+      int gl = 32;
+      while (gl > 1 && items * gl > kCT) gl >>= 1;
+      const int ipw = 32 / gl;  // items per warp and round
+      const size_t stride = (size_t)E * Bp;
+      for (int base = warp * ipw; base < items; base += kCW * ipw) {
+        const int z = base + lane / gl, sub = lane % gl;
         float s = 0.f;
-        int cc = 0;
-        for (; cc + 8 <= G; cc += 8) {
-          float v[8];
+        if (z < items) {
+          const float* p = a.ws.rpart + (size_t)(e0 + z / B) * Bp + z % B;
+          int cc = sub;
+          for (; cc + 7 * gl < G; cc += 8 * gl) {
+            float v[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) v[k] = ld_act(p + (size_t)(cc + k) * stride);
+            for (int k = 0; k < 8; ++k) v[k] = ld_act(p + (size_t)(cc + k * gl) * stride);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) s += v[k];
+            for (int k = 0; k < 8; ++k) s += v[k];
+          }
+          for (; cc < G; cc += gl) s += ld_act(p + (size_t)cc * stride);
         }
-        for (; cc < G; ++cc) s += ld_act(p + (size_t)cc * stride);
-        a.ws.logits[(size_t)t * E + e] = rstd_s[t] * s;
+        for (int o = gl >> 1; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (z < items && sub == 0) {
+          const int e = e0 + z / B, t = z % B;
+          a.ws.logits[(size_t)t * E + e] = rstd_s[t] * s;
+        }
       }
     }
     rk_barrier(bar_count, 2u * (unsigned)G, abort_flag, err);

@@ -4,9 +4,14 @@
 // that is still bound by the 117 MB of W_o.  CTA c owns output rows [r0, r1) (49 at most);
 // the K dimension (d_o) is streamed 256 at a time: per stage one TMA copy of W_o (56 rows x
 // four 64-wide k-blocks) and one of attn_out (B rounded up to 16 tokens x four k-blocks),
-// both with the 128-byte swizzle, so W_o is read once and the activations come from L2.  8 consumer warps run mma.sync m16n8k16
-// (tokens as M, weight rows as N): warp w owns tokens [16 (w % 4), +16) and weight-row
-// tiles 4 (w / 4) .. 4 (w / 4) + 3; ldmatrix reads both operands through the swizzle.
+// both with the 128-byte swizzle, so W_o is read once and the activations come from L2.  8
+// consumer warps run mma.sync m16n8k16 (tokens as M, weight rows as N).  The work of a stage
+// is (token tile, half of the weight rows, k-block) items; with fewer than four token tiles
+// the four k-blocks are split over the warps as well (each warp then sums its own k-blocks
+// and the warps' partial sums are added in a fixed order at the end), so that every warp, and
+// so every SM sub-partition's tensor pipe, takes an equal share: with one token tile on two
+// warps the two warps' MMAs, issued on one sub-partition, were the bound of the kernel.
+// ldmatrix reads both operands through the swizzle.
 // The epilogue adds the residual, writes h in fp32 and the CTA's sums of h^2 per token in a
 // fixed order.
 //
@@ -106,8 +111,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   pdl_wait();  // the residual may come from the previous kernel
-  const int mt = warp & 3, nh = warp >> 2;   // tokens [16 mt, +16), weight-row tiles 4 nh .. 4 nh + 3
-  const bool active = 16 * mt < B;
+  // warp -> (token tile mt, row half nh, k-block quarter kq): tokens [16 mt, +16), weight-row
+  // tiles 4 nh .. 4 nh + 3, k-blocks [kq kpw, kq kpw + kpw) of every stage
+  const int mtiles = tokb / 16, ksplit = mtiles == 1 ? 4 : (mtiles == 2 ? 2 : 1), kpw = kTcKB / ksplit;
+  const int combo = warp / ksplit, kq = warp - combo * ksplit;
+  const int mt = combo % mtiles, nh = combo / mtiles;
+  const bool active = combo < 2 * mtiles && 16 * mt < B;
   float acc[4][4];
 #pragma unroll
   for (int n = 0; n < 4; ++n)
@@ -123,40 +132,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_wait(&full[s], (ks / NS) & 1, abort_flag, a.ws.err);
     const uint32_t wbase = smem_addr(ring + (size_t)s * sb);
     const uint32_t abase = wbase + kTcAOff;
-    if (active) {
+    // each 64-wide k-block is summed by the tensor core into fresh registers (4 chained MMAs);
+    // the running sums over k-blocks are fp32 adds, which round more tightly than the tensor
+    // core's own accumulation of a chain as long as d_o
+    auto kblock = [&](int kb) {
+      const uint32_t wt = wbase + kb * kTcWTile, at = abase + (uint32_t)(kb * tokb * kTcBK * 2);
+      float blk[4][4];
 #pragma unroll
-      for (int kb = 0; kb < kTcKB; ++kb) {
-        const uint32_t wt = wbase + kb * kTcWTile, at = abase + (uint32_t)(kb * tokb * kTcBK * 2);
-        // each 64-wide k-block is summed by the tensor core into fresh registers (4 chained
-        // MMAs); the running sums over k-blocks are fp32 adds, which round more tightly than
-        // the tensor core's own accumulation of a chain as long as d_o
-        float blk[4][4];
+      for (int n = 0; n < 4; ++n)
 #pragma unroll
-        for (int n = 0; n < 4; ++n)
+        for (int e = 0; e < 4; ++e) blk[n][e] = 0.f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) blk[n][e] = 0.f;
+      for (int kk = 0; kk < kTcBK / 16; ++kk) {
+        uint32_t af[4];
+        ldsm4(af, at + swz(arow, 2 * kk + achk));
 #pragma unroll
-        for (int kk = 0; kk < kTcBK / 16; ++kk) {
-          uint32_t af[4];
-          ldsm4(af, at + swz(arow, 2 * kk + achk));
-#pragma unroll
-          for (int np = 0; np < 2; ++np) {
-            if (np < ntile2) {
-              uint32_t bf[4];
-              ldsm4(bf, wt + swz(brow0 + 16 * np, 2 * kk + bchk));
-              mma16816(blk[2 * np], af, bf[0], bf[1]);
-              mma16816(blk[2 * np + 1], af, bf[2], bf[3]);
-            }
+        for (int np = 0; np < 2; ++np) {
+          if (np < ntile2) {
+            uint32_t bf[4];
+            ldsm4(bf, wt + swz(brow0 + 16 * np, 2 * kk + bchk));
+            mma16816(blk[2 * np], af, bf[0], bf[1]);
+            mma16816(blk[2 * np + 1], af, bf[2], bf[3]);
           }
         }
+      }
 #pragma unroll
-        for (int n = 0; n < 4; ++n)
+      for (int n = 0; n < 4; ++n)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[n][e] += blk[n][e];
+        for (int e = 0; e < 4; ++e) acc[n][e] += blk[n][e];
+    };
+    if (active) {
+      if (ksplit == 1) {  // all four k-blocks: unrolled, so their loads and MMAs interleave
+#pragma unroll
+        for (int kb = 0; kb < kTcKB; ++kb) kblock(kb);
+      } else {
+#pragma unroll 1
+        for (int kb = kq * kpw; kb < kq * kpw + kpw; ++kb) kblock(kb);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+  }
+  if (ksplit > 1) {  // the k-block quarters' partial sums, added in a fixed order (ring reused)
+    consumer_sync();  // every stage has been read
+    float* red = reinterpret_cast<float*>(ring);  // [kConsumerWarps][16][32]
+#pragma unroll
+    for (int n = 0; n < 4; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) red[(warp * 16 + n * 4 + e) * 32 + lane] = acc[n][e];
+    consumer_sync();
+    if (kq == 0) {
+#pragma unroll
+      for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float v = 0.f;
+          for (int j = 0; j < ksplit; ++j) v += red[((warp + j) * 16 + n * 4 + e) * 32 + lane];
+          acc[n][e] = v;
+        }
+    }
   }
   // epilogue: D fragment of tile n: lane (g, q) holds tokens 16 mt + g (+8), rows 8 n' + 2q (+1)
   const int g = lane >> 2, q = lane & 3;
@@ -166,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int t = 16 * mt + g + ((e >> 1) << 3), rr = nrow + (e & 1);
-      if (active && t < B && rr < rows) {
+      if (active && kq == 0 && t < B && rr < rows) {
         const size_t o = (size_t)t * d + r0 + rr;
         const float hv = bf16f(__ldcg(reinterpret_cast<const unsigned short*>(a.resid + o))) + acc[n][e];
         a.ws.h[o] = hv;
