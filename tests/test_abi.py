@@ -152,6 +152,41 @@ def test_host_buffer_step_matches_device_step():
 
 
 @pytest.mark.gpu
+def test_host_buffer_step_pinned_caller_buffers():
+    """The caller's own pinned buffers: the graph copies straight from and to them (no host
+    gather or scatter); results equal the device step's, on a new graph and its replay, and
+    a mix with pageable outputs falls back to the staging copies."""
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import synth
+    from oracle.layer import build_case
+    from tests.harness import GpuStack
+    synth.build_device_fill()
+    dims = synth.Dims(256, 256, 16, 4, 128)  # top_k * 4 bytes per token: whole 16-byte words
+    seed = synth.config_seed(0) + 91
+    st = GpuStack(seed, dims, max_batch=4)
+    try:
+        for B in (1, 3, 3):
+            case = build_case(seed + B, dims, B, checked=[0])
+            out_d, idx_d, gate_d = st.step(case["attn"], case["resid"])
+            pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+            attn_p = pin(case["attn"].view(np.int16))
+            resid_p = pin(case["resid"].view(np.int16))
+            out_p = torch.zeros((B, dims.d), dtype=torch.int16).pin_memory()
+            idx_p = torch.zeros((1, B, dims.k), dtype=torch.int32).pin_memory()
+            gate_p = torch.zeros((1, B, dims.k), dtype=torch.float32).pin_memory()
+            st.md.moe_decode_step_host(st.h, B, attn_p, resid_p, out_p, idx_p, gate_p)
+            assert np.array_equal(out_p.numpy().view(np.uint16), out_d)
+            assert np.array_equal(idx_p.numpy(), idx_d) and np.array_equal(gate_p.numpy(), gate_d)
+            out_h = np.zeros((B, dims.d), np.uint16)
+            st.md.moe_decode_step_host(st.h, B, attn_p, resid_p, out_h)
+            assert np.array_equal(out_h, out_d)
+    finally:
+        st.close()
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("B", [1, 2, 5])
 def test_host_buffer_step_two_layer_stack(B):
     torch = pytest.importorskip("torch")
