@@ -131,17 +131,13 @@ MOE_API int moe_decode_step(moe_decode_handle* h, int batch, const void* attn_ou
                     const void* residual_in, void* out, int32_t* topk_idx, float* topk_gate,
                     void* stream);
 
-/* Same step with HOST buffers (same shapes as moe_decode_step), any host memory,
- * pinned or not; topk_idx / topk_gate may be NULL.  One graph launch and one
- * synchronisation of `stream` per call:
- *   - when every buffer passed is pinned and mapped into the device's address space
- *     (e.g. cudaHostAlloc / cudaMallocHost, torch pin_memory), 16-byte aligned and a
- *     whole number of 16-byte words long, the graph copies the inputs from them and
- *     the outputs into them directly (checked on every call);
- *   - otherwise the inputs are gathered into a handle-owned pinned buffer, moved in
- *     one copy, and the outputs moved back in one copy and scattered.
- * The first call allocates the staging (device and pinned host memory for max_batch
- * tokens); MOE_ERR_OOM if that fails. */
+/* Same step with HOST buffers (same shapes as moe_decode_step): gathers the
+ * inputs into a handle-owned pinned buffer, moves them to handle-owned device
+ * buffers in one copy, runs the step, moves the outputs back in one copy,
+ * synchronises `stream` and scatters them into the caller's buffers (any host
+ * memory, pinned or not).  topk_idx / topk_gate may be NULL.  The first call
+ * allocates the staging (device and pinned host memory for max_batch tokens);
+ * MOE_ERR_OOM if that fails. */
 MOE_API int moe_decode_step_host(moe_decode_handle* h, int batch, const void* attn_out_host,
                          const void* residual_in_host, void* out_host, int32_t* topk_idx_host,
                          float* topk_gate_host, void* stream);

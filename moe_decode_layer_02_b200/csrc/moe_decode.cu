@@ -38,46 +38,27 @@ namespace {
 
 struct GraphEntry {
   int batch;
-  const void* key[5];  // attn, resid, out, idx, gate: device buffers, or the caller's host buffers
-  int host;  // 0 device buffers; 1 host buffers through the handle's pinned staging; 2 the caller's
-             // own pinned (device-mapped) host buffers, copied straight from and to
+  const void *attn, *resid, *out, *idx, *gate;
+  bool host;  // host-buffer step: staging copies in the graph around the layer kernels
   cudaGraphExec_t exec;
   int kernels;
 };
 
-// Staging copies of the host-buffer step: up to three segments of n 16-byte words from src to
-// dst, one side pinned host memory (through its device address), the other device memory.  The
-// copy-in runs first in the graph and lets the first layer kernel launch at once (its producer
-// streams weights while the inputs arrive; its consumers wait for this grid); the copy-out
-// waits for the last kernel.
-struct CopySegs {
-  const uint4* src[3];
-  uint4* dst[3];
-  unsigned long long n[3];
-  int count;
-};
-
-__global__ void k_stage_copy(const CopySegs c, int after_previous) {
+// Staging copy of the host-buffer step: n 16-byte words from src to dst, one side pinned host
+// memory (through its device address), the other device memory.  The copy-in runs first in the
+// graph and lets the first layer kernel launch at once (its producer streams weights while the
+// inputs arrive; its consumers wait for this grid); the copy-out waits for the last kernel.
+__global__ void k_stage_copy(const uint4* __restrict__ src, uint4* __restrict__ dst, unsigned long long n,
+                             int after_previous) {
   if (after_previous) asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const unsigned long long stride = (unsigned long long)gridDim.x * blockDim.x;
-  for (int g = 0; g < c.count; ++g)
-    for (unsigned long long i = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; i < c.n[g]; i += stride)
-      c.dst[g][i] = c.src[g][i];
+  for (unsigned long long i = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    dst[i] = src[i];
 }
 
-CopySegs one_seg(const void* src, void* dst, size_t bytes) {
-  CopySegs c = {};
-  c.src[0] = static_cast<const uint4*>(src);
-  c.dst[0] = static_cast<uint4*>(dst);
-  c.n[0] = (bytes + 15) / 16;
-  c.count = 1;
-  return c;
-}
-
-cudaError_t launch_stage_copy(const CopySegs& c, bool after_previous, cudaStream_t s) {
-  unsigned long long n = 0;
-  for (int g = 0; g < c.count; ++g) n = std::max(n, c.n[g]);
+cudaError_t launch_stage_copy(const void* src, void* dst, size_t bytes, bool after_previous, cudaStream_t s) {
+  const unsigned long long n = (bytes + 15) / 16;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)std::min<unsigned long long>(148, std::max<unsigned long long>(1, (n + 1023) / 1024)));
   cfg.blockDim = dim3(256);
@@ -87,7 +68,8 @@ cudaError_t launch_stage_copy(const CopySegs& c, bool after_previous, cudaStream
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = after_previous ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_stage_copy, c, after_previous ? 1 : 0);
+  return cudaLaunchKernelEx(&cfg, k_stage_copy, static_cast<const uint4*>(src), static_cast<uint4*>(dst), n,
+                            after_previous ? 1 : 0);
 }
 
 constexpr size_t kPrefetchWoBytes = 16ull << 20;  // bytes of the next W_o prefetched into L2
@@ -235,18 +217,14 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
   return kernels;
 }
 
-// host != 0: the step's copy-in (cin) and copy-out (cout) segments wrap the layer kernels;
-// key: the pointers the graph is cached under (the caller's host buffers for host 2), by
-// default the five device buffers.
+// host: the step reads its inputs from, and writes its outputs to, the handle's pinned
+// staging (in_bytes from pin_in_dev to attn; out_bytes from out to pin_out_dev).
 int get_graph(moe_decode_handle* h, int B, const void* attn, const void* resid, void* out,
-              int32_t* idx, float* gate, GraphEntry** ge, int host = 0, const CopySegs* cin = nullptr,
-              const CopySegs* cout = nullptr, const void* const* key = nullptr) {
-  const void* k[5] = {attn, resid, out, idx, gate};
-  if (key)
-    for (int i = 0; i < 5; ++i) k[i] = key[i];
+              int32_t* idx, float* gate, GraphEntry** ge, bool host = false, size_t in_bytes = 0,
+              size_t out_bytes = 0) {
   for (auto& g : h->graphs)
-    if (g.batch == B && g.host == host && g.key[0] == k[0] && g.key[1] == k[1] && g.key[2] == k[2] &&
-        g.key[3] == k[3] && g.key[4] == k[4]) {
+    if (g.batch == B && g.attn == attn && g.resid == resid && g.out == out && g.idx == idx && g.gate == gate &&
+        g.host == host) {
       *ge = &g;
       return MOE_OK;
     }
@@ -258,9 +236,9 @@ int get_graph(moe_decode_handle* h, int B, const void* attn, const void* resid, 
   if (cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return MOE_ERR_CUDA;
   cudaError_t rec = cudaSuccess;
   int kernels = 0;
-  if (host) rec = launch_stage_copy(*cin, false, h->cap);
-  if (rec == cudaSuccess) kernels = record_step(h, B, attn, resid, out, idx, gate, &rec, host != 0);
-  if (host && rec == cudaSuccess) rec = launch_stage_copy(*cout, true, h->cap);
+  if (host) rec = launch_stage_copy(h->pin_in_dev, const_cast<void*>(attn), in_bytes, false, h->cap);
+  if (rec == cudaSuccess) kernels = record_step(h, B, attn, resid, out, idx, gate, &rec, host);
+  if (host && rec == cudaSuccess) rec = launch_stage_copy(out, h->pin_out_dev, out_bytes, true, h->cap);
   const cudaError_t end = cudaStreamEndCapture(h->cap, &graph);
   if (rec != cudaSuccess || end != cudaSuccess || !graph) {
     if (graph) cudaGraphDestroy(graph);
@@ -274,7 +252,7 @@ int get_graph(moe_decode_handle* h, int B, const void* attn, const void* resid, 
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
-  h->graphs.push_back(GraphEntry{B, {k[0], k[1], k[2], k[3], k[4]}, host, exec, kernels});
+  h->graphs.push_back(GraphEntry{B, attn, resid, out, idx, gate, host, exec, kernels});
   *ge = &h->graphs.back();
   return MOE_OK;
 }
@@ -488,66 +466,15 @@ int moe_decode_step_host(moe_decode_handle* h, int batch, const void* attn_out_h
   char* dout = static_cast<char*>(h->h_outs);
   char* pin = static_cast<char*>(h->pin_in);
   char* pout = static_cast<char*>(h->pin_out);
-  int32_t* didx = topk_idx_host ? (int32_t*)(dout + o_idx) : nullptr;
-  float* dgate = topk_gate_host ? (float*)(dout + o_gate) : nullptr;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The caller's buffers pinned and mapped into the device's address space, 16-byte aligned
-  // and whole 16-byte words: the graph copies straight from and to them, with no gather or
-  // scatter on the host.  Checked on every call (a buffer may have been freed and its
-  // address reused by pageable memory).
-  const void* src_in[2] = {attn_out_host, residual_in_host};
-  const size_t n_in[2] = {n_attn, n_res};
-  void* dst_out[3] = {out_host, topk_idx_host, topk_gate_host};
-  const size_t n_out[3] = {n_res, n_tk, n_tk};
-  void* dev_in[2] = {nullptr, nullptr};
-  void* dev_out[3] = {nullptr, nullptr, nullptr};
-  bool direct = true;
-  auto mapped = [&](const void* p, size_t n, void** dp) {
-    if (!p) return true;
-    if ((reinterpret_cast<uintptr_t>(p) & 15u) || (n & 15u)) return false;
-    cudaPointerAttributes at;
-    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
-      cudaGetLastError();
-      return false;
-    }
-    if (at.type != cudaMemoryTypeHost || !at.devicePointer) return false;
-    *dp = at.devicePointer;
-    return true;
-  };
-  for (int i = 0; i < 2 && direct; ++i) direct = mapped(src_in[i], n_in[i], &dev_in[i]);
-  for (int i = 0; i < 3 && direct; ++i) direct = mapped(dst_out[i], n_out[i], &dev_out[i]);
+  // One graph per (batch, outputs wanted): copy-in kernel -> the step's kernels -> copy-out
+  // kernel, so a call is one graph launch and one synchronisation.
   GraphEntry* ge = nullptr;
-  int rc;
-  if (direct) {
-    CopySegs cin = {}, cout = {};
-    cin.count = 2;
-    cin.src[0] = static_cast<const uint4*>(dev_in[0]);
-    cin.dst[0] = reinterpret_cast<uint4*>(din);
-    cin.n[0] = n_attn / 16;
-    cin.src[1] = static_cast<const uint4*>(dev_in[1]);
-    cin.dst[1] = reinterpret_cast<uint4*>(din + o_res);
-    cin.n[1] = n_res / 16;
-    const char* from[3] = {dout, dout + o_idx, dout + o_gate};
-    for (int i = 0; i < 3; ++i)
-      if (dev_out[i]) {
-        cout.src[cout.count] = reinterpret_cast<const uint4*>(from[i]);
-        cout.dst[cout.count] = static_cast<uint4*>(dev_out[i]);
-        cout.n[cout.count] = n_out[i] / 16;
-        ++cout.count;
-      }
-    const void* key[5] = {attn_out_host, residual_in_host, out_host, topk_idx_host, topk_gate_host};
-    rc = get_graph(h, batch, din, din + o_res, dout, didx, dgate, &ge, 2, &cin, &cout, key);
-  } else {
-    // One graph per (batch, outputs wanted): copy-in kernel -> the step's kernels -> copy-out
-    // kernel, through the handle's pinned staging.
-    const CopySegs cin = one_seg(h->pin_in_dev, din, in_used), cout = one_seg(dout, h->pin_out_dev, out_used);
-    rc = get_graph(h, batch, din, din + o_res, dout, didx, dgate, &ge, 1, &cin, &cout);
-    if (rc == MOE_OK) {
-      std::memcpy(pin, attn_out_host, n_attn);
-      std::memcpy(pin + o_res, residual_in_host, n_res);
-    }
-  }
+  int rc = get_graph(h, batch, din, din + o_res, dout, topk_idx_host ? (int32_t*)(dout + o_idx) : nullptr,
+                     topk_gate_host ? (float*)(dout + o_gate) : nullptr, &ge, true, in_used, out_used);
   if (rc) return rc;
+  std::memcpy(pin, attn_out_host, n_attn);
+  std::memcpy(pin + o_res, residual_in_host, n_res);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaGraphLaunch(ge->exec, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
@@ -555,11 +482,9 @@ int moe_decode_step_host(moe_decode_handle* h, int batch, const void* attn_out_h
     return MOE_ERR_CUDA;
   }
   h->last_batch = batch;
-  if (!direct) {
-    std::memcpy(out_host, pout, n_res);
-    if (topk_idx_host) std::memcpy(topk_idx_host, pout + o_idx, n_tk);
-    if (topk_gate_host) std::memcpy(topk_gate_host, pout + o_gate, n_tk);
-  }
+  std::memcpy(out_host, pout, n_res);
+  if (topk_idx_host) std::memcpy(topk_idx_host, pout + o_idx, n_tk);
+  if (topk_gate_host) std::memcpy(topk_gate_host, pout + o_gate, n_tk);
   return MOE_OK;
 }
 

@@ -153,9 +153,8 @@ def test_host_buffer_step_matches_device_step():
 
 @pytest.mark.gpu
 def test_host_buffer_step_pinned_caller_buffers():
-    """The caller's own pinned buffers: the graph copies straight from and to them (no host
-    gather or scatter); results equal the device step's, on a new graph and its replay, and
-    a mix with pageable outputs falls back to the staging copies."""
+    """Pinned host buffers of the caller (torch pin_memory) and a mix with pageable outputs:
+    results equal the device step's, on a new graph and on its replay."""
     torch = pytest.importorskip("torch")
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
