@@ -104,14 +104,14 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
   pdl_wait();  // attn_out and residual may come from the previous kernel
   constexpr int kRI = 2;  // rows per interleaved pass (a stage is two rows at d_o = 8192)
   const int qbase = (d_o / 8) * warp / kCW, qpw = (d_o / 8) * (warp + 1) / kCW - qbase;
-  float xa[NT][kCPLf][8];
+  uint4 xa[NT][kCPLf];  // attn_out stays packed bf16 (mixed-precision FMAs)
 #pragma unroll
   for (int t = 0; t < NT; ++t)
 #pragma unroll
     for (int j = 0; j < kCPLf; ++j) {
       uint4 u = make_uint4(0, 0, 0, 0);
       if (t < B && cvalid(qpw, j, lane)) u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)(qbase + j * 32 + lane) * 8);
-      unpack8f(u, xa[t][j]);
+      xa[t][j] = u;
     }
   int it = 0;
   for (int r = r0; r < r1; r += RS, ++it) {
@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
 #pragma unroll
       for (int k = 0; k < kRI; ++k) rp[k] = st + (size_t)min(j0 + k, n - 1) * d_o;
       float v[kRI * NT];
-      rows_dot<NT, kRI>(rp, n - j0, xa, qbase, qpw, lane, v);
+      rows_dot_bf<NT, kRI>(rp, n - j0, xa, qbase, qpw, lane, v);
       const float tot = warp_reduce_multi<kRI * NT>(v, lane);
       const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
       if (multi_writer<kRI * NT>(lane) && j < n) part[((r - r0 + j) * kCW + warp) * NT + t] = tot;
@@ -1020,7 +1020,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
     int nslot = 0;
     {
       constexpr int kRI = 2;
-      float xa[NT][kCPLf][8];
+      uint4 xa[NT][kCPLf];  // attn_out stays packed bf16 (mixed-precision FMAs)
 #pragma unroll
       for (int t = 0; t < NT; ++t)
 #pragma unroll
@@ -1028,7 +1028,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
           uint4 u = make_uint4(0, 0, 0, 0);
           if (t < B && cvalid(qpw_o, j, lane))
             u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)(qbase_o + j * 32 + lane) * 8);
-          unpack8f(u, xa[t][j]);
+          xa[t][j] = u;
         }
       while (true) {
         const int s = itO % SO;
@@ -1048,7 +1048,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
 #pragma unroll
           for (int k = 0; k < kRI; ++k) rp[k] = st + (size_t)min(j0 + k, n - 1) * d_o;
           float v[kRI * NT];
-          rows_dot<NT, kRI>(rp, n - j0, xa, qbase_o, qpw_o, lane, v);
+          rows_dot_bf<NT, kRI>(rp, n - j0, xa, qbase_o, qpw_o, lane, v);
           const float tot = warp_reduce_multi<kRI * NT>(v, lane);
           const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
           if (multi_writer<kRI * NT>(lane) && j < n) opart[(((size_t)nslot * RS + j) * kCW + warp) * NT + t] = tot;

@@ -90,6 +90,72 @@ __device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr,
     }
 }
 
+// d = a * b + c for the bf16 in the low (hi = false) or high half of a and of b, in fp32: the
+// product of two bf16 values is exact in fp32, so this rounds exactly like fmaf on the
+// unpacked values (one instruction instead of two unpacks and an FMA).
+template <bool HI>
+__device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float c) {
+  float d;
+  if (HI)
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(c));
+  else
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(c));
+  return d;
+}
+
+// rows_dot for an activation that is itself bf16 (attn_out): x is kept packed, 8 values per
+// uint4 chunk, and each product is one mixed-precision FMA.  The accumulators and their order
+// are rows_dot's (even elements in .x, odd in .y, kA pairs), so the sums are bit-identical.
+template <int NT, int R, int CPL>
+__device__ __forceinline__ void rows_dot_bf(const uint16_t* const (&rp)[R], int nr, const uint4 (&x)[NT][CPL],
+                                            int qbase, int qpw, int lane, float (&out)[R * NT]) {
+  constexpr int kA = (R * NT >= 4) ? 1 : 4 / (R * NT);
+  uint4 w[R][CPL];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < CPL; ++j)
+      w[r][j] = (r < nr && cvalid(qpw, j, lane))
+                    ? *reinterpret_cast<const uint4*>(rp[r] + (size_t)(qbase + j * 32 + lane) * 8)
+                    : make_uint4(0, 0, 0, 0);
+  float2 acc[R][NT][kA];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int e = 0; e < kA; ++e) acc[r][t][e] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < CPL; ++j)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint32_t wv[4] = {w[r][j].x, w[r][j].y, w[r][j].z, w[r][j].w};
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const uint32_t xv[4] = {x[t][j].x, x[t][j].y, x[t][j].z, x[t][j].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2& a = acc[r][t][e % kA];
+          a.x = fma_bf16<false>(wv[e], xv[e], a.x);
+          a.y = fma_bf16<true>(wv[e], xv[e], a.y);
+        }
+      }
+    }
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float v = 0.f;
+#pragma unroll
+      for (int e = 0; e < kA; ++e) v += acc[r][t][e].x + acc[r][t][e].y;
+      out[r * NT + t] = v;
+    }
+}
+
 // Warp sums of V per-lane values (V a power of two <= 32) with V - 1 + 5 - log2(V) shuffles
 // instead of 5 V: each halving step sends one value of every pair across the current lane
 // bit and keeps the other.  Every lane returns the total of value multi_index<V>(lane).
