@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
 //   CTA c owns rows [e0, e0 + nrows) of W_r: the whole slice is one bulk copy, issued before
 //   the dependency wait.  x is exact fp32 in registers.
 // =============================================================================
-template <int NT>
+template <int NT, int CPD>
 __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int G = gridDim.x, c = blockIdx.x;
@@ -212,9 +212,9 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
     if (lane == 0 && nrows > 0) mbar_drain(&full[0], 0, a.ws.err);
   } else {
     const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
-    float gam[kCPLf][8];
+    float gam[CPD][8];
 #pragma unroll
-    for (int j = 0; j < kCPLf; ++j) {
+    for (int j = 0; j < CPD; ++j) {
       uint4 u = make_uint4(0, 0, 0, 0);
       if (cvalid(qpw, j, lane)) u = ld_weight_u4(a.gamma + (size_t)(qbase + j * 32 + lane) * 8);
       unpack8f(u, gam[j]);
@@ -222,12 +222,12 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
     pdl_wait();  // h and the sums of h^2 come from the o_proj kernel
     if (c == 0 && tid == 0) a.ws.counters[kCntGateUp] = 0;  // the expert kernel's grid barrier count
     // h of the first token group, loaded while the sums of h^2 are reduced
-    float xr[NT][kCPLf][8];
+    float xr[NT][CPD][8];
     auto load_h = [&](int t0, int nt) {
 #pragma unroll
       for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int j = 0; j < kCPLf; ++j) {
+        for (int j = 0; j < CPD; ++j) {
           if (t < nt && cvalid(qpw, j, lane)) {
             const float* hp = a.ws.h + (size_t)(t0 + t) * d + (size_t)(qbase + j * 32 + lane) * 8;
             const float4 h0 = ld_act4(hp), h1 = ld_act4(hp + 4);
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
       for (int t = 0; t < NT; ++t) {
         const float r = (t < nt) ? rstd_s[t0 + t] : 0.f;
 #pragma unroll
-        for (int j = 0; j < kCPLf; ++j) {
+        for (int j = 0; j < CPD; ++j) {
           const int q = qbase + j * 32 + lane;
 #pragma unroll
           for (int e = 0; e < 8; ++e) xr[t][j][e] = xr[t][j][e] * r * gam[j][e];
@@ -638,7 +638,7 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
 //            holds elements [l*EPL, (l+1)*EPL) of each row and accumulates over all experts
 //            in registers; one warp reduction per (row, token) at the end.
 // =============================================================================
-template <int NT, int EPL>
+template <int NT, int EPL, int CPD>
 __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int kEPS = experts_per_stage(EPL);
@@ -684,12 +684,12 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   // x of every token, in registers (consumers).  Loaded after routing: the loads hit L2 and
   // land before the first weight stage, and holding x across the routing code would spill.
   const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
-  float xr[NT][kCPLf][8];
+  float xr[NT][CPD][8];
   if (warp < kCW) {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
-      for (int j = 0; j < kCPLf; ++j) {
+      for (int j = 0; j < CPD; ++j) {
         if (t < B && cvalid(qpw, j, lane)) {
           const float* xp = a.ws.x + (size_t)t * d + (size_t)(qbase + j * 32 + lane) * 8;
           const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
@@ -872,7 +872,7 @@ __device__ __forceinline__ void layer_exit(unsigned* counters) {
 
 }  // namespace
 
-template <int NT, int EPL>
+template <int NT, int EPL, int CPD>
 __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int kEPS = experts_per_stage(EPL);
@@ -1078,10 +1078,10 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
     {
       // h and gamma in one round of loads; the sum of h^2 over d from the same registers
       // (per lane, per warp, then the 15 warps in a fixed order: the same bits in every CTA)
-      float xr[NT][kCPLf][8];
-      float gam[kCPLf][8];
+      float xr[NT][CPD][8];
+      float gam[CPD][8];
 #pragma unroll
-      for (int j = 0; j < kCPLf; ++j) {
+      for (int j = 0; j < CPD; ++j) {
         uint4 u = make_uint4(0, 0, 0, 0);
         if (cvalid(qpw, j, lane)) u = ld_weight_u4(a.gamma + (size_t)(qbase + j * 32 + lane) * 8);
         unpack8f(u, gam[j]);
@@ -1089,7 +1089,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
 #pragma unroll
       for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int j = 0; j < kCPLf; ++j) {
+        for (int j = 0; j < CPD; ++j) {
           if (t < B && cvalid(qpw, j, lane)) {
             const float* hp = a.ws.h + (size_t)t * d + (size_t)(qbase + j * 32 + lane) * 8;
             const float4 h0 = ld_act4(hp), h1 = ld_act4(hp + 4);
@@ -1105,7 +1105,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
       for (int t = 0; t < NT; ++t) {
         float s2 = 0.f;
 #pragma unroll
-        for (int j = 0; j < kCPLf; ++j)
+        for (int j = 0; j < CPD; ++j)
 #pragma unroll
           for (int e = 0; e < 8; ++e) s2 = fmaf(xr[t][j][e], xr[t][j][e], s2);
         s2 = warp_sum(s2);
@@ -1121,7 +1121,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
         if (c == 0 && tid == 0 && t < B) a.ws.rstd[t] = rv[t];
       }
 #pragma unroll
-      for (int j = 0; j < kCPLf; ++j) {
+      for (int j = 0; j < CPD; ++j) {
         const int q = qbase + j * 32 + lane;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
@@ -1171,12 +1171,12 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   __syncthreads();  // the producer warp joins: logits are complete
 
   route_small_cta(a.ws.logits, B, E, a.k, a.user_idx, a.user_gate, a.ws.err, rt, sc, fb, c == 0);
-  float xr[NT][kCPLf][8];
+  float xr[NT][CPD][8];
   if (warp < kCW) {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
 #pragma unroll
-      for (int j = 0; j < kCPLf; ++j) {
+      for (int j = 0; j < CPD; ++j) {
         if (t < B && cvalid(qpw, j, lane)) {
           const float* xp = a.ws.x + (size_t)t * d + (size_t)(qbase + j * 32 + lane) * 8;
           const float4 x0 = ld_act4(xp), x1 = ld_act4(xp + 4);
@@ -1538,21 +1538,25 @@ cudaError_t set_small_attributes(size_t optin) {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100)
   SETS(k_oproj_f<1>);
   SETS(k_oproj_f<2>);
-  SETS(k_router_f<1>);
-  SETS(k_router_f<2>);
-  SETS((k_experts_f<1, 4>));
-  SETS((k_experts_f<2, 4>));
-  SETS((k_experts_f<1, 8>));
-  SETS((k_experts_f<2, 8>));
-  SETS((k_experts_f<1, 0>));
-  SETS((k_experts_f<2, 0>));
+#define SETS_D(k, ...) \
+  SETS((k<__VA_ARGS__, 2>)); \
+  SETS((k<__VA_ARGS__, 3>))
+  SETS_D(k_router_f, 1);
+  SETS_D(k_router_f, 2);
+  SETS_D(k_experts_f, 1, 4);
+  SETS_D(k_experts_f, 2, 4);
+  SETS_D(k_experts_f, 1, 8);
+  SETS_D(k_experts_f, 2, 8);
+  SETS_D(k_experts_f, 1, 0);
+  SETS_D(k_experts_f, 2, 0);
   SETS(k_router_big);
-  SETS((k_layer_f<1, 4>));
-  SETS((k_layer_f<2, 4>));
-  SETS((k_layer_f<1, 8>));
-  SETS((k_layer_f<2, 8>));
-  SETS((k_layer_f<1, 0>));
-  SETS((k_layer_f<2, 0>));
+  SETS_D(k_layer_f, 1, 4);
+  SETS_D(k_layer_f, 2, 4);
+  SETS_D(k_layer_f, 1, 8);
+  SETS_D(k_layer_f, 2, 8);
+  SETS_D(k_layer_f, 1, 0);
+  SETS_D(k_layer_f, 2, 0);
+#undef SETS_D
 #undef SETS
   return e;
 }
@@ -1562,6 +1566,45 @@ LayerArgs planned(const LayerArgs& a0, int grid, size_t optin) {
   LayerArgs a = a0;
   plan_small(a, grid, optin);
   return a;
+}
+
+// 8-element chunks per lane of a d-long activation slice over the 15 consumer warps: two cover
+// d <= 7680, three the rest of the supported range.  The smaller slice has no chunk slot that
+// is always empty (at d = 7168 a lane holds 1.9 chunks), so no loads or FMAs are spent on zeros.
+bool two_chunks(int d) { return d <= 8 * 32 * 2 * kCW; }
+
+template <int CPD>
+cudaError_t launch_router_d(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
+  return a.B == 1 ? launch_f(k_router_f<1, CPD>, grid, a.k2.smem, s, pdl, a)
+                  : launch_f(k_router_f<2, CPD>, grid, a.k2.smem, s, pdl, a);
+}
+
+template <int CPD>
+cudaError_t launch_experts_d(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
+  const int epl = a.I / 32;
+  const size_t sm = a.k3.smem;
+  if (epl == 4)
+    return a.B == 1 ? launch_f(k_experts_f<1, 4, CPD>, grid, sm, s, pdl, a, true)
+                    : launch_f(k_experts_f<2, 4, CPD>, grid, sm, s, pdl, a, true);
+  if (epl == 8)
+    return a.B == 1 ? launch_f(k_experts_f<1, 8, CPD>, grid, sm, s, pdl, a, true)
+                    : launch_f(k_experts_f<2, 8, CPD>, grid, sm, s, pdl, a, true);
+  return a.B == 1 ? launch_f(k_experts_f<1, 0, CPD>, grid, sm, s, pdl, a, true)
+                  : launch_f(k_experts_f<2, 0, CPD>, grid, sm, s, pdl, a, true);
+}
+
+template <int CPD>
+cudaError_t launch_layer_d(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
+  const int epl = a.I / 32;
+  const size_t sm = a.k1.smem;
+  if (epl == 4)
+    return a.B == 1 ? launch_f(k_layer_f<1, 4, CPD>, grid, sm, s, pdl, a, true)
+                    : launch_f(k_layer_f<2, 4, CPD>, grid, sm, s, pdl, a, true);
+  if (epl == 8)
+    return a.B == 1 ? launch_f(k_layer_f<1, 8, CPD>, grid, sm, s, pdl, a, true)
+                    : launch_f(k_layer_f<2, 8, CPD>, grid, sm, s, pdl, a, true);
+  return a.B == 1 ? launch_f(k_layer_f<1, 0, CPD>, grid, sm, s, pdl, a, true)
+                  : launch_f(k_layer_f<2, 0, CPD>, grid, sm, s, pdl, a, true);
 }
 }  // namespace
 
@@ -1576,30 +1619,18 @@ cudaError_t launch_router_s(const LayerArgs& a0, int grid, cudaStream_t s, bool 
   a.k2.smem = up128((size_t)a.k2.rows_max * a.d * 2) + up128((size_t)a.k2.rows_max * kCW * 2 * 4 + 64 * 4) +
               8 + 32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
   (void)optin;
-  return a.B == 1 ? launch_f(k_router_f<1>, grid, a.k2.smem, s, pdl, a) : launch_f(k_router_f<2>, grid, a.k2.smem, s, pdl, a);
+  return two_chunks(a.d) ? launch_router_d<2>(a, grid, s, pdl) : launch_router_d<3>(a, grid, s, pdl);
 }
 
 cudaError_t launch_experts_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   const LayerArgs a = planned(a0, grid, optin);
-  const int epl = a.I / 32;
-  const size_t sm = a.k3.smem;
-  if (epl == 4)
-    return a.B == 1 ? launch_f(k_experts_f<1, 4>, grid, sm, s, pdl, a, true) : launch_f(k_experts_f<2, 4>, grid, sm, s, pdl, a, true);
-  if (epl == 8)
-    return a.B == 1 ? launch_f(k_experts_f<1, 8>, grid, sm, s, pdl, a, true) : launch_f(k_experts_f<2, 8>, grid, sm, s, pdl, a, true);
-  return a.B == 1 ? launch_f(k_experts_f<1, 0>, grid, sm, s, pdl, a, true) : launch_f(k_experts_f<2, 0>, grid, sm, s, pdl, a, true);
+  return two_chunks(a.d) ? launch_experts_d<2>(a, grid, s, pdl) : launch_experts_d<3>(a, grid, s, pdl);
 }
 
 cudaError_t launch_layer_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   LayerArgs a = a0;
   if (!plan_fused(a, grid, optin)) return cudaErrorInvalidConfiguration;
-  const int epl = a.I / 32;
-  const size_t sm = a.k1.smem;
-  if (epl == 4)
-    return a.B == 1 ? launch_f(k_layer_f<1, 4>, grid, sm, s, pdl, a, true) : launch_f(k_layer_f<2, 4>, grid, sm, s, pdl, a, true);
-  if (epl == 8)
-    return a.B == 1 ? launch_f(k_layer_f<1, 8>, grid, sm, s, pdl, a, true) : launch_f(k_layer_f<2, 8>, grid, sm, s, pdl, a, true);
-  return a.B == 1 ? launch_f(k_layer_f<1, 0>, grid, sm, s, pdl, a, true) : launch_f(k_layer_f<2, 0>, grid, sm, s, pdl, a, true);
+  return two_chunks(a.d) ? launch_layer_d<2>(a, grid, s, pdl) : launch_layer_d<3>(a, grid, s, pdl);
 }
 
 cudaError_t launch_router_big(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {

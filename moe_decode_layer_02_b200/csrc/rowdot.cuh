@@ -29,6 +29,31 @@ __device__ __forceinline__ void unpack8f(uint4 w, float* f) {
 // Chunk of lane `lane` in warp w's K slice: q = w * qpw + j * 32 + lane, valid if j*32+lane < qpw.
 __device__ __forceinline__ bool cvalid(int qpw, int j, int lane) { return j * 32 + lane < qpw; }
 
+// 16 bytes from shared memory at a 32-bit shared-window address.  The row pointers of the dot
+// products below all point into the ring in shared memory; addressing them through the shared
+// window keeps the per-chunk address arithmetic 32-bit (with generic pointers the same loop
+// measured about 15% slower).  volatile: the load stays after the mbarrier wait that made the
+// stage's bytes visible, like every other volatile asm around it.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Loads the chunks of R rows (row pointers into shared memory) that lane `lane` covers; rows
+// r >= nr and chunks past the warp's slice read as zeros.
+template <int R, int CPL>
+__device__ __forceinline__ void load_row_chunks(const uint16_t* const (&rp)[R], int nr, int qbase, int qpw, int lane,
+                                                uint4 (&w)[R][CPL]) {
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const uint32_t base = (uint32_t)__cvta_generic_to_shared(rp[r]) + (uint32_t)(qbase + lane) * 16u;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j)
+      w[r][j] = (r < nr && cvalid(qpw, j, lane)) ? lds128(base + (uint32_t)j * 512u) : make_uint4(0, 0, 0, 0);
+  }
+}
+
 // d = a * b + d on a pair of fp32 lanes with one instruction (sm_100 packed FMA; each lane
 // rounds exactly like fmaf).
 __device__ __forceinline__ void ffma2(float2& d, float a0, float a1, float b0, float b1) {
@@ -42,7 +67,7 @@ __device__ __forceinline__ void ffma2(float2& d, float a0, float a1, float b0, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// Per-lane partial dots of R bf16 rows (shared memory) with NT register slices of the
+// Per-lane partial dots of R bf16 rows (shared memory only) with NT register slices of the
 // activations: out[r * NT + t].  Rows r >= nr contribute zeros.  All chunk loads of all
 // rows are issued before the first FMA; the accumulators are independent chains of packed
 // FMAs (an even and an odd element per instruction, kA pairs per row and token), so a
@@ -53,13 +78,7 @@ __device__ __forceinline__ void rows_dot(const uint16_t* const (&rp)[R], int nr,
                                          int qbase, int qpw, int lane, float (&out)[R * NT]) {
   constexpr int kA = (R * NT >= 4) ? 1 : 4 / (R * NT);  // accumulator pairs per (row, token)
   uint4 w[R][CPL];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int j = 0; j < CPL; ++j)
-      w[r][j] = (r < nr && cvalid(qpw, j, lane))
-                    ? *reinterpret_cast<const uint4*>(rp[r] + (size_t)(qbase + j * 32 + lane) * 8)
-                    : make_uint4(0, 0, 0, 0);
+  load_row_chunks<R, CPL>(rp, nr, qbase, qpw, lane, w);
   float2 acc[R][NT][kA];
 #pragma unroll
   for (int r = 0; r < R; ++r)
@@ -115,13 +134,7 @@ __device__ __forceinline__ void rows_dot_bf(const uint16_t* const (&rp)[R], int 
                                             int qbase, int qpw, int lane, float (&out)[R * NT]) {
   constexpr int kA = (R * NT >= 4) ? 1 : 4 / (R * NT);
   uint4 w[R][CPL];
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int j = 0; j < CPL; ++j)
-      w[r][j] = (r < nr && cvalid(qpw, j, lane))
-                    ? *reinterpret_cast<const uint4*>(rp[r] + (size_t)(qbase + j * 32 + lane) * 8)
-                    : make_uint4(0, 0, 0, 0);
+  load_row_chunks<R, CPL>(rp, nr, qbase, qpw, lane, w);
   float2 acc[R][NT][kA];
 #pragma unroll
   for (int r = 0; r < R; ++r)
