@@ -527,8 +527,11 @@ __device__ void grid_barrier(unsigned* count, unsigned target, volatile int* abo
 // Phase B of the batch <= 2 expert kernels (consumer warps): out = bf16(h + sum over the
 // union experts of W_down[e] rows [i0, i0 + nrows) . a_s[e]), the W_down blocks arriving in
 // the B ring.  A stage holds EPS experts' blocks of this CTA's rows; every load of a stage is
-// issued before its FMAs.  Warp w owns rows w, w + 15, ...; lane l holds elements
-// [l * epl, (l + 1) * epl) of each row and accumulates over all experts in registers.
+// issued before its FMAs (software-pipelining one expert ahead instead measured slower: fewer
+// loads in flight).  Warp w owns rows w, w + 15, ...; lane l holds elements
+// [l * epl, (l + 1) * epl) of each row and accumulates over all experts in registers: with
+// 4 or 8 elements per lane as one packed fp32x2 accumulator per (row, token) (even elements in
+// .x, odd in .y, experts in ascending union order), then .x + .y and one warp reduction.
 template <int NT, int EPL>
 __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned char* ring, size_t SB_B, int SBn,
                                              uint64_t* fullB, uint64_t* emptyB, volatile int* abort_flag,
@@ -538,10 +541,16 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
   const int d = a.d, I = a.I, B = a.B;
   const int epl = (EPL > 0) ? EPL : I / 32;
   float acc[kRPW][NT];
+  float2 acc2[kRPW][NT];
 #pragma unroll
   for (int i = 0; i < kRPW; ++i)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) acc[i][t] = 0.f;
+    for (int t = 0; t < NT; ++t) { acc[i][t] = 0.f; acc2[i][t] = make_float2(0.f, 0.f); }
+  // h of the (row, token) this lane writes at the end, loaded now so its latency is hidden
+  const int vi_w = multi_index<kRPW * NT>(lane), i_w = vi_w / NT, t_w = vi_w % NT, rl_w = warp + kCW * i_w;
+  const bool writer = multi_writer<kRPW * NT>(lane) && rl_w < nrows && t_w < B;
+  const size_t o_w = (size_t)t_w * d + i0 + rl_w;
+  const float h_w = writer ? ld_act(&a.ws.h[o_w]) : 0.f;
   int g = 0;
   for (int u0 = 0; u0 < U && nrows > 0; u0 += kEPS, ++g) {
     const int s = g % SBn, ne = min(kEPS, U - u0);
@@ -551,14 +560,17 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
       using WT = typename std::conditional<EPL == 4, uint2, uint4>::type;
       float av[kEPS][NT][EPL];
       WT wv[kEPS][kRPW];
+      // 32-bit shared-window addresses (the stage and a_s are both in shared memory)
+      const uint32_t st_l = (uint32_t)__cvta_generic_to_shared(st) + (uint32_t)(lane * EPL * 2);
+      const uint32_t as_l = (uint32_t)__cvta_generic_to_shared(a_s) + (uint32_t)(lane * EPL * 4);
 #pragma unroll
       for (int e = 0; e < kEPS; ++e) {
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          const float* ap = a_s + ((size_t)(u0 + min(e, ne - 1)) * NT + t) * I + lane * EPL;
+          const uint32_t ap = as_l + (uint32_t)(((u0 + min(e, ne - 1)) * NT + t) * I) * 4u;
 #pragma unroll
           for (int x = 0; x < EPL; x += 4) {
-            const float4 f = (e < ne) ? *reinterpret_cast<const float4*>(ap + x) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 f = (e < ne) ? lds128f(ap + (uint32_t)x * 4u) : make_float4(0.f, 0.f, 0.f, 0.f);
             av[e][t][x] = f.x; av[e][t][x + 1] = f.y; av[e][t][x + 2] = f.z; av[e][t][x + 3] = f.w;
           }
         }
@@ -566,7 +578,11 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
         for (int i = 0; i < kRPW; ++i) {
           const int rl = warp + kCW * i;
           WT w{};
-          if (e < ne && rl < nrows) w = *reinterpret_cast<const WT*>(st + ((size_t)e * nrows + rl) * I + lane * EPL);
+          if (e < ne && rl < nrows) {
+            const uint32_t wa = st_l + (uint32_t)((e * nrows + rl) * I) * 2u;
+            if constexpr (EPL == 4) w = lds64(wa);
+            else w = lds128(wa);
+          }
           wv[e][i] = w;
         }
       }
@@ -582,12 +598,9 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
             unpack8f(reinterpret_cast<const uint4&>(wv[e][i]), wf);
           }
 #pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            float sdot = 0.f;
+          for (int t = 0; t < NT; ++t)
 #pragma unroll
-            for (int x = 0; x < EPL; ++x) sdot = fmaf(wf[x], av[e][t][x], sdot);
-            acc[i][t] += sdot;
-          }
+            for (int x = 0; x < EPL; x += 2) ffma2(acc2[i][t], wf[x], wf[x + 1], av[e][t][x], av[e][t][x + 1]);
         }
     } else {  // any other I: one expert per stage, epl <= 16 elements per lane
       const float* ap = a_s + (size_t)u0 * NT * I + lane * epl;
@@ -615,13 +628,11 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
 #pragma unroll
     for (int i = 0; i < kRPW; ++i)
 #pragma unroll
-      for (int t = 0; t < NT; ++t) v[i * NT + t] = acc[i][t];
+      for (int t = 0; t < NT; ++t) v[i * NT + t] = acc[i][t] + (acc2[i][t].x + acc2[i][t].y);
     const float tot = warp_reduce_multi<kRPW * NT>(v, lane);
-    const int vi = multi_index<kRPW * NT>(lane), i = vi / NT, t = vi % NT, rl = warp + kCW * i;
-    if (multi_writer<kRPW * NT>(lane) && rl < nrows && t < B) {
-      const size_t o = (size_t)t * d + i0 + rl;
-      const __nv_bfloat16 bv = __float2bfloat16_rn(ld_act(&a.ws.h[o]) + tot);
-      a.out[o] = *reinterpret_cast<const uint16_t*>(&bv);
+    if (writer) {
+      const __nv_bfloat16 bv = __float2bfloat16_rn(h_w + tot);
+      a.out[o_w] = *reinterpret_cast<const uint16_t*>(&bv);
     }
   }
 }
