@@ -78,9 +78,9 @@ enum {
  *                    router matrix, RMSNorm scale and the leading 16 MB of its W_o,
  *                    split by the CTA that reads them), issued once layer l's own
  *                    router rows are in flight; no extra kernel
- *   force_variant    0: kernels by batch size (B = 1: one fused layer kernel; B = 2:
- *                    o_proj, router, small-M expert kernel; above: o_proj, router,
- *                    gate/up, down);
+ *   force_variant    0: kernels by batch size (B = 1: one fused layer kernel; B = 2 to 4
+ *                    with B * top_k <= 64: o_proj, router, small-M expert kernel; above:
+ *                    o_proj, router, gate/up, down);
  *                    1: at B = 1 too the three small-batch kernels (testing);
  *                    2: the large-batch kernels at every batch size (testing);
  *                    3: at B <= 2 the layer kernel whose expert phase is ordered by

@@ -47,7 +47,20 @@ namespace {
 static_assert(kThreadsS == kRouteThreads, "the expert kernel routes with all of its threads");
 
 // Phase B experts per stage for EPL elements per lane (registers bound it).
-__host__ __device__ constexpr int experts_per_stage(int epl) { return epl == 4 ? 4 : (epl == 8 ? 2 : 1); }
+// Union experts per phase-B stage: the stage's activations of every token are held in
+// registers (kEPS * NT * EPL floats per lane), so four tokens take half as many.
+__host__ __device__ constexpr int experts_per_stage(int epl, int nt) {
+  return epl == 4 ? (nt > 2 ? 2 : 4) : (epl == 8 ? (nt > 2 ? 1 : 2) : 1);
+}
+
+// Phase B's gated activations in shared memory.  Up to two tokens: dense, [U][NT][I] with
+// zeros where a token did not select the union expert.  Four tokens (where the dense form
+// would take up to 128 KB): one row per entry, [B K][I], then the entry of each (union
+// expert, token) pair, [min(E, B K)][NT] ints (-1 where the token did not select it).
+__host__ __device__ constexpr size_t a_s_floats(int B, int K, int E, int I, int NT) {
+  return NT <= 2 ? (size_t)(E < B * K ? E : B * K) * NT * I
+                 : (size_t)B * K * I + (((size_t)(E < B * K ? E : B * K) * NT + 3) & ~size_t(3));
+}
 
 }  // namespace
 
@@ -535,9 +548,10 @@ __device__ void grid_barrier(unsigned* count, unsigned target, volatile int* abo
 template <int NT, int EPL>
 __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned char* ring, size_t SB_B, int SBn,
                                              uint64_t* fullB, uint64_t* emptyB, volatile int* abort_flag,
-                                             const float* a_s, int U, int i0, int nrows, int warp, int lane) {
+                                             const float* a_s, const int* ent_of, int U, int i0, int nrows, int warp,
+                                             int lane) {
   constexpr int kRPW = 4;  // rows per warp (rows_max <= 60)
-  constexpr int kEPS = experts_per_stage(EPL);
+  constexpr int kEPS = experts_per_stage(EPL, NT);
   const int d = a.d, I = a.I, B = a.B;
   const int epl = (EPL > 0) ? EPL : I / 32;
   float acc[kRPW][NT];
@@ -567,10 +581,12 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
       for (int e = 0; e < kEPS; ++e) {
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-          const uint32_t ap = as_l + (uint32_t)(((u0 + min(e, ne - 1)) * NT + t) * I) * 4u;
+          // dense rows (u, t) up to two tokens; one row per entry, looked up, with four
+          const int en = NT <= 2 ? ((e < ne) ? (u0 + e) * NT + t : -1) : ((e < ne) ? ent_of[(u0 + e) * NT + t] : -1);
+          const uint32_t ap = as_l + (uint32_t)(max(en, 0) * I) * 4u;
 #pragma unroll
           for (int x = 0; x < EPL; x += 4) {
-            const float4 f = (e < ne) ? lds128f(ap + (uint32_t)x * 4u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 f = (en >= 0) ? lds128f(ap + (uint32_t)x * 4u) : make_float4(0.f, 0.f, 0.f, 0.f);
             av[e][t][x] = f.x; av[e][t][x + 1] = f.y; av[e][t][x + 2] = f.z; av[e][t][x + 3] = f.w;
           }
         }
@@ -603,7 +619,6 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
             for (int x = 0; x < EPL; x += 2) ffma2(acc2[i][t], wf[x], wf[x + 1], av[e][t][x], av[e][t][x + 1]);
         }
     } else {  // any other I: one expert per stage, epl <= 16 elements per lane
-      const float* ap = a_s + (size_t)u0 * NT * I + lane * epl;
 #pragma unroll
       for (int i = 0; i < kRPW; ++i) {
         const int rl = warp + kCW * i;
@@ -611,10 +626,13 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
           const uint16_t* wr = st + (size_t)rl * I + lane * epl;
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
+            const int en = NT <= 2 ? u0 * NT + t : ent_of[u0 * NT + t];
+            if (en < 0) continue;  // zero contribution, as a zero activation would give
+            const float* ap = a_s + (size_t)en * I + lane * epl;
             float sdot = 0.f;
 #pragma unroll
             for (int x = 0; x < 16; ++x)
-              if (x < epl) sdot = fmaf(bf16f(wr[x]), ap[(size_t)t * I + x], sdot);
+              if (x < epl) sdot = fmaf(bf16f(wr[x]), ap[x], sdot);
             acc[i][t] += sdot;
           }
         }
@@ -652,7 +670,7 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
 template <int NT, int EPL, int CPD>
 __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kEPS = experts_per_stage(EPL);
+  constexpr int kEPS = experts_per_stage(EPL, NT);
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, I = a.I, B = a.B;
   const int SA = a.k3.stages, PS = a.k3.rows_per_stage, PM = a.k3.rows_max;
@@ -660,8 +678,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   const uint32_t row_bytes = (uint32_t)d * 2u, drow_bytes = (uint32_t)I * 2u;
   const size_t SA_B = al128((size_t)2 * PS * row_bytes), SB_B = al128((size_t)kEPS * RM * drow_bytes);
   const size_t region = std::max((size_t)SA * SA_B, (size_t)SBn * SB_B);
-  const size_t scratch_f =
-      std::max((size_t)PM * 2 * kCW * NT, (size_t)std::min(a.E, B * a.k) * NT * I);  // floats
+  const size_t scratch_f = std::max((size_t)PM * 2 * kCW * NT, a_s_floats(B, a.k, a.E, I, NT));  // floats
   long long lo, hi;
   split_range(d, G, c, lo, hi);
   const int i0 = (int)lo, nrows = (int)(hi - lo);
@@ -669,11 +686,12 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   unsigned char* ring = smem;
   float* part = reinterpret_cast<float*>(ring + region);  // phase A partials, then phase B's a
   float* a_s = part;
-  SmallRoute* rt = reinterpret_cast<SmallRoute*>(smem + al128(region + scratch_f * sizeof(float)));
-  RouteScratch* sc = reinterpret_cast<RouteScratch*>(rt + 1);
+  using RO = RouteOf<NT>;
+  auto* rt = reinterpret_cast<typename RO::Route*>(smem + al128(region + scratch_f * sizeof(float)));
+  auto* sc = reinterpret_cast<typename RO::Scratch*>(rt + 1);
   float* fb = reinterpret_cast<float*>(sc + 1);
   uint64_t* fullA = reinterpret_cast<uint64_t*>(
-      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + 2 * 2 * kCandStride) - smem)));
+      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + RO::kFbFloats) - smem)));
   uint64_t* emptyA = fullA + kMaxStages;
   uint64_t* fullB = emptyA + kMaxStages;
   uint64_t* emptyB = fullB + kMaxStages;
@@ -691,7 +709,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   pdl_trigger();
 
   // barriers inside also publish the ring init
-  route_small_cta(a.ws.logits, B, a.E, a.k, a.user_idx, a.user_gate, a.ws.err, rt, sc, fb, c == 0);
+  route_small_cta<NT>(a.ws.logits, B, a.E, a.k, a.user_idx, a.user_gate, a.ws.err, rt, sc, fb, c == 0);
   // x of every token, in registers (consumers).  Loaded after routing: the loads hit L2 and
   // land before the first weight stage, and holding x across the routing code would spill.
   const int qbase = (d / 8) * warp / kCW, qpw = (d / 8) * (warp + 1) / kCW - qbase;
@@ -818,22 +836,41 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   grid_barrier(&a.ws.counters[kCntGateUp], gridDim.x, abort_flag, a.ws.err);
 
   // ---- phase B (consumers) ------------------------------------------------------------
-  // a_s[u][t][:] = gate * a of (union expert u, token t), zero where t did not select u, so
-  // the accumulation below is branch-free.
-  for (int z = tid; z < U * NT * (I / 4); z += kCT) {
-    const int cq = z % (I / 4), ut = z / (I / 4), t = ut % NT, u = ut / NT;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
-      if (rt->ent_tok[en] == t) {
-        const float g = rt->ent_gate[en];
-        const float4 x4 = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
-        v = make_float4(g * x4.x, g * x4.y, g * x4.z, g * x4.w);
-      }
-    *reinterpret_cast<float4*>(a_s + ((size_t)u * NT + t) * I + cq * 4) = v;
+  // Up to two tokens a_s[u][t][:] = gate * a of (union expert u, token t), zero where t did
+  // not select u; with four, a_s[en][:] = gate * a of entry en and ent_of[u][t] = the entry of
+  // (u, t), -1 where t did not select u (phase B then adds nothing for that pair, as a zero
+  // activation would).
+  int* ent_of = reinterpret_cast<int*>(a_s + (size_t)B * a.k * I);  // four tokens only
+  if constexpr (NT <= 2) {
+    for (int z = tid; z < U * NT * (I / 4); z += kCT) {
+      const int cq = z % (I / 4), ut = z / (I / 4), t = ut % NT, u = ut / NT;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+        if (rt->ent_tok[en] == t) {
+          const float g = rt->ent_gate[en];
+          const float4 x4 = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
+          v = make_float4(g * x4.x, g * x4.y, g * x4.z, g * x4.w);
+        }
+      *reinterpret_cast<float4*>(a_s + ((size_t)u * NT + t) * I + cq * 4) = v;
+    }
+  } else {
+    for (int z = tid; z < rt->n_ent * (I / 4); z += kCT) {
+      const int cq = z % (I / 4), en = z / (I / 4);
+      const float g = rt->ent_gate[en];
+      const float4 x4 = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
+      *reinterpret_cast<float4*>(a_s + (size_t)en * I + cq * 4) = make_float4(g * x4.x, g * x4.y, g * x4.z, g * x4.w);
+    }
+    for (int z = tid; z < U * NT; z += kCT) {
+      const int u = z / NT, t = z - u * NT;
+      int f = -1;
+      for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+        if (rt->ent_tok[en] == t) f = en;
+      ent_of[z] = f;
+    }
   }
   csync();
 
-  combine_down<NT, EPL>(a, ring, SB_B, SBn, fullB, emptyB, abort_flag, a_s, U, i0, nrows, warp, lane);
+  combine_down<NT, EPL>(a, ring, SB_B, SBn, fullB, emptyB, abort_flag, a_s, ent_of, U, i0, nrows, warp, lane);
 }
 
 // =============================================================================
@@ -886,7 +923,7 @@ __device__ __forceinline__ void layer_exit(unsigned* counters) {
 template <int NT, int EPL, int CPD>
 __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int kEPS = experts_per_stage(EPL);
+  constexpr int kEPS = experts_per_stage(EPL, NT);
   const int G = gridDim.x, c = blockIdx.x;
   const int d = a.d, d_o = a.d_o, I = a.I, B = a.B, E = a.E;
   const int SO = a.k1.stages, RS = a.k1.rows_per_stage, RM = a.k1.rows_max;
@@ -896,7 +933,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   const uint32_t orow_bytes = (uint32_t)d_o * 2u, row_bytes = (uint32_t)d * 2u, drow_bytes = (uint32_t)I * 2u;
   const size_t SO_B = std::max(al128((size_t)RS * orow_bytes), al128(row_bytes));  // a W_r row fits a stage
   const size_t SA_B = al128((size_t)2 * PS * row_bytes), SB_B = al128((size_t)kEPS * RM * drow_bytes);
-  const size_t a_s_bytes = (size_t)std::min(E, B * a.k) * NT * I * 4;
+  const size_t a_s_bytes = a_s_floats(B, a.k, E, I, NT) * 4;
   const size_t region =
       std::max(std::max((size_t)SO * SO_B, (size_t)SA * SA_B), (size_t)SBn * SB_B + a_s_bytes);
   const int UC = oproj_unit_cap(d, RS, G);
@@ -912,11 +949,12 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   float* rstd_s = part + RMr * kCW * NT;  // router
   // phase B: after phase B's stages (phase A's fills have all landed and been read by then)
   float* a_s = reinterpret_cast<float*>(ring + (size_t)SBn * SB_B);
-  SmallRoute* rt = reinterpret_cast<SmallRoute*>(smem + al128(region + scratch_f * sizeof(float)));
-  RouteScratch* sc = reinterpret_cast<RouteScratch*>(rt + 1);
+  using RO = RouteOf<NT>;
+  auto* rt = reinterpret_cast<typename RO::Route*>(smem + al128(region + scratch_f * sizeof(float)));
+  auto* sc = reinterpret_cast<typename RO::Scratch*>(rt + 1);
   float* fb = reinterpret_cast<float*>(sc + 1);
   uint64_t* fullO = reinterpret_cast<uint64_t*>(
-      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + 2 * 2 * kCandStride) - smem)));
+      smem + al128(static_cast<size_t>(reinterpret_cast<unsigned char*>(fb + RO::kFbFloats) - smem)));
   uint64_t* emptyO = fullO + kMaxStages;
   uint64_t* fullA = emptyO + kMaxStages;
   uint64_t* emptyA = fullA + kMaxStages;
@@ -1181,7 +1219,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   }
   __syncthreads();  // the producer warp joins: logits are complete
 
-  route_small_cta(a.ws.logits, B, E, a.k, a.user_idx, a.user_gate, a.ws.err, rt, sc, fb, c == 0);
+  route_small_cta<NT>(a.ws.logits, B, E, a.k, a.user_idx, a.user_gate, a.ws.err, rt, sc, fb, c == 0);
   float xr[NT][CPD][8];
   if (warp < kCW) {
 #pragma unroll
@@ -1303,19 +1341,36 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
   if (tid == 0) layer_exit(a.ws.counters);
 
   // ---- phase B (consumers) ------------------------------------------------------------
-  for (int z = tid; z < U * NT * (I / 4); z += kCT) {
-    const int cq = z % (I / 4), ut = z / (I / 4), t = ut % NT, u = ut / NT;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
-      if (rt->ent_tok[en] == t) {
-        const float g = rt->ent_gate[en];
-        const float4 x4 = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
-        v = make_float4(g * x4.x, g * x4.y, g * x4.z, g * x4.w);
-      }
-    *reinterpret_cast<float4*>(a_s + ((size_t)u * NT + t) * I + cq * 4) = v;
+  int* ent_of = reinterpret_cast<int*>(a_s + (size_t)B * a.k * I);  // four tokens only
+  if constexpr (NT <= 2) {
+    for (int z = tid; z < U * NT * (I / 4); z += kCT) {
+      const int cq = z % (I / 4), ut = z / (I / 4), t = ut % NT, u = ut / NT;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+        if (rt->ent_tok[en] == t) {
+          const float g = rt->ent_gate[en];
+          const float4 x4 = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
+          v = make_float4(g * x4.x, g * x4.y, g * x4.z, g * x4.w);
+        }
+      *reinterpret_cast<float4*>(a_s + ((size_t)u * NT + t) * I + cq * 4) = v;
+    }
+  } else {
+    for (int z = tid; z < rt->n_ent * (I / 4); z += kCT) {
+      const int cq = z % (I / 4), en = z / (I / 4);
+      const float g = rt->ent_gate[en];
+      const float4 x4 = ld_act4(a.ws.a + (size_t)en * I + cq * 4);
+      *reinterpret_cast<float4*>(a_s + (size_t)en * I + cq * 4) = make_float4(g * x4.x, g * x4.y, g * x4.z, g * x4.w);
+    }
+    for (int z = tid; z < U * NT; z += kCT) {
+      const int u = z / NT, t = z - u * NT;
+      int f = -1;
+      for (int en = rt->un_off[u]; en < rt->un_off[u + 1]; ++en)
+        if (rt->ent_tok[en] == t) f = en;
+      ent_of[z] = f;
+    }
   }
   csync();
-  combine_down<NT, EPL>(a, ring, SB_B, SBn, fullB, emptyB, abort_flag, a_s, U, i0, nrows, warp, lane);
+  combine_down<NT, EPL>(a, ring, SB_B, SBn, fullB, emptyB, abort_flag, a_s, ent_of, U, i0, nrows, warp, lane);
 }
 
 // =============================================================================
@@ -1393,14 +1448,14 @@ cudaError_t launch_f(Kern k, int grid, size_t smem, cudaStream_t s, bool pdl, co
 }
 
 size_t up128(size_t x) { return (x + 127) & ~size_t(127); }
-constexpr size_t kRouteBytes = sizeof(SmallRoute) + sizeof(RouteScratch) + 2 * 2 * kCandStride * 4 + 128;
+
 constexpr size_t kRingCap = 200 * 1024;
 
 }  // namespace
 
 bool plan_small(LayerArgs& a, int G, size_t optin) {
   const size_t budget = optin - 1024 - 256;
-  const int NT = 2;
+  const int NT = a.B <= 2 ? 2 : kSmallB;  // tokens the kernels hold at once (planned at two for B <= 2)
   {  // K1: whole rows of W_o, ~32 KB stages
     KTune& t = a.k1;
     const size_t row = (size_t)a.d_o * 2;
@@ -1428,10 +1483,11 @@ bool plan_small(LayerArgs& a, int G, size_t optin) {
     t.rows_max = (int)((umax * a.I + G - 1) / G);  // pairs per CTA
     t4.rows_max = (a.d + G - 1) / G;                // output rows per CTA
     if (t4.rows_max > 4 * kCW) return false;
-    const int eps = experts_per_stage(a.I / 32);
+    const int eps = experts_per_stage(a.I / 32, NT);
     t4.rows_per_stage = eps;
-    const size_t scratch_f = std::max((size_t)t.rows_max * 2 * kCW * NT, (size_t)umax * NT * a.I);
-    const size_t extra = up128(scratch_f * 4) + kRouteBytes + 4 * kMaxStages * 8 + 64;
+    const size_t scratch_f =
+        std::max((size_t)t.rows_max * 2 * kCW * NT, a_s_floats(std::max(a.B, 1), a.k, a.E, a.I, NT));
+    const size_t extra = up128(scratch_f * 4) + route_bytes(NT) + 4 * kMaxStages * 8 + 64;
     const size_t SBd = up128((size_t)eps * t4.rows_max * a.I * 2);
     t.stages = 0;
     for (int ps = 2; ps >= 1 && t.stages < 2; --ps) {
@@ -1466,8 +1522,8 @@ bool plan_fused(LayerArgs& a, int G, size_t optin) {
   o.rows_per_stage = (int)std::max<size_t>(1, std::min<size_t>(32768 / orow, (size_t)o.rows_max));
   const size_t scratch_f =
       layer_scratch_floats(NT, oproj_unit_cap(a.d, o.rows_per_stage, G), o.rows_per_stage, r.rows_max, pa.rows_max, a.d);
-  const size_t a_s_bytes = (size_t)umax * NT * a.I * 4;
-  const size_t extra = up128(scratch_f * 4) + kRouteBytes + 6 * kMaxStages * 8 + 8 + 64;
+  const size_t a_s_bytes = a_s_floats(std::max(a.B, 1), a.k, a.E, a.I, NT) * 4;
+  const size_t extra = up128(scratch_f * 4) + route_bytes(NT) + 6 * kMaxStages * 8 + 8 + 64;
   if (extra >= budget) return false;
   const size_t cap = budget - extra;
   const size_t SO = std::max(up128((size_t)o.rows_per_stage * orow), up128(row));
@@ -1482,7 +1538,7 @@ bool plan_fused(LayerArgs& a, int G, size_t optin) {
     SA = up128((size_t)2 * ps * row);
     pa.stages = (int)std::min<size_t>(kMaxStages, cap / SA);
   }
-  const int eps = experts_per_stage(a.I / 32);
+  const int eps = experts_per_stage(a.I / 32, NT);
   pb.rows_per_stage = eps;
   const size_t SBd = up128((size_t)eps * pb.rows_max * a.I * 2);
   pb.stages = cap > a_s_bytes ? (int)std::min<size_t>(kMaxStages, (cap - a_s_bytes) / SBd) : 0;
@@ -1526,7 +1582,9 @@ bool layer_fused_ok(const LayerArgs& a0, size_t optin) {
 
 bool small_path_ok(const LayerArgs& a0, size_t optin) {
   LayerArgs a = a0;
-  return a.B <= 2 && a.k <= 32 && a.d <= 8192 && a.d_o <= 8192 && plan_small(a, 148, optin);
+  // up to kSmallB tokens with at most 64 (token, expert) entries: the per-CTA routing's tables
+  return a.B <= kSmallB && a.B * a.k <= 64 && a.k <= 32 && a.d <= 8192 && a.d_o <= 8192 &&
+         plan_small(a, 148, optin);
 }
 
 bool oproj_small_ok(const LayerArgs& a, size_t optin) { return small_path_ok(a, optin); }
@@ -1549,6 +1607,7 @@ cudaError_t set_small_attributes(size_t optin) {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100)
   SETS(k_oproj_f<1>);
   SETS(k_oproj_f<2>);
+  SETS(k_oproj_f<kSmallB>);
 #define SETS_D(k, ...) \
   SETS((k<__VA_ARGS__, 2>)); \
   SETS((k<__VA_ARGS__, 3>))
@@ -1560,6 +1619,9 @@ cudaError_t set_small_attributes(size_t optin) {
   SETS_D(k_experts_f, 2, 8);
   SETS_D(k_experts_f, 1, 0);
   SETS_D(k_experts_f, 2, 0);
+  SETS_D(k_experts_f, kSmallB, 4);
+  SETS_D(k_experts_f, kSmallB, 8);
+  SETS_D(k_experts_f, kSmallB, 0);
   SETS(k_router_big);
   SETS_D(k_layer_f, 1, 4);
   SETS_D(k_layer_f, 2, 4);
@@ -1594,6 +1656,11 @@ template <int CPD>
 cudaError_t launch_experts_d(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
   const int epl = a.I / 32;
   const size_t sm = a.k3.smem;
+  if (a.B > 2) {
+    if (epl == 4) return launch_f(k_experts_f<kSmallB, 4, CPD>, grid, sm, s, pdl, a, true);
+    if (epl == 8) return launch_f(k_experts_f<kSmallB, 8, CPD>, grid, sm, s, pdl, a, true);
+    return launch_f(k_experts_f<kSmallB, 0, CPD>, grid, sm, s, pdl, a, true);
+  }
   if (epl == 4)
     return a.B == 1 ? launch_f(k_experts_f<1, 4, CPD>, grid, sm, s, pdl, a, true)
                     : launch_f(k_experts_f<2, 4, CPD>, grid, sm, s, pdl, a, true);
@@ -1621,6 +1688,7 @@ cudaError_t launch_layer_d(const LayerArgs& a, int grid, cudaStream_t s, bool pd
 
 cudaError_t launch_oproj_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   const LayerArgs a = planned(a0, grid, optin);
+  if (a.B > 2) return launch_f(k_oproj_f<kSmallB>, grid, a.k1.smem, s, pdl, a);
   return a.B == 1 ? launch_f(k_oproj_f<1>, grid, a.k1.smem, s, pdl, a) : launch_f(k_oproj_f<2>, grid, a.k1.smem, s, pdl, a);
 }
 

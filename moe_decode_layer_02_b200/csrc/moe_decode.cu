@@ -124,14 +124,14 @@ void release(moe_decode_handle* h) {
 }
 
 bool use_large(const moe_decode_handle* h, int B) {
-  if (B >= 3) return true;                        // separate large-batch kernels above batch two
-  return h->cfg.force_variant == 2;               // small-matrix kernels at batch one or two
+  if (B > 4) return true;           // separate large-batch kernels above batch four
+  return h->cfg.force_variant == 2;  // small-matrix kernels up to batch four where they fit
 }
 
 // Kernel choice of one layer step.
 struct Variant {
-  bool oproj_small;   // whole-row o_proj (batch <= 2)
-  bool experts_small; // small-M gate/up and down with per-CTA routing (batch <= 2)
+  bool oproj_small;   // whole-row o_proj (batch <= 4)
+  bool experts_small; // small-M gate/up and down with per-CTA routing (batch <= 4)
   bool layer2;        // the batch <= 2 layer kernel with per-expert counters (one launch)
   bool fused;         // the three batch <= 2 kernels as one launch with three grid barriers
 };
@@ -141,7 +141,7 @@ Variant variant_of(const moe_decode_handle* h, const LayerArgs& a) {
   v.experts_small = !use_large(h, a.B) && small_path_ok(a, h->smem_optin);
   v.oproj_small = v.experts_small && oproj_small_ok(a, h->smem_optin);
   const bool by_batch = !use_large(h, a.B) && h->cfg.force_variant == 0;
-  v.layer2 = !use_large(h, a.B) && h->cfg.force_variant == 3 && layer2_ok(a, h->smem_optin);
+  v.layer2 = !use_large(h, a.B) && a.B <= 2 && h->cfg.force_variant == 3 && layer2_ok(a, h->smem_optin);
   // Where the counter-based kernel does not fit: one fused launch at batch 1; at batch 2 the
   // three kernels were measured ahead of that fused launch, so they stay.
   v.fused = !v.layer2 && by_batch && v.oproj_small && a.B == 1 && layer_fused_ok(a, h->smem_optin);

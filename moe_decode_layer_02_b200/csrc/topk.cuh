@@ -8,6 +8,7 @@
 // the layer's stated gate function.
 #pragma once
 #include <cstddef>
+#include <type_traits>
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -270,15 +271,18 @@ __device__ void topk_route(const LayerArgs& a, unsigned char* scratch, bool sele
 
 }  // namespace
 
-// Per-CTA routing of a batch of at most 2 tokens (shared memory only).
-struct alignas(16) SmallRoute {
+// Per-CTA routing of a batch of at most R (2 or kSmallB) tokens with at most 64 entries
+// (tokens x top-k), in shared memory only.
+constexpr int kSmallB = 4;
+template <int R>
+struct alignas(16) SmallRouteR {
   int U, n_ent;
   int un_e[64];        // union experts, ascending
   int un_off[65];      // entries of union expert u: [un_off[u], un_off[u + 1])
   int ent_tok[64];     // token of each entry (tokens ascending within an expert)
   float ent_gate[64];  // gate of each entry
-  int idx[2][32];      // per-token selection, descending logit
-  float gate[2][32];
+  int idx[R][32];      // per-token selection, descending logit
+  float gate[R][32];
 };
 
 // Threads of the CTA that runs route_small_cta.
@@ -286,25 +290,43 @@ constexpr int kRouteThreads = 512;
 constexpr int kRouteGroups = kRouteThreads / 8;  // quarter-warp groups
 
 // Scratch of route_small_cta.  Arrays read with 16-byte vector loads are 16-byte aligned.
-struct alignas(16) RouteScratch {
-  alignas(16) float cv[2][kCandMax];         // candidate logits
-  alignas(16) int ci[2][kCandMax];           // candidate experts
-  alignas(16) float gmax[2][kRouteGroups];   // quarter-warp maxima
-  float sel_v[2][32];                        // selection in rank order
-  int sel_i[2][32];
-  unsigned bm[2][32];                        // selected-expert bitmaps (E <= 1024)
-  float T[2];                                // candidate bound per token
-  int cnt[2];                                // candidates per token
+template <int R>
+struct alignas(16) RouteScratchR {
+  alignas(16) float cv[R][kCandMax];         // candidate logits
+  alignas(16) int ci[R][kCandMax];           // candidate experts
+  alignas(16) float gmax[R][kRouteGroups];   // quarter-warp maxima
+  float sel_v[R][32];                        // selection in rank order
+  int sel_i[R][32];
+  unsigned bm[R][32];                        // selected-expert bitmaps (E <= 1024)
+  float T[R];                                // candidate bound per token
+  int cnt[R];                                // candidates per token
 };
-static_assert(offsetof(RouteScratch, cv) % 16 == 0 && offsetof(RouteScratch, ci) % 16 == 0 &&
-                  offsetof(RouteScratch, gmax) % 16 == 0,
+// The routing scratch of a kernel holding NT tokens: sized for two tokens up to two (so the
+// one- and two-token kernels share a layout), for kSmallB above.
+template <int NT>
+struct RouteOf {
+  static constexpr int R = NT <= 2 ? 2 : kSmallB;
+  using Route = SmallRouteR<R>;
+  using Scratch = RouteScratchR<R>;
+  static constexpr int kFbFloats = R * 2 * kCandStride;  // the mass-tie fallback's candidates
+};
+// Bytes of a routing scratch for r (2 or kSmallB) tokens: tables, scratch, fallback, alignment.
+__host__ __device__ constexpr size_t route_bytes(int r) {
+  return r <= 2 ? sizeof(SmallRouteR<2>) + sizeof(RouteScratchR<2>) + (size_t)2 * 2 * kCandStride * 4 + 128
+                : sizeof(SmallRouteR<kSmallB>) + sizeof(RouteScratchR<kSmallB>) +
+                      (size_t)kSmallB * 2 * kCandStride * 4 + 128;
+}
+static_assert(offsetof(RouteScratchR<2>, cv) % 16 == 0 && offsetof(RouteScratchR<2>, ci) % 16 == 0 &&
+                  offsetof(RouteScratchR<2>, gmax) % 16 == 0 && offsetof(RouteScratchR<kSmallB>, ci) % 16 == 0 &&
+                  offsetof(RouteScratchR<kSmallB>, gmax) % 16 == 0,
               "vector-loaded routing arrays must be 16-byte aligned");
-static_assert(sizeof(SmallRoute) % 16 == 0, "RouteScratch follows SmallRoute");
+static_assert(sizeof(SmallRouteR<2>) % 16 == 0 && sizeof(SmallRouteR<kSmallB>) % 16 == 0,
+              "the routing scratch follows the tables");
 
 namespace {
 
-// CTA-wide routing of a batch of at most 2 tokens (all kRouteThreads threads call it;
-// 5 barriers).
+// CTA-wide routing of a batch of B <= NT <= kSmallB tokens, B * K <= 64 (all kRouteThreads
+// threads call it; 5 barriers).
 //  1. each thread loads its strided share of the logits (E <= 2 * kRouteThreads);
 //     quarter-warp maxima go to shared memory;
 //  2. T = the k-th largest of a token's group maxima (each group maximum ranked against
@@ -314,16 +336,20 @@ namespace {
 //     else through shared memory; with more than kCandMax, e.g. mass ties, it selects by
 //     repeated arg-max instead), computes the gates and marks the selection in a bitmap;
 //  5. warp 0 scans the bitmaps (word = lane) and places every entry: its union index and
-//     its position in the (expert, token)-sorted entry list are a scan value plus a popcount.
+//     its position in the (expert, token)-sorted entry list are a scan value plus a popcount
+//     (per-token and union counts packed 8 bits each into one scanned word).
 // Inlined: a separate (non-inlined) function measured twice as slow in the fused kernel.
+template <int NT>
 __device__ __forceinline__ void route_small_cta(const float* logits, int B, int E, int K, int* user_idx,
-                                             float* user_gate, uint32_t* err, SmallRoute* rt, RouteScratch* sc,
+                                             float* user_gate, uint32_t* err, typename RouteOf<NT>::Route* rt,
+                                             typename RouteOf<NT>::Scratch* sc,
                                              float* fallback_cand, bool write_user) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int kPer = 2;  // logits per thread per token
-  float v[2][kPer];
+  static_assert(NT >= 1 && NT <= kSmallB, "at most kSmallB tokens");
+  float v[NT][kPer];
 #pragma unroll
-  for (int t = 0; t < 2; ++t)
+  for (int t = 0; t < NT; ++t)
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
       const int e = tid + i * kRouteThreads;
@@ -334,10 +360,10 @@ __device__ __forceinline__ void route_small_cta(const float* logits, int B, int 
       }
       v[t][i] = x;
     }
-  if (tid < 2) sc->cnt[tid] = 0;
-  if (tid < 64) (&sc->bm[0][0])[tid] = 0u;
+  if (tid < NT) sc->cnt[tid] = 0;
+  if (tid < NT * 32) (&sc->bm[0][0])[tid] = 0u;
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
+  for (int t = 0; t < NT; ++t) {
     float m = fmaxf(v[t][0], v[t][1]);
 #pragma unroll
     for (int o = 4; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -363,7 +389,7 @@ __device__ __forceinline__ void route_small_cta(const float* logits, int B, int 
   // (3) candidates
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
+  for (int t = 0; t < NT; ++t) {
     if (t >= B) break;
     const float T = sc->T[t];
 #pragma unroll
@@ -443,15 +469,24 @@ __device__ __forceinline__ void route_small_cta(const float* logits, int B, int 
   __syncthreads();
   // (5) entries sorted by (expert, token); union experts ascending (warp 0)
   if (warp == 0) {
-    const unsigned b0 = sc->bm[0][lane], b1 = sc->bm[1][lane];
-    const int own = __popc(b0) | (__popc(b1) << 8) | (__popc(b0 | b1) << 16);  // totals <= 64
-    int inc = own;
+    using Pack = typename std::conditional<(NT + 1) * 8 <= 32, unsigned, unsigned long long>::type;
+    unsigned bw[NT];
+    unsigned un = 0;
+    Pack own = 0;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      bw[t] = sc->bm[t][lane];
+      un |= bw[t];
+      own |= (Pack)__popc(bw[t]) << (8 * t);
+    }
+    own |= (Pack)__popc(un) << (8 * NT);  // every field's total is <= 64
+    Pack inc = own;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      const Pack y = __shfl_up_sync(0xffffffffu, inc, o);
       if (lane >= o) inc += y;
     }
-    const int base = inc - own;
+    const Pack base = inc - own;
     const int n = B * K;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -459,23 +494,32 @@ __device__ __forceinline__ void route_small_cta(const float* logits, int B, int 
       const int t = (p < n) ? p / K : 0, j = (p < n) ? p - t * K : 0;
       const int e = rt->idx[t][j], w = e >> 5;
       const unsigned below = (1u << (e & 31)) - 1u;
-      const int bs = __shfl_sync(0xffffffffu, base, w);
-      const unsigned w0 = __shfl_sync(0xffffffffu, b0, w), w1 = __shfl_sync(0xffffffffu, b1, w);
+      const Pack bs = __shfl_sync(0xffffffffu, base, w);
+      int pe = 0;
+      unsigned wu = 0;
+      bool earlier = false;  // a lower token selected e too
+#pragma unroll
+      for (int tt = 0; tt < NT; ++tt) {
+        const unsigned wt = __shfl_sync(0xffffffffu, bw[tt], w);
+        wu |= wt;
+        pe += (int)((bs >> (8 * tt)) & 0xFFu) + __popc(wt & below);
+        if (tt < t && ((wt >> (e & 31)) & 1u)) {
+          ++pe;
+          earlier = true;
+        }
+      }
+      const int pu = (int)((bs >> (8 * NT)) & 0xFFu) + __popc(wu & below);
       if (p < n) {
-        const int p0 = (bs & 0xFF) + __popc(w0 & below), p1 = ((bs >> 8) & 0xFF) + __popc(w1 & below);
-        const int pu = ((bs >> 16) & 0xFF) + __popc((w0 | w1) & below);
-        const bool t0_has = (w0 >> (e & 31)) & 1u;
-        const int pe = p0 + p1 + ((t == 1 && t0_has) ? 1 : 0);
         rt->ent_tok[pe] = t;
         rt->ent_gate[pe] = rt->gate[t][j];
-        if (t == 0 || !t0_has) {  // first entry of expert e
+        if (!earlier) {  // first entry of expert e
           rt->un_e[pu] = e;
           rt->un_off[pu] = pe;
         }
       }
     }
     if (lane == 31) {
-      const int u = (inc >> 16) & 0xFF;
+      const int u = (int)((inc >> (8 * NT)) & 0xFFu);
       rt->U = u;
       rt->n_ent = n;
       rt->un_off[u] = n;

@@ -100,7 +100,7 @@ def test_step_argument_checks():
         assert md.moe_decode_sync_status(h) == 0
         assert md.moe_decode_kernels_per_step(h, 1) == 1  # batch 1: one layer kernel
         assert md.moe_decode_kernels_per_step(h, 2) == 3  # batch 2: o_proj, router, small-M experts
-        assert md.moe_decode_kernels_per_step(h, 4) == 4  # o_proj, router, gate/up, down
+        assert md.moe_decode_kernels_per_step(h, 4) == 3  # up to batch 4 the same three kernels
     finally:
         assert md.moe_decode_destroy(h) == 0
     assert md.moe_decode_destroy(h) == md.MOE_ERR_INVALID_ARG  # destroyed twice: rejected

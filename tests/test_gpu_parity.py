@@ -164,7 +164,7 @@ def tp16_tied():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("B", [1, 2, 16])
+@pytest.mark.parametrize("B", [1, 2, 4, 16])
 def test_ties_all_logits_zero(tp16_tied, B):
     seed, st, ref = tp16_tied
     D = synth.TP16
@@ -180,7 +180,7 @@ def test_ties_all_logits_zero(tp16_tied, B):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("B", [1, 2, 16])
+@pytest.mark.parametrize("B", [1, 2, 4, 16])
 def test_ties_duplicated_router_rows(tp16_tied, B):
     from oracle.layer import top_gap_distinct
     seed, st, ref = tp16_tied
@@ -277,6 +277,40 @@ def test_tp16_speculative_max_batch_4(tp16):
         check_case(st, build_case(seed, synth.TP16, 4, attn0=attn0, resid0=resid0, refs=[ref]))
     finally:
         st.close()
+
+
+# --- the small-batch kernels up to four tokens: they take a batch while its (token, expert)
+#     entries fit the per-CTA routing's 64, else the large-batch kernels run ------------------
+def kernels_run(st, B):
+    """Names of the kernels one eager step of this batch launches."""
+    import torch
+    D = st.dims
+    attn = torch.zeros((1, B, D.d_o), dtype=torch.bfloat16, device="cuda")
+    resid = torch.zeros((B, D.d), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((B, D.d), dtype=torch.bfloat16, device="cuda")
+    return [n for n, _ in st.md.moe_decode_profile_step(st.h, B, attn, resid, out)]
+
+
+@pytest.mark.parametrize("B,k,small", [(3, 20, True), (4, 16, True), (4, 20, False)])
+def test_small_path_entry_limit(B, k, small):
+    dims = synth.Dims(256, 256, 64, k, 128)
+    seed = synth.config_seed(12) + 10 * B + k
+    st = H.GpuStack(seed, dims, max_batch=4)
+    try:
+        names = kernels_run(st, B)
+        assert ("experts_small_m" in names) == small, names
+        check_case(st, build_case(seed, dims, B))
+    finally:
+        st.close()
+
+
+@pytest.mark.slow
+def test_tp16_b4_independent(tp16):
+    """Four independent tokens: the largest union (64 experts) the four-token kernels hold."""
+    seed, st, ref = tp16
+    case = build_case(seed + 4, synth.TP16, 4, refs=[ref])
+    out, idx, gate, _ = check_case(st, case)  # every token
+    assert "experts_small_m" in kernels_run(st, 4)
 
 
 # --- full-size layer (1/8 shard, I=256), batch 16 and 64 -------------------------------------
