@@ -60,6 +60,7 @@ WORKLOADS = {
     # profiling case: tp16 o_proj/router/expert shapes with 64 experts (~0.6 GB on the device)
     "tp16e64_b1": ("TP16E64", 1, 1, "indep"),
     "tp16e64_b2": ("TP16E64", 2, 1, "indep"),
+    "tp16e64_spec4": ("TP16E64", 4, 1, "spec"),
     "tp8e64_b64": ("TP8E64", 64, 1, "indep"),
     "tp8e224k4_b16": ("TP8E224K4", 16, 1, "indep"),
     # profiling case for the next-layer prefetch: two such layers (~1.2 GB on the device)
@@ -561,7 +562,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="tp16_b1", choices=sorted(WORKLOADS))
-    ap.add_argument("--prefetch", type=int, default=1)
+    ap.add_argument("--prefetch", type=int, default=0,
+                    help="stacks: 1 enables the next-layer L2 prefetch (measured slower on the current "
+                         "kernels, so off by default)")
     ap.add_argument("--force-variant", type=int, default=0, choices=[0, 1, 2, 3],
                     help="kernel choice: 0 by batch size, 1 unfused batch <= 2 kernels, 2 large-batch "
                          "kernels at every batch, 3 counter-ordered batch <= 2 layer kernel "
