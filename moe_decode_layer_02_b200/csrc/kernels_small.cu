@@ -68,7 +68,10 @@ __host__ __device__ constexpr size_t a_s_floats(int B, int K, int E, int I, int 
 // K1: o_proj + residual + per-CTA sums of h^2 (batch <= 2)
 //   CTA c owns rows [r0, r1) of W_o (contiguous); a stage is RS whole rows (one copy).
 // =============================================================================
-template <int NT>
+// CPO 2: d_o <= 7680, the K slice split evenly over the 15 warps in at most two 32-lane chunk
+// rounds; CPO 3: two full rounds per warp (64 chunks) and the rest as a third round in the
+// first warps only (rows_dot_bf_2x).
+template <int NT, int CPO>
 __global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int G = gridDim.x, c = blockIdx.x;
@@ -116,14 +119,20 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
 
   pdl_wait();  // attn_out and residual may come from the previous kernel
   constexpr int kRI = 2;  // rows per interleaved pass (a stage is two rows at d_o = 8192)
-  const int qbase = (d_o / 8) * warp / kCW, qpw = (d_o / 8) * (warp + 1) / kCW - qbase;
-  uint4 xa[NT][kCPLf];  // attn_out stays packed bf16 (mixed-precision FMAs)
+  const int nch = d_o / 8;
+  const int qbase = CPO == 2 ? nch * warp / kCW : 64 * warp;
+  const int qpw = CPO == 2 ? nch * (warp + 1) / kCW - qbase : 64;
+  const int qx = kCW * 64 + 32 * warp;  // CPO 3: this warp's third round, if any
+  const bool has_x = CPO == 3 && qx < nch;
+  uint4 xa[NT][CPO];  // attn_out stays packed bf16 (mixed-precision FMAs)
 #pragma unroll
   for (int t = 0; t < NT; ++t)
 #pragma unroll
-    for (int j = 0; j < kCPLf; ++j) {
+    for (int j = 0; j < CPO; ++j) {
       uint4 u = make_uint4(0, 0, 0, 0);
-      if (t < B && cvalid(qpw, j, lane)) u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)(qbase + j * 32 + lane) * 8);
+      const int q = (j < 2) ? qbase + j * 32 + lane : qx + lane;
+      const bool ok = (j < 2) ? cvalid(qpw, j, lane) : (has_x && q < nch);
+      if (t < B && ok) u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)q * 8);
       xa[t][j] = u;
     }
   int it = 0;
@@ -136,7 +145,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_oproj_f(const LayerArgs a) {
 #pragma unroll
       for (int k = 0; k < kRI; ++k) rp[k] = st + (size_t)min(j0 + k, n - 1) * d_o;
       float v[kRI * NT];
-      rows_dot_bf<NT, kRI>(rp, n - j0, xa, qbase, qpw, lane, v);
+      if constexpr (CPO == 2) rows_dot_bf<NT, kRI>(rp, n - j0, xa, qbase, qpw, lane, v);
+      else rows_dot_bf_2x<NT, kRI>(rp, n - j0, xa, qbase, qx, nch, has_x, lane, v);
       const float tot = warp_reduce_multi<kRI * NT>(v, lane);
       const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
       if (multi_writer<kRI * NT>(lane) && j < n) part[((r - r0 + j) * kCW + warp) * NT + t] = tot;
@@ -1605,9 +1615,12 @@ cudaError_t set_small_attributes(size_t optin) {
 #define SETS(k)                                                                                              \
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, v); \
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100)
-  SETS(k_oproj_f<1>);
-  SETS(k_oproj_f<2>);
-  SETS(k_oproj_f<kSmallB>);
+  SETS((k_oproj_f<1, 2>));
+  SETS((k_oproj_f<2, 2>));
+  SETS((k_oproj_f<kSmallB, 2>));
+  SETS((k_oproj_f<1, 3>));
+  SETS((k_oproj_f<2, 3>));
+  SETS((k_oproj_f<kSmallB, 3>));
 #define SETS_D(k, ...) \
   SETS((k<__VA_ARGS__, 2>)); \
   SETS((k<__VA_ARGS__, 3>))
@@ -1688,8 +1701,14 @@ cudaError_t launch_layer_d(const LayerArgs& a, int grid, cudaStream_t s, bool pd
 
 cudaError_t launch_oproj_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   const LayerArgs a = planned(a0, grid, optin);
-  if (a.B > 2) return launch_f(k_oproj_f<kSmallB>, grid, a.k1.smem, s, pdl, a);
-  return a.B == 1 ? launch_f(k_oproj_f<1>, grid, a.k1.smem, s, pdl, a) : launch_f(k_oproj_f<2>, grid, a.k1.smem, s, pdl, a);
+  if (two_chunks(a.d_o)) {
+    if (a.B > 2) return launch_f(k_oproj_f<kSmallB, 2>, grid, a.k1.smem, s, pdl, a);
+    return a.B == 1 ? launch_f(k_oproj_f<1, 2>, grid, a.k1.smem, s, pdl, a)
+                    : launch_f(k_oproj_f<2, 2>, grid, a.k1.smem, s, pdl, a);
+  }
+  if (a.B > 2) return launch_f(k_oproj_f<kSmallB, 3>, grid, a.k1.smem, s, pdl, a);
+  return a.B == 1 ? launch_f(k_oproj_f<1, 3>, grid, a.k1.smem, s, pdl, a)
+                  : launch_f(k_oproj_f<2, 3>, grid, a.k1.smem, s, pdl, a);
 }
 
 cudaError_t launch_router_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {

@@ -180,6 +180,63 @@ __device__ __forceinline__ void rows_dot_bf(const uint16_t* const (&rp)[R], int 
     }
 }
 
+// rows_dot_bf for a K slice laid out as two full 32-lane chunk rounds per warp at qbase (64
+// chunks) plus, in the warps with has_x (warp-uniform), one more round at qx, valid below nch:
+// for K above 15 warps x 64 chunks (d_o up to 8192), where an even split over the 15 warps
+// would give every warp a third round that is nearly empty (4 of 32 lanes at d_o = 8192), and
+// its FMAs on zeros.  x[t][2] holds the extra round's chunk.  Same accumulators as rows_dot_bf;
+// the extra round is added last.
+template <int NT, int R>
+__device__ __forceinline__ void rows_dot_bf_2x(const uint16_t* const (&rp)[R], int nr, const uint4 (&x)[NT][3],
+                                               int qbase, int qx, int nch, bool has_x, int lane,
+                                               float (&out)[R * NT]) {
+  constexpr int kA = (R * NT >= 4) ? 1 : 4 / (R * NT);
+  uint4 w[R][3];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const uint32_t base = (uint32_t)__cvta_generic_to_shared(rp[r]);
+    w[r][0] = (r < nr) ? lds128(base + (uint32_t)(qbase + lane) * 16u) : make_uint4(0, 0, 0, 0);
+    w[r][1] = (r < nr) ? lds128(base + (uint32_t)(qbase + 32 + lane) * 16u) : make_uint4(0, 0, 0, 0);
+    w[r][2] = (has_x && r < nr && qx + lane < nch) ? lds128(base + (uint32_t)(qx + lane) * 16u)
+                                                   : make_uint4(0, 0, 0, 0);
+  }
+  float2 acc[R][NT][kA];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int e = 0; e < kA; ++e) acc[r][t][e] = make_float2(0.f, 0.f);
+  auto round = [&](int j) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint32_t wv[4] = {w[r][j].x, w[r][j].y, w[r][j].z, w[r][j].w};
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        const uint32_t xv[4] = {x[t][j].x, x[t][j].y, x[t][j].z, x[t][j].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2& a = acc[r][t][e % kA];
+          a.x = fma_bf16<false>(wv[e], xv[e], a.x);
+          a.y = fma_bf16<true>(wv[e], xv[e], a.y);
+        }
+      }
+    }
+  };
+  round(0);
+  round(1);
+  if (has_x) round(2);
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float v = 0.f;
+#pragma unroll
+      for (int e = 0; e < kA; ++e) v += acc[r][t][e].x + acc[r][t][e].y;
+      out[r * NT + t] = v;
+    }
+}
+
 // Warp sums of V per-lane values (V a power of two <= 32) with V - 1 + 5 - log2(V) shuffles
 // instead of 5 V: each halving step sends one value of every pair across the current lane
 // bit and keeps the other.  Every lane returns the total of value multi_index<V>(lane).
