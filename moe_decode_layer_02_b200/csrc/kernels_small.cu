@@ -1604,7 +1604,8 @@ bool router_ok(const LayerArgs& a0, size_t optin) {
   const int G = 148;
   KTune& t = a.k2;
   t.rows_max = (a.E + G - 1) / G;
-  t.smem = up128((size_t)t.rows_max * a.d * 2) + up128((size_t)t.rows_max * kCW * 2 * 4 + 64 * 4) + 8 +
+  const int nt = (a.d <= 8 * 32 * 2 * kCW && a.B > 2) ? kSmallB : 2;  // as launch_router_s
+  t.smem = up128((size_t)t.rows_max * a.d * 2) + up128((size_t)t.rows_max * kCW * nt * 4 + 64 * 4) + 8 +
            32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
   return a.d <= 8192 && t.smem <= optin - 1024 - 256;
 }
@@ -1626,6 +1627,7 @@ cudaError_t set_small_attributes(size_t optin) {
   SETS((k<__VA_ARGS__, 3>))
   SETS_D(k_router_f, 1);
   SETS_D(k_router_f, 2);
+  SETS((k_router_f<kSmallB, 2>));
   SETS_D(k_experts_f, 1, 4);
   SETS_D(k_experts_f, 2, 4);
   SETS_D(k_experts_f, 1, 8);
@@ -1661,6 +1663,8 @@ bool two_chunks(int d) { return d <= 8 * 32 * 2 * kCW; }
 
 template <int CPD>
 cudaError_t launch_router_d(const LayerArgs& a, int grid, cudaStream_t s, bool pdl) {
+  // above two tokens, four at a time where two chunks per lane leave the registers for them
+  if (CPD == 2 && a.B > 2) return launch_f(k_router_f<kSmallB, 2>, grid, a.k2.smem, s, pdl, a);
   return a.B == 1 ? launch_f(k_router_f<1, CPD>, grid, a.k2.smem, s, pdl, a)
                   : launch_f(k_router_f<2, CPD>, grid, a.k2.smem, s, pdl, a);
 }
@@ -1714,7 +1718,8 @@ cudaError_t launch_oproj_s(const LayerArgs& a0, int grid, cudaStream_t s, bool p
 cudaError_t launch_router_s(const LayerArgs& a0, int grid, cudaStream_t s, bool pdl, size_t optin) {
   LayerArgs a = a0;
   a.k2.rows_max = (a.E + grid - 1) / grid;
-  a.k2.smem = up128((size_t)a.k2.rows_max * a.d * 2) + up128((size_t)a.k2.rows_max * kCW * 2 * 4 + 64 * 4) +
+  const int nt = (two_chunks(a.d) && a.B > 2) ? kSmallB : 2;  // tokens per pass of the launched kernel
+  a.k2.smem = up128((size_t)a.k2.rows_max * a.d * 2) + up128((size_t)a.k2.rows_max * kCW * nt * 4 + 64 * 4) +
               8 + 32 * 4 + (a.route_tables ? kTopkScratch : 0) + 64;
   (void)optin;
   return two_chunks(a.d) ? launch_router_d<2>(a, grid, s, pdl) : launch_router_d<3>(a, grid, s, pdl);
