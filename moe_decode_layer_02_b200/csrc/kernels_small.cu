@@ -1079,14 +1079,22 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
     int nslot = 0;
     {
       constexpr int kRI = 2;
+      // K split of d_o as in k_oproj_f: evenly in at most two chunk rounds up to d_o = 7680,
+      // else two full rounds per warp and a third in the first warps only
+      const int nch = d_o / 8;
+      const bool split2x = nch > 64 * kCW;
+      const int qb = split2x ? 64 * warp : qbase_o, qp = split2x ? 64 : qpw_o;
+      const int qx = 64 * kCW + 32 * warp;
+      const bool has_x = split2x && qx < nch;
       uint4 xa[NT][kCPLf];  // attn_out stays packed bf16 (mixed-precision FMAs)
 #pragma unroll
       for (int t = 0; t < NT; ++t)
 #pragma unroll
         for (int j = 0; j < kCPLf; ++j) {
           uint4 u = make_uint4(0, 0, 0, 0);
-          if (t < B && cvalid(qpw_o, j, lane))
-            u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)(qbase_o + j * 32 + lane) * 8);
+          const int q = (j < 2 || !split2x) ? qb + j * 32 + lane : qx + lane;
+          const bool ok = (j < 2 || !split2x) ? cvalid(qp, j, lane) : (has_x && q < nch);
+          if (t < B && ok) u = ld_act_u4(a.attn + (size_t)t * d_o + (size_t)q * 8);
           xa[t][j] = u;
         }
       while (true) {
@@ -1107,7 +1115,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_layer_f(const LayerArgs a) {
 #pragma unroll
           for (int k = 0; k < kRI; ++k) rp[k] = st + (size_t)min(j0 + k, n - 1) * d_o;
           float v[kRI * NT];
-          rows_dot_bf<NT, kRI>(rp, n - j0, xa, qbase_o, qpw_o, lane, v);
+          if (split2x) rows_dot_bf_2x<NT, kRI>(rp, n - j0, xa, qb, qx, nch, has_x, lane, v);
+          else rows_dot_bf<NT, kRI>(rp, n - j0, xa, qbase_o, qpw_o, lane, v);
           const float tot = warp_reduce_multi<kRI * NT>(v, lane);
           const int vi = multi_index<kRI * NT>(lane), j = j0 + vi / NT, t = vi % NT;
           if (multi_writer<kRI * NT>(lane) && j < n) opart[(((size_t)nslot * RS + j) * kCW + warp) * NT + t] = tot;
