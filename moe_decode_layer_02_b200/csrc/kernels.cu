@@ -1,6 +1,6 @@
 // sm_100a kernels of one MoE decode-layer step.
 //
-// The fallback large-batch o_proj, used above batch 2 where the TMA tensor maps of
+// The fallback large-batch o_proj, used on the large-batch path where the TMA tensor maps of
 // k_oproj_tc (kernels_tc.cu) cannot be encoded (the small-batch kernels and the router are
 // in kernels_small.cu, the large-batch expert kernels in kernels_large.cu):
 //   K1 k_oproj           h = residual + W_o . attn_out on the tensor cores (weights as the

@@ -42,7 +42,7 @@ struct Workspace {
   // (zero between launches), and the activations [kMaxUnion][B][I]
   unsigned* ecnt;      // [kMaxUnion]
   float* a_u;          // [kMaxUnion][2][I]
-  float* rpart;        // split-K routers' per-CTA partial logits: [G][E][8 ceil(B / 8)] above batch 2,
+  float* rpart;        // split-K routers' per-CTA partial logits: [G][E][8 ceil(B / 8)] on the large-batch path,
                        // [G][E][maxB] in the counter-ordered kernel (8 ceil(maxB / 8) per CTA and expert allocated)
 };
 
@@ -90,7 +90,7 @@ cudaError_t set_small_attributes(size_t smem_optin);
 cudaError_t launch_oproj_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t launch_router_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 cudaError_t launch_experts_s(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
-// The router above batch 2 with h staged by TMA (plus the routing tables).
+// A router of the large-batch path with h staged by TMA (plus the routing tables).
 bool plan_router_big(LayerArgs& a, int grid, size_t smem_optin);
 bool router_big_ok(const LayerArgs& a, size_t smem_optin);
 cudaError_t launch_router_big(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
@@ -110,18 +110,18 @@ bool layer2_ok(const LayerArgs& a, size_t smem_optin);
 cudaError_t set_layer2_attributes(size_t smem_optin);
 cudaError_t launch_layer2(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 
-// The router above batch 2 with K split over the CTAs, partial logits on the tensor cores,
+// The router of the large-batch path with K split over the CTAs, partial logits on the tensor cores,
 // and the routing tables (kernels_router.cu).
 bool router_ks_ok(const LayerArgs& a, int grid, size_t smem_optin);
 cudaError_t set_router_ks_attributes(size_t smem_optin);
 cudaError_t launch_router_ks(const LayerArgs& a, int grid, cudaStream_t s, bool pdl);
 
-// o_proj above batch 2 on the tensor cores with 2-D TMA tiles (kernels_tc.cu).
+// o_proj of the large-batch path on the tensor cores with 2-D TMA tiles (kernels_tc.cu).
 bool oproj_tc_ok(const LayerArgs& a, int grid, size_t smem_optin);
 cudaError_t set_tc_attributes(size_t smem_optin);
 cudaError_t launch_oproj_tc(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);
 
-// Expert kernels above batch 2 (kernels_large.cu): whole rows, tokens grouped per expert.
+// Expert kernels of the large-batch path (kernels_large.cu): whole rows, tokens grouped per expert.
 bool plan_large(LayerArgs& a, int grid, size_t smem_optin);
 cudaError_t set_large_attributes(size_t smem_optin);
 cudaError_t launch_gateup_rows(const LayerArgs& a, int grid, cudaStream_t s, bool pdl, size_t smem_optin);

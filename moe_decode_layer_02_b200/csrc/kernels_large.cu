@@ -1,6 +1,7 @@
-// Expert kernels above batch 2: whole weight rows streamed by TMA, tokens grouped per expert.
+// Expert kernels of the large-batch path (above batch 4, or batch x top-k > 64): whole weight
+// rows streamed by TMA, tokens grouped per expert.
 //
-// At batch >= 3 the union of selected experts holds 10^4..10^5 independent weight rows
+// At those batches the union of selected experts holds 10^4..10^5 independent weight rows
 // (224 experts x 512 gate/up rows at batch 16 with I = 256), far more than the 148 SMs
 // need, so the rows are not split along K: every row is one contiguous bulk copy and every
 // dot product is finished inside one CTA, with no partial sums in global memory.  Each
@@ -74,7 +75,7 @@ __device__ __forceinline__ void load_tables(const LayerArgs& a, int U, int n_ent
 }
 
 // =============================================================================
-// gate/up + SiLU*mul (batch >= 3)
+// gate/up + SiLU*mul (large-batch path)
 //   The CTA's pairs are taken in chunks of up to PC consecutive pairs of one expert; a chunk
 //   is two stages, its PC gate rows and then its PC up rows, each one contiguous bulk copy
 //   (fewer, larger copies stream faster).  The partial sums of a chunk are reduced once its
@@ -266,7 +267,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
 }
 
 // =============================================================================
-// down + gate-weighted combine (batch >= 3)
+// down + gate-weighted combine (large-batch path)
 //   A stage holds EPS experts' blocks of this CTA's rows plus the activations a of their
 //   entries (one more bulk copy: the entries of consecutive experts are contiguous), up to
 //   kAEnt entries; entries past that are read from L2.

@@ -1,4 +1,4 @@
-// The router above batch 2 with K split over the CTAs (one cooperative launch per layer).
+// The router of the large-batch path with K split over the CTAs (one cooperative launch per layer).
 //
 // logits[t][e] = sum_i W_r[e][i] x[t][i] with x = h * rstd * gamma, so
 // logits[t][e] = rstd[t] * sum_i W_r[e][i] (h[t][i] gamma[i]).  CTA c owns the same d-rows

@@ -16,12 +16,13 @@
 //
 //   k_layer_f    batch 1: the whole layer step as one cooperative launch (the three kernels
 //                below as phases, with grid barriers where the kernel boundaries were)
-//   k_oproj_f    h = residual + W_o . attn_out, per-CTA sums of h^2                (batch 2)
-//   k_router_f   rstd, x = h * rstd * gamma, logits = W_r . x   (batch 2; above batch 2
-//                where k_router_big does not fit, its last CTA also building the global
-//                routing tables)
-//   k_router_big the router above batch 2, h staged by TMA, plus the routing tables
-//   k_experts_f  the expert kernel (batch 2): routing once per CTA; gate/up + SiLU*mul
+//   k_oproj_f    h = residual + W_o . attn_out, per-CTA sums of h^2         (batch 2 to 4)
+//   k_router_f   rstd, x = h * rstd * gamma, logits = W_r . x   (batch 2 to 4; on the
+//                large-batch path where k_router_big does not fit, its last CTA also
+//                building the global routing tables)
+//   k_router_big a router of the large-batch path, h staged by TMA, plus the routing tables
+//   k_experts_f  the expert kernel (batch 2 to 4, batch x top-k <= 64): routing once per
+//                CTA; gate/up + SiLU*mul
 //                for each (selected expert, row pair), each pair streamed once; a grid
 //                barrier; then out = bf16(h + sum_j gate_j * W_down[e_j] . a_j), with W_down
 //                streaming into the freed ring while the barrier is open
@@ -65,7 +66,7 @@ __host__ __device__ constexpr size_t a_s_floats(int B, int K, int E, int I, int 
 }  // namespace
 
 // =============================================================================
-// K1: o_proj + residual + per-CTA sums of h^2 (batch <= 2)
+// K1: o_proj + residual + per-CTA sums of h^2 (batch <= 4)
 //   CTA c owns rows [r0, r1) of W_o (contiguous); a stage is RS whole rows (one copy).
 // =============================================================================
 // CPO 2: d_o <= 7680, the K slice split evenly over the 15 warps in at most two 32-lane chunk
@@ -339,7 +340,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_f(const LayerArgs a) {
 }
 
 // =============================================================================
-// Router for batch >= 3: the same arithmetic as k_router_f, with h staged by TMA.
+// Router of the large-batch path: the same arithmetic as k_router_f, with h staged by TMA.
 //   The CTA's W_r slice is one bulk copy issued before the dependency wait (as in
 //   k_router_f).  After it, the producer streams h two tokens at a time (one bulk copy of
 //   2 x d fp32) into a ring, so the consumers never wait on an L2 round trip per token pair:
@@ -547,7 +548,7 @@ __device__ void grid_barrier(unsigned* count, unsigned target, volatile int* abo
 
 }  // namespace
 
-// Phase B of the batch <= 2 expert kernels (consumer warps): out = bf16(h + sum over the
+// Phase B of the batch <= 4 expert kernels (consumer warps): out = bf16(h + sum over the
 // union experts of W_down[e] rows [i0, i0 + nrows) . a_s[e]), the W_down blocks arriving in
 // the B ring.  A stage holds EPS experts' blocks of this CTA's rows; every load of a stage is
 // issued before its FMAs (software-pipelining one expert ahead instead measured slower: fewer
@@ -666,7 +667,7 @@ __device__ __forceinline__ void combine_down(const LayerArgs& a, const unsigned 
 }
 
 // =============================================================================
-// K3 (batch <= 2): the expert kernel.  Routing once per CTA, then
+// K3 (batch <= 4): the expert kernel.  Routing once per CTA, then
 //   phase A  gate/up + SiLU*mul: pairs (union expert u, row p) in flattened order, CTA c takes
 //            [q0, q1); a stage is up to PS consecutive pairs of one expert (its gate rows and
 //            its up rows, two copies).  a goes to global memory.
@@ -1572,7 +1573,7 @@ bool plan_fused(LayerArgs& a, int G, size_t optin) {
   return o.smem <= budget;
 }
 
-// The TMA-staged router above batch 2: W_r slice, h ring (>= 2 stages of two tokens; also
+// The TMA-staged router of the large-batch path: W_r slice, h ring (>= 2 stages of two tokens; also
 // the routing-table builder's scratch), two partial buffers, rstd, barriers.
 bool plan_router_big(LayerArgs& a, int G, size_t optin) {
   const size_t budget = optin - 1024 - 256;

@@ -1,4 +1,4 @@
-// o_proj above batch 2 on the tensor cores with TMA tensor tiles.
+// o_proj of the large-batch path on the tensor cores with TMA tensor tiles.
 //
 // At batch 16-64, h = residual + attn_out . W_o^T is a skinny GEMM ([B x d_o] x [d_o x d])
 // that is still bound by the 117 MB of W_o.  CTA c owns output rows [r0, r1) (49 at most);

@@ -4,8 +4,8 @@
 // A step of n_layers layers is captured once per (batch, buffer addresses) into one
 // CUDA graph.  At batch 1 a layer is one cooperative kernel (o_proj + residual + RMS
 // statistics, router, per-CTA routing, gate/up, down + combine, with grid barriers
-// between the phases); at batch 2 it is o_proj -> router -> the small-M expert kernel
-// (per-CTA routing, gate/up, down + combine); above batch 2 it is o_proj -> router +
+// between the phases); at batch 2 to 4 (batch x top-k <= 64) it is o_proj -> router -> the
+// small-M expert kernel (per-CTA routing, gate/up, down + combine); above it is o_proj -> router +
 // routing tables -> gate/up -> down + combine.  Kernels are chained with programmatic dependent launch so
 // each one's producer fetches its static weights while the previous kernel drains.  With
 // prefetch on, layer l also prefetches into L2 what layer l+1 reads first (its router
