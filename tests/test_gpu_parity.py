@@ -205,11 +205,15 @@ def test_degenerate_k_equals_e_and_k1(B):
             st.close()
 
 
-def test_determinism_replay():
-    seed = synth.config_seed(0) + 7
+@pytest.mark.parametrize("B", [1, 2, 4, 16])
+def test_determinism_replay(B):
+    """Replays give the same bits on every kernel path: the fused kernel (its o_proj units
+    taken from a counter in a different order every launch; at d = 256 all of them are), the
+    small-batch kernels for two and four tokens, and the large-batch kernels."""
+    seed = synth.config_seed(0) + 7 + B
     st = H.GpuStack(seed, synth.TINY, max_batch=16)
     try:
-        case = build_case(seed, synth.TINY, 16)
+        case = build_case(seed, synth.TINY, B)
         o1, i1, g1 = st.step(case["attn"], case["resid"])
         o2, i2, g2 = st.step(case["attn"], case["resid"], reps=3)
         assert np.array_equal(o1, o2) and np.array_equal(i1, i2) and np.array_equal(g1, g2)
@@ -225,6 +229,16 @@ def tp16():
     ref = LayerRef(seed, synth.TP16, 0)
     yield seed, st, ref
     st.close()
+
+
+@pytest.mark.slow
+def test_tp16_b1_replay_bits(tp16):
+    """Full-size batch 1: two launches of the fused kernel give the same output bits."""
+    seed, st, ref = tp16
+    case = build_case(seed + 11, synth.TP16, 1, refs=[ref])
+    o1, i1, g1 = st.step(case["attn"], case["resid"])
+    o2, i2, g2 = st.step(case["attn"], case["resid"], reps=2)
+    assert np.array_equal(o1, o2) and np.array_equal(i1, i2) and np.array_equal(g1, g2)
 
 
 @pytest.mark.slow
