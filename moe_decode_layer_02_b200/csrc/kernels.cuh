@@ -58,6 +58,13 @@ struct KTune {
   size_t smem = 0;         // dynamic shared memory bytes
 };
 
+// Batches of 5 to 8 tokens whose union of experts is under half their (token, expert)
+// entries share most experts (draft tokens of one sequence): their expert phase runs as two
+// launches of the four-token kernel, each streaming its half's experts once; otherwise the
+// large-batch gate/up and down kernels run.  Decided on the device from the router's union,
+// the same in every kernel of the step.
+__host__ __device__ inline bool split_chosen(int U, int B, int K) { return 2 * U < B * K; }
+
 struct LayerArgs {
   int B, maxB, d, d_o, E, k, I;
   float eps;
@@ -68,6 +75,10 @@ struct LayerArgs {
   int* user_idx;          // [B][k] or null
   float* user_gate;       // [B][k] or null
   int route_tables;       // the router's last CTA builds the global routing tables
+  int bar_base;           // the expert kernel's grid barrier opens at (bar_base + 1) x grid
+                          // (1 for the second half of a batch split over two launches)
+  int split_B;            // 5 to 8 tokens: the step launches both expert paths and each kernel
+                          // runs only if split_chosen() says its path is the one (0: no choice)
   // Next layer's weights for the router kernel's L2 prefetch (null: no prefetch)
   const uint16_t *pf_w_o, *pf_w_r, *pf_gamma;
   int pf_w_o_rows;        // leading rows of each CTA's share of the next W_o to prefetch

@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_gateup_rows(const LayerArgs a)
   pdl_trigger();
 
   const int U = min(ld_act_i(a.ws.n_union), E);
+  if (a.split_B && split_chosen(U, a.split_B, a.k)) return;  // the four-token kernels take this step
   long long q0l, q1l;
   split_range((long long)U * I, G, c, q0l, q1l);
   const int q0 = (int)q0l, q1 = (int)q1l;
@@ -310,6 +311,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_down_rows(const LayerArgs a) {
   pdl_wait();  // routing tables, gates and a come from earlier kernels
   pdl_trigger();
   const int U = min(ld_act_i(a.ws.n_union), E);
+  if (a.split_B && split_chosen(U, a.split_B, a.k)) return;  // the four-token kernels take this step
 
   if (warp == kCW) {
     if (lane == 0 && nrows > 0) {

@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
     __syncwarp();
   } else {
     pdl_wait();  // h and the sums of h^2 come from the o_proj kernel
+    if (c == 0 && threadIdx.x == 0) a.ws.counters[kCntGateUp] = 0;  // the expert kernels' grid barrier count
     for (int t = warp; t < B; t += kCW) {
       const float r = rk_rstd(a, t, G, lane);
       if (lane == 0) {

@@ -429,6 +429,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_big(const LayerArgs a) 
       unpack8f(u, gam[j]);
     }
     pdl_wait();  // the sums of h^2 come from the o_proj kernel
+    if (c == 0 && tid == 0) a.ws.counters[kCntGateUp] = 0;  // the expert kernels' grid barrier count
     for (int t = warp; t < B; t += kCW) {  // fixed order: same bits in every CTA
       float ss = 0.f;
       for (int c0 = 0; c0 < G; c0 += 8 * 32) {
@@ -718,6 +719,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
   }
   pdl_wait();  // logits and x come from the router kernel
   pdl_trigger();
+  // one half of a 5-to-8-token step: runs only if the router's union says the halves take it
+  if (a.split_B && !split_chosen(min(ld_act_i(a.ws.n_union), a.E), a.split_B, a.k)) return;
 
   // barriers inside also publish the ring init
   route_small_cta<NT>(a.ws.logits, B, a.E, a.k, a.user_idx, a.user_gate, a.ws.err, rt, sc, fb, c == 0);
@@ -847,7 +850,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_experts_f(const LayerArgs a) {
     }
   }
 
-  grid_barrier(&a.ws.counters[kCntGateUp], gridDim.x, abort_flag, a.ws.err);
+  grid_barrier(&a.ws.counters[kCntGateUp], (unsigned)(a.bar_base + 1) * gridDim.x, abort_flag, a.ws.err);
 
   // ---- phase B (consumers) ------------------------------------------------------------
   // Up to two tokens a_s[u][t][:] = gate * a of (union expert u, token t), zero where t did

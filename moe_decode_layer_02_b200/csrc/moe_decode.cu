@@ -134,7 +134,28 @@ struct Variant {
   bool experts_small; // small-M gate/up and down with per-CTA routing (batch <= 4)
   bool layer2;        // the batch <= 2 layer kernel with per-expert counters (one launch)
   bool fused;         // the three batch <= 2 kernels as one launch with three grid barriers
+  bool split;         // batch 5 to 8: the large-batch o_proj and router, then both expert
+                      // paths, of which the kernels run only the one split_chosen() picks on
+                      // the device: gate/up and down, or the small-M expert kernel once per
+                      // half of the batch (at most four tokens each)
 };
+
+// The arguments of the expert kernel for tokens [t0, t0 + nt) of a step (pointers offset to
+// them; the routing is recomputed from their logits), its grid barrier the half-th of the step.
+LayerArgs half_args(const LayerArgs& a, int t0, int nt, int half) {
+  LayerArgs ah = a;
+  ah.B = nt;
+  ah.ws.logits = a.ws.logits + (size_t)t0 * a.E;
+  ah.ws.x = a.ws.x + (size_t)t0 * a.d;
+  ah.ws.h = a.ws.h + (size_t)t0 * a.d;
+  ah.out = a.out + (size_t)t0 * a.d;
+  ah.user_idx = a.user_idx ? a.user_idx + (size_t)t0 * a.k : nullptr;
+  ah.user_gate = a.user_gate ? a.user_gate + (size_t)t0 * a.k : nullptr;
+  ah.route_tables = 0;
+  ah.bar_base = half;
+  ah.split_B = a.B;
+  return ah;
+}
 
 Variant variant_of(const moe_decode_handle* h, const LayerArgs& a) {
   Variant v;
@@ -145,6 +166,16 @@ Variant variant_of(const moe_decode_handle* h, const LayerArgs& a) {
   // Where the counter-based kernel does not fit: one fused launch at batch 1; at batch 2 the
   // three kernels were measured ahead of that fused launch, so they stay.
   v.fused = !v.layer2 && by_batch && v.oproj_small && a.B == 1 && layer_fused_ok(a, h->smem_optin);
+  // Five to eight tokens: both expert paths are launched and the kernels choose on the device
+  // (split_chosen): tokens sharing most experts run as two launches of the four-token kernel
+  // (each streams its half's experts once), where the large-batch gate/up and down kernels
+  // run well below the HBM rate with one or two tokens per expert.
+  v.split = false;
+  if (!v.experts_small && h->cfg.force_variant == 0 && a.B > 4 && a.B <= 8) {
+    LayerArgs ah = a;
+    ah.B = 4;
+    v.split = small_path_ok(ah, h->smem_optin);
+  }
   return v;
 }
 
@@ -207,6 +238,16 @@ int record_step(moe_decode_handle* h, int B, const void* attn, const void* resid
     if (v.experts_small) {
       if (e == cudaSuccess) e = launch_experts_s(a, G, h->cap, true, h->smem_optin);
       kernels += 1;
+    } else if (v.split) {
+      LayerArgs al = a;
+      al.split_B = B;
+      if (e == cudaSuccess) e = launch_gateup_rows(al, G, h->cap, true, h->smem_optin);
+      if (e == cudaSuccess) e = launch_down_rows(al, G, h->cap, true, h->smem_optin);
+      kernels += 2;
+      for (int t0 = 0, half = 0; t0 < B; t0 += 4, ++half) {
+        if (e == cudaSuccess) e = launch_experts_s(half_args(a, t0, std::min(4, B - t0), half), G, h->cap, true, h->smem_optin);
+        kernels += 1;
+      }
     } else {
       if (e == cudaSuccess) e = launch_gateup_rows(a, G, h->cap, true, h->smem_optin);
       if (e == cudaSuccess) e = launch_down_rows(a, G, h->cap, true, h->smem_optin);
@@ -552,7 +593,7 @@ int moe_decode_kernels_per_step(moe_decode_handle* h, int batch) {
   a.B = batch;
   plan_layer(a, h->num_sms, h->smem_optin);
   const Variant v = variant_of(h, a);
-  const int per_layer = (v.layer2 || v.fused) ? 1 : v.experts_small ? 3 : 4;
+  const int per_layer = (v.layer2 || v.fused) ? 1 : v.experts_small ? 3 : v.split ? 4 + (batch + 3) / 4 : 4;
   return per_layer * L;
 }
 
@@ -602,6 +643,15 @@ int moe_decode_profile_step(moe_decode_handle* h, int batch, const void* attn_ou
     });
     if (v.experts_small) {
       timed(3, s, [&](cudaStream_t st) { return launch_experts_s(a, G, st, false, h->smem_optin); });
+    } else if (v.split) {
+      LayerArgs al = a;
+      al.split_B = batch;
+      timed(4, s, [&](cudaStream_t st) { return launch_gateup_rows(al, G, st, false, h->smem_optin); });
+      timed(5, s, [&](cudaStream_t st) { return launch_down_rows(al, G, st, false, h->smem_optin); });
+      for (int t0 = 0, half = 0; t0 < batch; t0 += 4, ++half)
+        timed(3, s, [&](cudaStream_t st) {
+          return launch_experts_s(half_args(a, t0, std::min(4, batch - t0), half), G, st, false, h->smem_optin);
+        });
     } else {
       timed(4, s, [&](cudaStream_t st) { return launch_gateup_rows(a, G, st, false, h->smem_optin); });
       timed(5, s, [&](cudaStream_t st) { return launch_down_rows(a, G, st, false, h->smem_optin); });
