@@ -281,6 +281,19 @@ def test_tp16_speculative_shapes(tp16, B):
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("B", [5, 6])
+def test_tp16_speculative_split_halves(tp16, B):
+    """5 or 6 draft tokens sharing 12 experts: the expert phase runs as a four-token launch
+    and a one- or two-token launch (the union, 12 + 4 B experts, is under half the 16 B
+    entries); every token is checked."""
+    seed, st, ref = tp16
+    attn0, resid0, _ = H.constructed_shared(seed, synth.TP16, B, core=12, ref=ref)
+    case = build_case(seed, synth.TP16, B, attn0=attn0, resid0=resid0, refs=[ref])
+    out, idx, gate, _ = check_case(st, case)
+    assert len(set(idx[0].ravel().tolist())) == 12 + B * (synth.TP16.k - 12)
+
+
+@pytest.mark.slow
 def test_tp16_speculative_max_batch_4(tp16):
     """The speculative shape on a handle whose max_batch is the batch (4), as a verifier that
     sizes its handle exactly would create it."""
