@@ -7,7 +7,8 @@
 //   1. the producer brings W_r[:, x0 .. x0 + 64) with x0 = r0 rounded down to 8 (a 2-D tensor
 //      map, boxes of 224 experts x 64 columns, 128-byte swizzle; columns outside [r0, r1) meet
 //      zeros below), issued before the dependency wait since W_r is static;
-//   2. consumers compute rstd of every token (the same fixed-order sum as every other kernel),
+//   2. consumers stage the o_proj CTAs' sums of h^2 in shared memory (one coalesced pass) and
+//      compute rstd of every token from them (the same fixed-order sum as every other kernel),
 //      write x for their slice, and place h * gamma of the slice, split into three bf16 terms
 //      hi + mid + lo (together within 2^-26 of the fp32 value; two terms leave 2^-18, which
 //      over d = 8192 columns moves a logit by ~1e-5), in three swizzled tiles;
@@ -47,23 +48,51 @@ constexpr int kRkTileBytes = kRkTok * 128;   // one h tile (hi or lo)
 
 __host__ __device__ inline int rk_boxes(int E) { return (E + kRkBox - 1) / kRkBox; }
 
-// Shared memory: W_r boxes (also the routing-table scratch of the last CTA), h tiles, rstd.
-__host__ __device__ inline size_t rk_smem(int E) {
+constexpr int kRkSsStride = kRkTok + 1;  // floats per staged row of h^2 sums (odd: no bank conflicts)
+constexpr int kRkItems = (kRkTok * 64 + kCT - 1) / kCT;  // h-tile items per consumer thread
+
+// Shared memory: W_r boxes (also the routing-table scratch of the last CTA), h tiles, the
+// staged sums of h^2 of G CTAs, rstd.
+__host__ __device__ inline size_t rk_ss_bytes(int G) { return ((size_t)G * kRkSsStride * 4 + 15) & ~size_t(15); }
+__host__ __device__ inline size_t rk_smem(int E, int G) {
   size_t w = (size_t)rk_boxes(E) * kRkBoxBytes;
   if (w < (size_t)kTopkScratch) w = kTopkScratch;
   w = (w + 1023) & ~size_t(1023);
-  return 1024 + w + 3 * kRkTileBytes + 64 * 4 + 64;
+  return 1024 + w + 3 * kRkTileBytes + rk_ss_bytes(G) + 64 * 4 + 64;
 }
 
-// Fixed-order RMS statistics (the same sum as the other router kernels).
-__device__ __forceinline__ float rk_rstd(const LayerArgs& a, int t, int G, int lane) {
+// The o_proj CTAs' sums of h^2 ([G][maxB] in global memory) of the B tokens, copied into
+// shared memory rows of kRkSsStride floats by the consumer threads: consecutive threads take
+// consecutive tokens of a row, and each thread has eight loads in flight at a time (sixteen
+// or 24 were slower).  (Read straight from L2, one token per warp and round, every CTA asked
+// for the same 148 lines once per token, and a round took about 2.5 us.)
+constexpr int kRkSsRound = 8;
+__device__ __forceinline__ void rk_stage_ss(const LayerArgs& a, float* s_ss, int G, int B, int tid) {
+  const int n = G * B;
+  for (int z0 = tid; z0 < n; z0 += kRkSsRound * kCT) {
+    float v[kRkSsRound];
+#pragma unroll
+    for (int k = 0; k < kRkSsRound; ++k) {
+      const int z = z0 + k * kCT;
+      v[k] = z < n ? ld_act(&a.ws.ss_part[(size_t)(z / B) * a.maxB + z % B]) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kRkSsRound; ++k) {
+      const int z = z0 + k * kCT;
+      if (z < n) s_ss[(z / B) * kRkSsStride + z % B] = v[k];
+    }
+  }
+}
+
+// Fixed-order RMS statistics (the same sum as the other router kernels), from the staged sums.
+__device__ __forceinline__ float rk_rstd(const LayerArgs& a, const float* s_ss, int t, int G, int lane) {
   float ss = 0.f;
   for (int c0 = 0; c0 < G; c0 += 8 * 32) {
     float pv[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const int cc = c0 + k * 32 + lane;
-      pv[k] = cc < G ? ld_act(&a.ws.ss_part[(size_t)cc * a.maxB + t]) : 0.f;
+      pv[k] = cc < G ? s_ss[cc * kRkSsStride + t] : 0.f;
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) ss += pv[k];
@@ -110,7 +139,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
   unsigned char* th = smem + wbytes;       // h * gamma, bf16 hi  [64 tokens][64 columns], swizzled
   unsigned char* tm = th + kRkTileBytes;   // bf16 mid
   unsigned char* tl = tm + kRkTileBytes;   // bf16 lo
-  float* rstd_s = reinterpret_cast<float*>(tl + kRkTileBytes);
+  float* s_ss = reinterpret_cast<float*>(tl + kRkTileBytes);  // [G][kRkSsStride] sums of h^2
+  float* rstd_s = reinterpret_cast<float*>(tl + kRkTileBytes + rk_ss_bytes(G));
   uint64_t* bar = reinterpret_cast<uint64_t*>(rstd_s + 64);
   int* s_misc = reinterpret_cast<int*>(bar + 1);
   volatile int* abort_flag = s_misc;
@@ -137,8 +167,17 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
   } else {
     pdl_wait();  // h and the sums of h^2 come from the o_proj kernel
     if (c == 0 && threadIdx.x == 0) a.ws.counters[kCntGateUp] = 0;  // the expert kernels' grid barrier count
+    // h of this thread's items of the slice, in flight while the sums of h^2 are staged
+    float hv[kRkItems];
+#pragma unroll
+    for (int n = 0; n < kRkItems; ++n) {
+      const int z = tid + n * kCT, t = z >> 6, i = x0 + (z & 63);
+      hv[n] = (z < kRkTok * 64 && t < B && i >= r0 && i < r0 + rows) ? ld_act(&a.ws.h[(size_t)t * d + i]) : 0.f;
+    }
+    rk_stage_ss(a, s_ss, G, B, tid);
+    csync();
     for (int t = warp; t < B; t += kCW) {
-      const float r = rk_rstd(a, t, G, lane);
+      const float r = rk_rstd(a, s_ss, t, G, lane);
       if (lane == 0) {
         rstd_s[t] = r;
         if (c == 0) a.ws.rstd[t] = r;
@@ -146,14 +185,16 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
     }
     csync();
     // x of this CTA's slice, and the slice's h * gamma as bf16 hi + lo tiles (zeros outside)
-    for (int z = tid; z < kRkTok * 64; z += kCT) {
+#pragma unroll
+    for (int n = 0; n < kRkItems; ++n) {
+      const int z = tid + n * kCT;
+      if (z >= kRkTok * 64) break;
       const int t = z >> 6, k = z & 63, i = x0 + k;
       float v = 0.f;
       if (t < B && i >= r0 && i < r0 + rows) {
-        const float hv = ld_act(&a.ws.h[(size_t)t * d + i]);
         const float g = bf16f(a.gamma[i]);
-        v = hv * g;
-        a.ws.x[(size_t)t * d + i] = hv * rstd_s[t] * g;
+        v = hv[n] * g;
+        a.ws.x[(size_t)t * d + i] = hv[n] * rstd_s[t] * g;
       }
       const __nv_bfloat16 vh = __float2bfloat16_rn(v);
       const float r1 = v - __bfloat162float(vh);
@@ -288,7 +329,7 @@ __global__ void __launch_bounds__(kThreadsS, 1) k_router_ks(const __grid_constan
 bool router_ks_ok(const LayerArgs& a, int grid, size_t optin) {
   CUtensorMap probe;
   return a.B >= 1 && a.B <= kRkTok && a.E <= 1024 && a.k <= 32 && (a.d + grid - 1) / grid <= 57 &&
-         rk_smem(a.E) <= optin - 1024 && a.ws.rpart != nullptr &&
+         rk_smem(a.E, grid) <= optin - 1024 && a.ws.rpart != nullptr &&
          make_map_2d(&probe, a.w_r ? a.w_r : reinterpret_cast<const uint16_t*>(256), (uint64_t)a.d, (uint64_t)a.E,
                      64, kRkBox);
 }
@@ -305,7 +346,7 @@ cudaError_t launch_router_ks(const LayerArgs& a, int grid, cudaStream_t s, bool 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreadsS);
-  cfg.dynamicSmemBytes = rk_smem(a.E);
+  cfg.dynamicSmemBytes = rk_smem(a.E, grid);
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   int n = 0;
